@@ -1,0 +1,390 @@
+"""Benchmark of the DiG GLA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Workload (N=1): DiG-XL/2 at 1792 resolution -- B=2, H=16, a 112x112 token grid
+(T=12544), dk=dv=72, bf16 q/k/v, fp32 log_alpha with g ~ N(0,1).  One step is one
+pass of the whole path over the four-direction cycle: for layer l = 0..3,
+gla_fwd(dir = l) -> dwconv3x3 on the output viewed as the [B,112,112,1152] grid
+-> srem_reorient into the next layer's scan order (dir = (l+1) % 4).  Each layer
+has its own seeded inputs (347 MB, larger than the 126 MB L2), so no L2 flush is
+needed between iterations.
+
+The metric is token-heads per second (B*T*H per layer) over the whole step;
+`roofline` reports the GLA forward (the dominant op) against measured HBM
+bandwidth; `cpu_baseline` times the fp64 CPU oracle on a bounded sample of the
+same workload.  Under torchrun (N > 1) every rank runs its own replica of the
+workload (no data exchange: heads and batches are independent), and rank 0
+prints the aggregate.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "GLA fwd tokens·heads/s and % of roofline at T=12544, dk=dv=72, bf16"
+UNIT = "tokens·heads/s"
+WORKLOAD = workloads.WORKLOADS["c4"]
+LAYERS = 4
+# Algorithmic bytes of one GLA forward per token-head: q, k, v (bf16) + log_alpha
+# (fp32) read once, out (bf16) written once.
+GLA_BYTES_PER_TOKEN_HEAD = 2 * (2 * WORKLOAD.dk + WORKLOAD.dv) + 4 * WORKLOAD.dk + 2 * WORKLOAD.dv
+GLA_FLOP_PER_TOKEN_HEAD = 65 * (WORKLOAD.dk + WORKLOAD.dv) + 4 * WORKLOAD.dk * WORKLOAD.dv
+FALLBACK_HBM_GBS = 6650.0
+
+
+def config_dict(extra=None):
+    w = WORKLOAD
+    d = {"workload": w.name, "B": w.B, "H": w.H, "grid": f"{w.Hgrid}x{w.Wgrid}", "T": w.T, "dk": w.dk, "dv": w.dv,
+         "layers_per_step": LAYERS, "dirs": "layer % 4", "conv_channels": w.C,
+         "step": "4 x (gla_fwd + dwconv3x3 + srem_reorient)", "qkv_scale": "1/sqrt(72)",
+         "log_alpha": "logsigmoid(g)/16, g~N(0,1)", "l2": "inputs larger than L2 (347 MB per layer), no flush"}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_linear_attention_chunkwise_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per GLA forward from the committed ncu summary, if it was taken
+    on the current kernel sources; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "gla_fwd_c4_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except OSError:
+        return None
+    if rec.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_gla_fwd")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if bits & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- CPU oracle timing
+def oracle_sample(seconds_target: float = 12.0):
+    """Times the fp64 oracle on a bounded sample of the workload: whole heads of the
+    GLA scan (all four directions) plus the matching conv channels.  Returns
+    (token_heads, seconds, threads, description)."""
+    import oracle
+    w = WORKLOAD
+    cores = oracle.hardware_threads()
+    q, k, v, la = (t.double().numpy() for t in workloads.gla_inputs(w, seed=0))  # widened once
+    conv_w = workloads.conv_weight(w.C, seed=0).double().numpy()
+    # probe: one head, one direction, one thread
+    t0 = time.perf_counter()
+    oracle.gla_fwd(q, k, v, la, w.Hgrid, w.Wgrid, 0, nthreads=1, heads=(0, 1))
+    per_head = time.perf_counter() - t0
+    nh = max(1, min(w.B * w.H, int(seconds_target * cores / (LAYERS * per_head * 1.1))))
+    nh = min(w.B * w.H, max(nh, min(cores, w.B * w.H)))
+    t0 = time.perf_counter()
+    threads = 1
+    for layer in range(LAYERS):
+        out, threads = oracle.gla_fwd(q, k, v, la, w.Hgrid, w.Wgrid, layer, nthreads=cores, heads=(0, nh),
+                                      return_threads=True)
+        # conv over the channels of the sampled heads of batch 0 (whole grid)
+        hb = min(nh, w.H)
+        grid = out[:1, :, :hb, :].reshape(1, w.Hgrid, w.Wgrid, hb * w.dv)
+        oracle.dwconv3x3(grid, conv_w[: hb * w.dv], nthreads=cores)
+        oracle.reorient(grid.reshape(1, w.T, hb * w.dv), (layer + 1) % 4, 0, w.Hgrid, w.Wgrid)
+    secs = time.perf_counter() - t0
+    desc = (f"fp64 C oracle on heads 0..{nh - 1} of {w.B * w.H} (whole 12544-token scans) x 4 directions, "
+            f"plus dwconv3x3 + reorient on the sampled heads' channels")
+    return nh * w.T * LAYERS, secs, threads, desc
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    w = WORKLOAD
+    cores = oracle.hardware_threads()
+    q, k, v, la = (t.double().numpy() for t in workloads.gla_inputs(w, seed=0))  # widened once
+    conv_w = workloads.conv_weight(w.C, seed=0).double().numpy()
+    nh = min(w.B * w.H, cores)
+
+    def step():
+        for layer in range(LAYERS):
+            out = oracle.gla_fwd(q, k, v, la, w.Hgrid, w.Wgrid, layer, nthreads=cores, heads=(0, nh))
+            hb = min(nh, w.H)
+            grid = out[:1, :, :hb, :].reshape(1, w.Hgrid, w.Wgrid, hb * w.dv)
+            oracle.dwconv3x3(grid, conv_w[: hb * w.dv], nthreads=cores)
+            oracle.reorient(grid.reshape(1, w.T, hb * w.dv), (layer + 1) % 4, 0, w.Hgrid, w.Wgrid)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    secs = time.perf_counter() - t0
+    th_per_step = nh * w.T * LAYERS
+    value = th_per_step * args.steps / secs
+    desc = f"fp64 C oracle, heads 0..{nh - 1} of {w.B * w.H} per step, 4 directions, conv + reorient on their channels"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict({"sample": desc}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import torch.distributed as dist
+
+    import gated_linear_attention_chunkwise_b200 as dig
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = WORKLOAD
+
+    # Inputs: one seeded set per layer, generated on the host, resident in HBM.
+    host = [workloads.gla_inputs(w, seed=layer + 97 * rank) for layer in range(LAYERS)]
+    dev_in = [[t.to(dev) for t in layer] for layer in host]
+    conv_w = workloads.conv_weight(w.C, seed=rank).to(dev)
+    outs = [torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
+    convs = [torch.empty((w.B, w.Hgrid, w.Wgrid, w.C), dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
+    reor = [torch.empty((w.B, w.T, w.C), dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
+    stream = torch.cuda.current_stream(dev)
+    launches_per_layer = 3 + 1 + 1  # gla_fwd (chunk state, prefix, output) + dwconv3x3 + srem_reorient
+
+    def layer(l, ev=None):
+        q, k, v, la = dev_in[l]
+        if ev is not None:
+            ev[0].record(stream)
+        dig.gla_fwd(q, k, v, la, w.Hgrid, w.Wgrid, l % 4, out=outs[l])
+        if ev is not None:
+            ev[1].record(stream)
+        dig.dwconv3x3(outs[l].view(w.B, w.Hgrid, w.Wgrid, w.C), conv_w, out=convs[l])
+        if ev is not None:
+            ev[2].record(stream)
+        dig.srem_reorient(convs[l].view(w.B, w.T, w.C), (l + 1) % 4, 0, w.Hgrid, w.Wgrid, out=reor[l])
+        if ev is not None:
+            ev[3].record(stream)
+
+    def step(evs=None):
+        for l in range(LAYERS):
+            layer(l, None if evs is None else evs[l])
+
+    for _ in range(args.warmup):
+        step()
+    status = dig.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {dig.status_string(status)}")
+
+    # Timed region: exactly K steps, per-op events inside.
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(LAYERS)]
+           for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(stop)
+    gla_ms = [e[l][0].elapsed_time(e[l][1]) for e in evs for l in range(LAYERS)]
+    conv_ms = [e[l][1].elapsed_time(e[l][2]) for e in evs for l in range(LAYERS)]
+    reor_ms = [e[l][2].elapsed_time(e[l][3]) for e in evs for l in range(LAYERS)]
+    status = dig.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {dig.status_string(status)}")
+
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    th_per_step = w.token_heads * LAYERS
+    value = th_per_step * args.steps * world / (max_ms / 1e3)
+
+    # End to end through the public API: pinned host inputs -> device -> path -> host result.
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    pinned = [[t.pin_memory() for t in layer] for layer in host]
+    host_out = [torch.empty((w.B, w.T, w.C), dtype=torch.bfloat16).pin_memory() for _ in range(LAYERS)]
+    h2d = sum(t.numel() * t.element_size() for layer in pinned for t in layer)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def e2e_step():
+        for l in range(LAYERS):
+            for dst, src in zip(dev_in[l], pinned[l]):
+                dst.copy_(src, non_blocking=True)
+        step()
+        for l in range(LAYERS):
+            host_out[l].copy_(reor[l], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = th_per_step * e2e_steps * world / (float(te.item()) / 1e3)
+
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    gla_avg_s = statistics.mean(gla_ms) / 1e3
+    gla_bytes = GLA_BYTES_PER_TOKEN_HEAD * w.token_heads
+    achieved = gla_bytes / gla_avg_s / 1e9
+    traffic = recorded_traffic()
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            th, secs, threads, desc = oracle_sample(args.cpu_seconds)
+            cpu = {"value": th / secs, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+                   "seconds": secs}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_dict({"parallelism": f"replicas x{world}" if world > 1 else "single GPU"}),
+            "roofline": {
+                "bound": "hbm", "kernel": "gla_fwd (chunk state + prefix + output)",
+                "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "peak_source": f"{peak_kind} hbm_gbs", "traffic": traffic,
+                "algorithmic_bytes_per_launch": gla_bytes, "avg_launch_us": gla_avg_s * 1e6,
+            },
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
+            "gpu_launches": launches_per_layer * LAYERS * args.steps,
+            "clocks": clk.summary(),
+            "breakdown_us_per_layer": {"gla_fwd": statistics.mean(gla_ms) * 1e3,
+                                       "dwconv3x3": statistics.mean(conv_ms) * 1e3,
+                                       "srem_reorient": statistics.mean(reor_ms) * 1e3},
+            "gla_only": {"tokens_heads_per_s": w.token_heads / gla_avg_s,
+                         "tflops": GLA_FLOP_PER_TOKEN_HEAD * w.token_heads / gla_avg_s / 1e12},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

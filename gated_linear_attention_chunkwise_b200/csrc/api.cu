@@ -1,0 +1,202 @@
+// api.cu -- the extern "C" entry points declared in include/dig_gla.h.
+//
+// Each entry point validates its arguments on the host (returning a status code
+// before anything is enqueued), checks that the current device is an sm_100
+// part, and enqueues the kernels on the caller's stream.  Scratch memory for the
+// GLA passes comes from the stream-ordered allocator and is released on the same
+// stream, so calls never synchronise.
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "dev_common.cuh"
+#include "dig_gla.h"
+#include "internal.h"
+
+namespace dig {
+
+namespace {
+
+std::mutex g_mu;
+int g_arch_ok[64];  // per device: 0 unknown, 1 sm_100, -1 other
+
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GLA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return GLA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_arch_ok[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return GLA_ERR_CUDA;
+    g_arch_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return g_arch_ok[dev] == 1 ? GLA_OK : GLA_ERR_UNSUPPORTED;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+int validate_gla(const void* q, const void* k, const void* v, const void* la, const void* out, int B, int H,
+                 int Hg, int Wg, int dk, int dv, int dir, size_t elt) {
+  if (!q || !k || !v || !la || !out) return GLA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Hg <= 0 || Wg <= 0 || dk <= 0 || dv <= 0) return GLA_ERR_INVALID_ARG;
+  if (dir < 0 || dir > 3) return GLA_ERR_INVALID_ARG;
+  if (dk % 8 || dv % 8 || dk > 128 || dv > 128) return GLA_ERR_UNSUPPORTED;
+  const int64_t T = (int64_t)Hg * Wg;
+  if (T > (int64_t)1 << 30) return GLA_ERR_UNSUPPORTED;
+  if ((int64_t)B * H > 65535) return GLA_ERR_UNSUPPORTED;
+  const int64_t rows = (int64_t)B * T * H;
+  if (rows > ((int64_t)1 << 40) / 128) return GLA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(la) || !aligned16(out))
+    return GLA_ERR_ALIGNMENT;
+  const size_t nq = (size_t)rows * dk * elt, nv = (size_t)rows * dv * elt, nl = (size_t)rows * dk * 4;
+  const size_t no = (size_t)rows * dv * elt;
+  if (overlaps(out, no, q, nq) || overlaps(out, no, k, nq) || overlaps(out, no, v, nv) || overlaps(out, no, la, nl))
+    return GLA_ERR_INVALID_ARG;
+  return GLA_OK;
+}
+
+int validate_grid(const void* x, const void* y, int B, int Hg, int Wg, int C, int dtype, size_t* row_bytes) {
+  if (!x || !y) return GLA_ERR_INVALID_ARG;
+  if (B <= 0 || Hg <= 0 || Wg <= 0 || C <= 0) return GLA_ERR_INVALID_ARG;
+  if (dtype != GLA_BF16 && dtype != GLA_F32) return GLA_ERR_INVALID_ARG;
+  const size_t elt = dtype == GLA_BF16 ? 2 : 4;
+  const size_t rb = (size_t)C * elt;
+  if (rb % 16) return GLA_ERR_ALIGNMENT;
+  if (!aligned16(x) || !aligned16(y)) return GLA_ERR_ALIGNMENT;
+  const int64_t T = (int64_t)Hg * Wg;
+  if (T > (int64_t)1 << 30 || (int64_t)B * T > ((int64_t)1 << 40) / (int64_t)rb) return GLA_ERR_UNSUPPORTED;
+  if ((int64_t)B * ((Hg + 15) / 16) > 65535 || (Wg + 3) / 4 > 65535) return GLA_ERR_UNSUPPORTED;
+  const size_t n = (size_t)B * T * rb;
+  if (overlaps(x, n, y, n)) return GLA_ERR_INVALID_ARG;
+  *row_bytes = rb;
+  return GLA_OK;
+}
+
+int run_with_workspace(size_t bytes, cudaStream_t st, cudaError_t (*fn)(void*, void*), void* ctx) {
+  void* ws = nullptr;
+  if (bytes) {
+    if (cudaMallocAsync(&ws, bytes, st) != cudaSuccess) {
+      cudaGetLastError();
+      return GLA_ERR_NOMEM;
+    }
+  }
+  const cudaError_t e = fn(ws, ctx);
+  if (ws) cudaFreeAsync(ws, st);
+  return e == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+}
+
+}  // namespace
+
+cudaError_t read_and_clear_device_status(int* status, cudaStream_t st) {
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return e;
+  int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int));
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return e;
+  *status = v;
+  return cudaSuccess;
+}
+
+}  // namespace dig
+
+using dig::GlaShape;
+
+namespace {
+struct GlaCall {
+  const void *q, *k, *v;
+  const float* la;
+  void* out;
+  GlaShape s;
+  cudaStream_t st;
+};
+cudaError_t run_tc(void* ws, void* ctx) {
+  const GlaCall* c = static_cast<const GlaCall*>(ctx);
+  return dig::gla_tc_forward(c->q, c->k, c->v, c->la, c->out, c->s, ws, c->st);
+}
+cudaError_t run_f32(void* ws, void* ctx) {
+  const GlaCall* c = static_cast<const GlaCall*>(ctx);
+  return dig::gla_f32_forward(static_cast<const float*>(c->q), static_cast<const float*>(c->k),
+                              static_cast<const float*>(c->v), c->la, static_cast<float*>(c->out), c->s, ws, c->st);
+}
+}  // namespace
+
+extern "C" {
+
+int gla_fwd(const void* q, const void* k, const void* v, const float* log_alpha, int B, int H, int Hgrid, int Wgrid,
+            int dk, int dv, int dir, void* out, cudaStream_t stream) {
+  int rc = dig::validate_gla(q, k, v, log_alpha, out, B, H, Hgrid, Wgrid, dk, dv, dir, 2);
+  if (rc != GLA_OK) return rc;
+  if ((rc = dig::check_device()) != GLA_OK) return rc;
+  GlaCall c{q, k, v, log_alpha, out, GlaShape{B, H, Hgrid, Wgrid, dk, dv, dir}, stream};
+  return dig::run_with_workspace(dig::gla_tc_workspace_bytes(c.s), stream, run_tc, &c);
+}
+
+int gla_fwd_f32(const float* q, const float* k, const float* v, const float* log_alpha, int B, int H, int Hgrid,
+                int Wgrid, int dk, int dv, int dir, float* out, cudaStream_t stream) {
+  int rc = dig::validate_gla(q, k, v, log_alpha, out, B, H, Hgrid, Wgrid, dk, dv, dir, 4);
+  if (rc != GLA_OK) return rc;
+  if ((rc = dig::check_device()) != GLA_OK) return rc;
+  GlaCall c{q, k, v, log_alpha, out, GlaShape{B, H, Hgrid, Wgrid, dk, dv, dir}, stream};
+  return dig::run_with_workspace(dig::gla_f32_workspace_bytes(c.s), stream, run_f32, &c);
+}
+
+int srem_reorient(const void* x, int dir, int inverse, int B, int Hgrid, int Wgrid, int C, int dtype, void* y,
+                  cudaStream_t stream) {
+  size_t rb = 0;
+  int rc = dig::validate_grid(x, y, B, Hgrid, Wgrid, C, dtype, &rb);
+  if (rc != GLA_OK) return rc;
+  if (dir < 0 || dir > 3 || (inverse != 0 && inverse != 1)) return GLA_ERR_INVALID_ARG;
+  if ((rc = dig::check_device()) != GLA_OK) return rc;
+  return dig::srem_reorient_launch(x, y, dir, inverse, B, Hgrid, Wgrid, rb, stream) == cudaSuccess ? GLA_OK
+                                                                                                   : GLA_ERR_CUDA;
+}
+
+int dwconv3x3(const void* x, const float* w, int B, int Hgrid, int Wgrid, int C, int dtype, void* y,
+              cudaStream_t stream) {
+  size_t rb = 0;
+  int rc = dig::validate_grid(x, y, B, Hgrid, Wgrid, C, dtype, &rb);
+  if (rc != GLA_OK) return rc;
+  if (!w) return GLA_ERR_INVALID_ARG;
+  if (!dig::aligned16(w)) return GLA_ERR_ALIGNMENT;
+  if ((rc = dig::check_device()) != GLA_OK) return rc;
+  return dig::dwconv3x3_launch(x, w, y, B, Hgrid, Wgrid, C, dtype, stream) == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+}
+
+int dig_gla_device_status(cudaStream_t stream) {
+  int rc = dig::check_device();
+  if (rc != GLA_OK) return rc;
+  int v = 0;
+  if (dig::read_and_clear_device_status(&v, stream) != cudaSuccess) return GLA_ERR_CUDA;
+  return v;
+}
+
+const char* dig_gla_status_string(int status) {
+  switch (status) {
+    case GLA_OK: return "GLA_OK";
+    case GLA_ERR_INVALID_ARG: return "GLA_ERR_INVALID_ARG";
+    case GLA_ERR_UNSUPPORTED: return "GLA_ERR_UNSUPPORTED";
+    case GLA_ERR_ALIGNMENT: return "GLA_ERR_ALIGNMENT";
+    case GLA_ERR_CUDA: return "GLA_ERR_CUDA";
+    case GLA_ERR_TIMEOUT: return "GLA_ERR_TIMEOUT";
+    case GLA_ERR_NOMEM: return "GLA_ERR_NOMEM";
+    case GLA_ERR_RANGE: return "GLA_ERR_RANGE";
+    default: return "GLA_ERR_UNKNOWN";
+  }
+}
+
+void dig_gla_release(void) {
+  std::lock_guard<std::mutex> lk(dig::g_mu);
+  memset(dig::g_arch_ok, 0, sizeof(dig::g_arch_ok));
+}
+
+}  // extern "C"

@@ -1,0 +1,274 @@
+// gla_simt.cu -- chunk-wise GLA forward with fp32 q/k/v/out on CUDA cores.
+//
+// Same decomposition as the tensor-core path (gla_tc.cu), with chunks of 64 scan
+// positions and every product in fp32 FMA, so the result carries no bf16/tf32
+// operand rounding:
+//   pass 1  S_loc = K^T V with K^_s = k_s exp(u_s),  gamma = exp(g)
+//   pass 2  G_c = Diag(gamma_c) S_in(c),  S_in(c+1) = G_c + S_loc(c)
+//   pass 3  O = mask(Q~ K^T) V + Q~ G_c with Q~_r = q_r exp(-u_r)
+// (u_r = sum of the log-gates scanned after row r inside the chunk, g the chunk
+// total.)  Chunks whose gates decay by more than e^80 inside the chunk are
+// flagged by pass 1 and evaluated token by token in pass 3 from the exact fp32
+// incoming state, so every log_alpha <= 0 (including -inf) is handled.
+#include <math.h>
+
+#include "dev_common.cuh"
+#include "internal.h"
+
+namespace dig {
+
+namespace {
+
+constexpr int MC = kChunkF32;
+constexpr int NT = 256;
+constexpr float kMaxGateRange = 80.0f;
+
+struct F32Args {
+  const float* q;
+  const float* k;
+  const float* v;
+  const float* la;
+  float* out;
+  float* s_locT;  // [BH][NC][dv][dk]
+  float* gamma;   // [BH][NC][dk]
+  float* GT;      // [BH][NC][dv][dk]  (Diag(gamma) S_in)^T
+  int* flags;     // [BH][NC]  1: evaluate this chunk token by token
+  int H, dk, dv, NC;
+  ScanGeom g;
+};
+
+// Rows f0..f0+MC-1 of head h, batch b of a [B][T][H][d] fp32 tensor into a
+// plain tile with a pitch of d+4 floats; rows outside the sequence are zero.
+__device__ __forceinline__ void stage_rows(float* dst, const float* src, int d, const ScanGeom& g, int f0, int b,
+                                           int h, int H) {
+  const int cpr = d / 4;
+  const int pitch = d + 4;
+  for (int idx = threadIdx.x; idx < MC * cpr; idx += NT) {
+    const int r = idx / cpr;
+    const int cc = idx - r * cpr;
+    const int f = f0 + r;
+    float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (f >= 0 && f < g.T)
+      val = *reinterpret_cast<const float4*>(src + (((int64_t)b * g.T + base_pos_to_token(g, f)) * H + h) * d +
+                                             cc * 4);
+    *reinterpret_cast<float4*>(dst + r * pitch + cc * 4) = val;
+  }
+}
+
+// Threads i < dk: exclusive suffix sums of the log-gate along the scan order, in
+// place; chunk total in sBL[i].  Returns bit 1 if the factorised form would leave
+// fp32 range (use the serial path), bit 2 if the gates grow the state beyond it.
+__device__ __forceinline__ int suffix64(float* sLA, float* sBL, int dk, int reverse) {
+  const int i = threadIdx.x;
+  int code = 0;
+  if (i < dk) {
+    const int pw = dk + 4;
+    float acc = 0.f, lo = 0.f, hi = 0.f;
+    for (int s = 0; s < MC; ++s) {
+      const int r = reverse ? s : (MC - 1 - s);
+      const float la = sLA[r * pw + i];
+      sLA[r * pw + i] = acc;
+      lo = fminf(lo, acc);
+      hi = fmaxf(hi, acc);
+      acc += la;
+    }
+    sBL[i] = acc;
+    hi = fmaxf(hi, acc);
+    if (!(lo >= -kMaxGateRange) || !(hi <= kMaxGateRange)) code |= 1;
+    if (!(hi <= kMaxGateRange)) code |= 2;
+  }
+  return code;
+}
+
+__global__ void __launch_bounds__(NT) gla_f32_chunk_state(const F32Args a) {
+  extern __shared__ float4 smem_f4[];
+  float* smem = reinterpret_cast<float*>(smem_f4);
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int pk = a.dk + 4, pv = a.dv + 4;
+  float* sK = smem;
+  float* sV = sK + MC * pk;
+  float* sLA = sV + MC * pv;
+  float* sBL = sLA + MC * pk;
+
+  const int f0 = chunk_first_base_pos(a.g, c, MC);
+  stage_rows(sK, a.k, a.dk, a.g, f0, b, h, a.H);
+  stage_rows(sV, a.v, a.dv, a.g, f0, b, h, a.H);
+  stage_rows(sLA, a.la, a.dk, a.g, f0, b, h, a.H);
+  __syncthreads();
+  const int code = suffix64(sLA, sBL, a.dk, a.g.reverse);
+  if (code & 2) report_status(GLA_ERR_RANGE);
+  const int wide = __syncthreads_or(code != 0);
+  for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
+    const int r = e / a.dk, i = e - r * a.dk;
+    sK[r * pk + i] *= expf(sLA[r * pk + i]);
+  }
+  __syncthreads();
+  const int64_t cid = (int64_t)bh * a.NC + c;
+  for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+    const int j = e / a.dk, i = e - j * a.dk;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int s = 0; s < MC; ++s) acc = fmaf(sK[s * pk + i], sV[s * pv + j], acc);
+    a.s_locT[(cid * a.dv + j) * a.dk + i] = acc;
+  }
+  if (threadIdx.x < a.dk) a.gamma[cid * a.dk + threadIdx.x] = expf(sBL[threadIdx.x]);
+  if (threadIdx.x == 0) a.flags[cid] = wide;
+}
+
+__global__ void __launch_bounds__(256) gla_f32_prefix(const F32Args a) {
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= a.dk * a.dv) return;
+  const int j = e / a.dk, i = e - j * a.dk;
+  float S = 0.f;
+  for (int c = 0; c < a.NC; ++c) {
+    const int64_t cid = (int64_t)bh * a.NC + c;
+    const float G = a.gamma[cid * a.dk + i] * S;
+    const float sl = a.s_locT[(cid * a.dv + j) * a.dk + i];
+    a.GT[(cid * a.dv + j) * a.dk + i] = G;
+    if (a.flags[cid]) a.s_locT[(cid * a.dv + j) * a.dk + i] = S;  // exact S_in for pass 3
+    S = G + sl;
+  }
+}
+
+__global__ void __launch_bounds__(NT) gla_f32_output(const F32Args a) {
+  extern __shared__ float4 smem_f4[];
+  float* smem = reinterpret_cast<float*>(smem_f4);
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int pk = a.dk + 4, pv = a.dv + 4, pa = MC + 1;
+  float* sQ = smem;
+  float* sK = sQ + MC * pk;
+  float* sLA = sK + MC * pk;
+  float* sV = sLA + MC * pk;
+  float* sG = sV + MC * pv;          // [dv][dk+4]: G^T
+  float* sA = sG + a.dv * pk;        // [MC][MC+1]
+  float* sBL = sA + MC * pa;
+
+  const int f0 = chunk_first_base_pos(a.g, c, MC);
+  stage_rows(sQ, a.q, a.dk, a.g, f0, b, h, a.H);
+  stage_rows(sK, a.k, a.dk, a.g, f0, b, h, a.H);
+  stage_rows(sV, a.v, a.dv, a.g, f0, b, h, a.H);
+  stage_rows(sLA, a.la, a.dk, a.g, f0, b, h, a.H);
+  const int64_t cid = (int64_t)bh * a.NC + c;
+  {
+    const float* src = a.GT + cid * a.dv * a.dk;
+    const int cpr = a.dk / 4;
+    for (int idx = threadIdx.x; idx < a.dv * cpr; idx += NT) {
+      const int j = idx / cpr, cc = idx - j * cpr;
+      *reinterpret_cast<float4*>(sG + j * pk + cc * 4) =
+          *reinterpret_cast<const float4*>(src + (int64_t)j * a.dk + cc * 4);
+    }
+  }
+  __syncthreads();
+  if (a.flags[cid]) {
+    // Exact token-by-token recurrence from S_in (left in the S_loc slot by pass 2):
+    // thread j owns value column j of the state sS[dk][dv] (reuses sG and sA).
+    float* sS = sG;
+    const float* src = a.s_locT + cid * a.dv * a.dk;
+    for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+      const int j = e / a.dk, i = e - j * a.dk;
+      sS[i * a.dv + j] = src[e];
+    }
+    for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
+      const int r = e / a.dk, i = e - r * a.dk;
+      sLA[r * pk + i] = expf(sLA[r * pk + i]);
+    }
+    __syncthreads();
+    for (int s = 0; s < MC; ++s) {
+      const int r = a.g.reverse ? (MC - 1 - s) : s;
+      const int f = f0 + r;
+      if (f < 0 || f >= a.g.T) continue;
+      for (int j = threadIdx.x; j < a.dv; j += NT) {
+        const float vj = sV[r * pv + j];
+        float acc = 0.f;
+        for (int i = 0; i < a.dk; ++i) {
+          const float st = fmaf(sLA[r * pk + i], sS[i * a.dv + j], sK[r * pk + i] * vj);
+          sS[i * a.dv + j] = st;
+          acc = fmaf(sQ[r * pk + i], st, acc);
+        }
+        a.out[(((int64_t)b * a.g.T + base_pos_to_token(a.g, f)) * a.H + h) * a.dv + j] = acc;
+      }
+    }
+    return;
+  }
+  suffix64(sLA, sBL, a.dk, a.g.reverse);
+  __syncthreads();
+  for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
+    const int r = e / a.dk, i = e - r * a.dk;
+    const float u = sLA[r * pk + i];
+    sQ[r * pk + i] *= expf(-u);
+    sK[r * pk + i] *= expf(u);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < MC * MC; e += NT) {
+    const int t = e / MC, s = e - t * MC;
+    const bool keep = a.g.reverse ? (s >= t) : (s <= t);
+    float acc = 0.f;
+    if (keep) {
+      for (int i = 0; i < a.dk; ++i) acc = fmaf(sQ[t * pk + i], sK[s * pk + i], acc);
+    }
+    sA[t * pa + s] = acc;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < MC * a.dv; e += NT) {
+    const int t = e / a.dv, j = e - t * a.dv;
+    const int f = f0 + t;
+    if (f < 0 || f >= a.g.T) continue;
+    float acc = 0.f;
+    for (int s = 0; s < MC; ++s) acc = fmaf(sA[t * pa + s], sV[s * pv + j], acc);
+    for (int i = 0; i < a.dk; ++i) acc = fmaf(sQ[t * pk + i], sG[j * pk + i], acc);
+    a.out[(((int64_t)b * a.g.T + base_pos_to_token(a.g, f)) * a.H + h) * a.dv + j] = acc;
+  }
+}
+
+size_t rup(size_t x, size_t m) { return (x + m - 1) / m * m; }
+
+}  // namespace
+
+size_t gla_f32_workspace_bytes(const GlaShape& s) {
+  const size_t NC = (size_t)(s.T() + MC - 1) / MC;
+  const size_t BH = (size_t)s.B * s.H;
+  return rup(BH * NC * s.dv * s.dk * 4, 256) * 2 + rup(BH * NC * s.dk * 4, 256) + rup(BH * NC * 4, 256);
+}
+
+cudaError_t gla_f32_forward(const float* q, const float* k, const float* v, const float* la, float* out,
+                            const GlaShape& s, void* workspace, cudaStream_t st) {
+  F32Args a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.la = la;
+  a.out = out;
+  a.H = s.H;
+  a.dk = s.dk;
+  a.dv = s.dv;
+  a.NC = (s.T() + MC - 1) / MC;
+  a.g = make_geom(s.Hg, s.Wg, s.dir);
+  const size_t BH = (size_t)s.B * s.H;
+  const size_t sl = rup(BH * a.NC * s.dv * s.dk * 4, 256);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.s_locT = reinterpret_cast<float*>(ws);
+  a.GT = reinterpret_cast<float*>(ws + sl);
+  a.gamma = reinterpret_cast<float*>(ws + 2 * sl);
+  a.flags = reinterpret_cast<int*>(ws + 2 * sl + rup(BH * a.NC * s.dk * 4, 256));
+
+  const size_t pk = s.dk + 4, pv = s.dv + 4;
+  const size_t smem_state = (MC * pk * 2 + MC * pv + s.dk) * sizeof(float);
+  const size_t smem_out = (MC * pk * 3 + MC * pv + s.dv * pk + MC * (MC + 1) + s.dk) * sizeof(float);
+  cudaError_t e;
+  e = cudaFuncSetAttribute(gla_f32_chunk_state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_state);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(gla_f32_output, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_out);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(a.NC, s.B * s.H);
+  gla_f32_chunk_state<<<grid, NT, smem_state, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  gla_f32_prefix<<<dim3((s.dk * s.dv + 255) / 256, s.B * s.H), 256, 0, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  gla_f32_output<<<grid, NT, smem_out, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace dig

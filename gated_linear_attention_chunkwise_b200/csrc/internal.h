@@ -1,0 +1,38 @@
+// internal.h -- launchers behind the C ABI (host side, C++).  Every launcher
+// assumes its arguments were validated by api.cu and only enqueues work.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace dig {
+
+// Geometry of one GLA call, shared by the launchers.
+struct GlaShape {
+  int B, H, Hg, Wg, dk, dv, dir;
+  int T() const { return Hg * Wg; }
+};
+
+// ---- bf16 tensor-core path (chunks of 128 scan positions) ----
+constexpr int kChunkTC = 128;
+size_t gla_tc_workspace_bytes(const GlaShape& s);
+cudaError_t gla_tc_forward(const void* q, const void* k, const void* v, const float* la, void* out,
+                           const GlaShape& s, void* workspace, cudaStream_t st);
+
+// ---- fp32 SIMT path (chunks of 64 scan positions) ----
+constexpr int kChunkF32 = 64;
+size_t gla_f32_workspace_bytes(const GlaShape& s);
+cudaError_t gla_f32_forward(const float* q, const float* k, const float* v, const float* la, float* out,
+                            const GlaShape& s, void* workspace, cudaStream_t st);
+
+// ---- SREM ----
+cudaError_t srem_reorient_launch(const void* x, void* y, int dir, int inverse, int B, int Hg, int Wg,
+                                 size_t row_bytes, cudaStream_t st);
+cudaError_t dwconv3x3_launch(const void* x, const float* w, void* y, int B, int Hg, int Wg, int C, int dtype,
+                             cudaStream_t st);
+
+// ---- status word ----
+cudaError_t read_and_clear_device_status(int* status, cudaStream_t st);
+
+}  // namespace dig

@@ -1,0 +1,139 @@
+/*
+ * dig_gla.h -- C ABI of the DiG gated-linear-attention hot path on NVIDIA B200
+ * (sm_100a): the chunk-wise GLA forward over one of the four SREM scan orders,
+ * the SREM reorientation of the token grid, and SREM's 3x3 depthwise conv.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor arguments are DEVICE pointers to dense, contiguous buffers owned
+ *    by the caller.  The library keeps no reference to them after the call.
+ *  - Token grids are Hgrid x Wgrid patches, T = Hgrid*Wgrid, and token t is the
+ *    raster index t = y*Wgrid + x.  Sequence tensors are token-major with heads
+ *    interleaved: q, k, log_alpha are [B][T][H][dk]; v and out are [B][T][H][dv]
+ *    (the layout a fused q/k/v projection writes).  Grid tensors for the conv and
+ *    the reorientation are channels-last [B][Hgrid][Wgrid][C] (== [B][T][C]).
+ *  - Scan directions (DiG paper notes, "空间重定向与增强模块 (SREM)": four scan
+ *    orders -- left-to-right, right-to-left, top-to-bottom, bottom-to-top --
+ *    produced by transposing the 2D token matrix and flipping the sequence),
+ *    numbered in the order the notes list them:
+ *      GLA_DIR_L2R = 0: raster order t = p
+ *      GLA_DIR_R2L = 1: reversed raster order t = T-1-p
+ *      GLA_DIR_T2B = 2: column-major order t = (p mod Hgrid)*Wgrid + p div Hgrid
+ *      GLA_DIR_B2T = 3: reversed column-major order
+ *  - Every call is asynchronous on `stream` (0 = the legacy default stream) and
+ *    never synchronises it.  Argument errors are returned synchronously before
+ *    anything is launched; a launch failure returns GLA_ERR_CUDA.  Conditions a
+ *    kernel detects while running (a bounded wait that expired, growth gates that
+ *    overflow fp32) are recorded in a per-device status word that
+ *    dig_gla_device_status() reads and clears.
+ *  - Pointers must be 16-byte aligned.  There is no CPU fallback: a call on a
+ *    device other than sm_100 returns GLA_ERR_UNSUPPORTED.
+ */
+#ifndef DIG_GLA_H_
+#define DIG_GLA_H_
+
+#include <cuda_runtime_api.h>
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GLA_OK = 0,
+  GLA_ERR_INVALID_ARG = -1, /* null pointer, non-positive size, bad enum, aliasing */
+  GLA_ERR_UNSUPPORTED = -2, /* a size or device this build does not handle */
+  GLA_ERR_ALIGNMENT = -3,   /* a pointer or a row pitch that is not 16-byte aligned */
+  GLA_ERR_CUDA = -4,        /* a CUDA runtime call failed (see cudaGetLastError) */
+  GLA_ERR_TIMEOUT = -5,     /* a kernel gave up a bounded wait (device status only) */
+  GLA_ERR_NOMEM = -6,       /* the stream-ordered workspace could not be allocated */
+  GLA_ERR_RANGE = -7        /* growth gates (log_alpha > 0) overflowed fp32 inside a chunk
+                               (device status only; the output is not valid) */
+} gla_status_t;
+
+enum { GLA_DIR_L2R = 0, GLA_DIR_R2L = 1, GLA_DIR_T2B = 2, GLA_DIR_B2T = 3 };
+enum { GLA_BF16 = 0, GLA_F32 = 1 };
+
+/*
+ * gla_fwd -- chunk-wise gated linear attention forward, bf16 inputs.
+ *
+ * Computes, for every batch b and head h, the recurrence over the scan order of
+ * direction `dir` (DiG: "gated linear attention", S_t = Diag(alpha_t) S_{t-1} +
+ * k_t^T v_t, o_t = q_t S_t; chunk-wise parallel form, DiG paper notes "硬件友好的
+ * 效率设计": the sequence is cut into chunks processed in on-chip memory):
+ *     S_0 = 0 (dk x dv),  alpha_{t,i} = exp(log_alpha[b][t][h][i])
+ *     S  <- Diag(alpha_t) S + k_t^T v_t      (gate per key channel, broadcast over dv)
+ *     out[b][t][h][:] = q_t S                (read after the update)
+ * The output of token t is written at t (canonical position) for every dir.
+ * No feature map, normaliser or 1/sqrt(dk) is applied: pre-scale q, k, v.
+ *
+ *   q, k       [B][T][H][dk] bf16        log_alpha [B][T][H][dk] fp32
+ *   v          [B][T][H][dv] bf16        out       [B][T][H][dv] bf16 (written)
+ *   dk, dv     multiples of 8 in [8, 128]
+ *   dir        GLA_DIR_*
+ * Arithmetic: tensor-core products of bf16 operands with fp32 accumulation; the
+ * chunk state and all gate arithmetic are fp32; out is rounded to nearest even.
+ * Gates: any log_alpha <= 0 is handled, -inf (a full reset of the channel)
+ * included.  Chunks of 128 positions whose gates decay by more than e^80 inside
+ * the chunk are evaluated token by token (exact, slower).  Growth gates
+ * (log_alpha > 0) whose product exceeds e^80 inside a chunk cannot be represented
+ * in fp32: GLA_ERR_RANGE is recorded in the device status.
+ * Workspace: stream-ordered (cudaMallocAsync), freed on the same stream.
+ * `out` must not overlap any input.
+ */
+int gla_fwd(const void* q, const void* k, const void* v, const float* log_alpha, int B, int H, int Hgrid,
+            int Wgrid, int dk, int dv, int dir, void* out, cudaStream_t stream);
+
+/*
+ * gla_fwd_f32 -- the same recurrence with fp32 q, k, v and out (all arithmetic
+ * fp32, no tensor-core rounding).  Same shapes, directions and errors as gla_fwd.
+ */
+int gla_fwd_f32(const float* q, const float* k, const float* v, const float* log_alpha, int B, int H,
+                int Hgrid, int Wgrid, int dk, int dv, int dir, float* out, cudaStream_t stream);
+
+/*
+ * srem_reorient -- SREM's change of scan direction as an explicit row gather
+ * (DiG paper notes, SREM: the block ends by transposing the 2D token matrix and
+ * flipping the sequence, both O(T) operations; DiG Block step (5)).
+ *   inverse = 0:  y[b][p][:] = x[b][order_dir(p)][:]   (canonical -> scan order)
+ *   inverse = 1:  y[b][order_dir(p)][:] = x[b][p][:]   (scan order -> canonical)
+ * where order_dir(p) is the raster token visited at scan position p.
+ *   x, y   [B][T][C] elements of `dtype` (GLA_BF16 or GLA_F32); C*sizeof(elt)
+ *          must be a multiple of 16 bytes.  Bit-exact copy.  y must not overlap x.
+ */
+int srem_reorient(const void* x, int dir, int inverse, int B, int Hgrid, int Wgrid, int C, int dtype, void* y,
+                  cudaStream_t stream);
+
+/*
+ * dwconv3x3 -- SREM's 3x3 depthwise convolution on the 2D token grid (DiG paper
+ * notes, SREM and DiG Block step (4): DWConv2d after reshaping the sequence to
+ * 2D, identity-initialised):
+ *   y[b][r][c][ch] = sum_{i,j in {-1,0,1}} w[ch][i+1][j+1] * x[b][r+i][c+j][ch]
+ * with zero padding outside the grid (cross-correlation, no kernel flip, no bias).
+ *   x, y   [B][Hgrid][Wgrid][C] of `dtype` (GLA_BF16 or GLA_F32), channels-last;
+ *          C*sizeof(elt) must be a multiple of 16 bytes.  y must not overlap x.
+ *   w      [C][3][3] fp32.
+ * Accumulation is fp32; a bf16 result is rounded to nearest even.
+ */
+int dwconv3x3(const void* x, const float* w, int B, int Hgrid, int Wgrid, int C, int dtype, void* y,
+              cudaStream_t stream);
+
+/*
+ * dig_gla_device_status -- synchronises `stream`, then returns and clears the
+ * current device's status word: GLA_OK, or the first GLA_ERR_TIMEOUT /
+ * GLA_ERR_RANGE a kernel recorded since the last call.  Returns GLA_ERR_CUDA if
+ * the synchronisation itself fails.
+ */
+int dig_gla_device_status(cudaStream_t stream);
+
+/* Human-readable name of a gla_status_t value (static storage). */
+const char* dig_gla_status_string(int status);
+
+/* Releases cached host-side state (nothing is cached on the device). */
+void dig_gla_release(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIG_GLA_H_ */
