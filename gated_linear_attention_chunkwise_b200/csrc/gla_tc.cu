@@ -167,28 +167,36 @@ __device__ __forceinline__ float tile_at(const uint8_t* tile, int r, int i) {
 }
 
 // Exact token-by-token recurrence for one chunk, used when the chunk's gates
-// decay too fast for the factorised form: thread j < dv owns value column j of
-// the fp32 state sS[dk][dv] (loaded with S_in); sLA holds the raw log-gates.
-__device__ void chunk_serial(const uint8_t* sQ, const uint8_t* sK, const uint8_t* sV, float* sLA, float* sS,
+// decay too fast for the factorised form.  Thread j < dv keeps value column j of
+// the fp32 state in registers, starting from S_in (stored [dv][dk] at `s_in`);
+// sLA holds the raw log-gates of the chunk.
+__device__ void chunk_serial(const uint8_t* sQ, const uint8_t* sK, const uint8_t* sV, float* sLA, const float* s_in,
                              const TcArgs& a, int f0, int b, int h) {
   const int pw = a.dk + 4;
   for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
     const int r = e / a.dk, i = e - r * a.dk;
     sLA[r * pw + i] = __expf(sLA[r * pw + i]);  // alpha; exp(-inf) = 0 is a full reset
   }
-  __syncthreads();
   const int j = threadIdx.x;
+  const bool own = j < a.dv;
+  float st[128];
+#pragma unroll
+  for (int i = 0; i < 128; ++i) st[i] = (own && i < a.dk) ? s_in[(int64_t)j * a.dk + i] : 0.f;
+  __syncthreads();
   for (int s = 0; s < MC; ++s) {
     const int r = a.g.reverse ? (MC - 1 - s) : s;
     const int f = f0 + r;
     if (f < 0 || f >= a.g.T) continue;  // padding rows (uniform across the block)
-    if (j < a.dv) {
+    if (own) {
       const float vj = tile_at(sV, r, j);
+      const float* al = sLA + r * pw;
       float acc = 0.f;
-      for (int i = 0; i < a.dk; ++i) {
-        const float st = fmaf(sLA[r * pw + i], sS[i * a.dv + j], tile_at(sK, r, i) * vj);
-        sS[i * a.dv + j] = st;
-        acc = fmaf(tile_at(sQ, r, i), st, acc);
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        if (i < a.dk) {
+          st[i] = fmaf(al[i], st[i], tile_at(sK, r, i) * vj);
+          acc = fmaf(tile_at(sQ, r, i), st[i], acc);
+        }
       }
       a.out[(((int64_t)b * a.g.T + base_pos_to_token(a.g, f)) * a.H + h) * a.dv + j] = __float2bfloat16_rn(acc);
     }
@@ -328,13 +336,16 @@ __global__ void __launch_bounds__(NT, 1) gla_tc_output(const TcArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5;
 
   const uint32_t gpart = (uint32_t)a.Np * 128u;
+  const uint32_t la_bytes = (uint32_t)MC * (uint32_t)(a.dk + 4) * 4u;
   const uint32_t oQ = 0;
   const uint32_t oK = oQ + (uint32_t)a.PK * PART;
   const uint32_t oV = oK + (uint32_t)a.PK * PART;
-  const uint32_t oP = oV + (uint32_t)a.PV * PART;
-  const uint32_t oG = oP + 2 * PART;
+  const uint32_t oG = oV + (uint32_t)a.PV * PART;
+  // Scratch: the log-gate tile lives here until the gates are applied; the bf16
+  // score tile P (2 parts, K = 128 keys) reuses it after the score MMA.
   const uint32_t oLA = oG + (uint32_t)a.PK * gpart;
-  const uint32_t oBL = oLA + (uint32_t)MC * (uint32_t)(a.dk + 4) * 4u;
+  const uint32_t oP = oLA;
+  const uint32_t oBL = oLA + (la_bytes > 2 * PART ? la_bytes : 2 * PART);
   const uint32_t oBar = (oBL + (uint32_t)a.dk * 4u + 15u) & ~15u;
   const uint32_t oTm = oBar + 8;
   float* sLA = reinterpret_cast<float*>(smem + oLA);
@@ -371,14 +382,7 @@ __global__ void __launch_bounds__(NT, 1) gla_tc_output(const TcArgs a) {
   const int64_t cid = (int64_t)bh * a.NC + c;
   if (a.flags[cid]) {
     // Exact serial path; S_in (fp32, [dv][dk]) was left in the S_loc slot by pass 2.
-    float* sS = reinterpret_cast<float*>(smem + oP);  // reuses sP and sG: dk*dv*4 <= 64 KB
-    const float* src = a.s_locT + cid * a.dv * a.dk;
-    for (int e = tid; e < a.dk * a.dv; e += NT) {
-      const int j = e / a.dk, i = e - j * a.dk;
-      sS[i * a.dv + j] = src[e];
-    }
-    __syncthreads();
-    chunk_serial(smem + oQ, smem + oK, smem + oV, sLA, sS, a, f0, b, h);
+    chunk_serial(smem + oQ, smem + oK, smem + oV, sLA, a.s_locT + cid * a.dv * a.dk, a, f0, b, h);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, 256);
@@ -492,7 +496,9 @@ TcLayout tc_layout(const GlaShape& s) {
   L.img_bytes = round_up(BH * L.NC * (size_t)L.PK * L.Np * 128, 256);
   const size_t la = (size_t)MC * (s.dk + 4) * 4 + (size_t)s.dk * 4 + 16 + 16;
   L.smem_state = 1024 + (size_t)(2 + L.PV) * PART + la;
-  L.smem_out = 1024 + (size_t)(2 * L.PK + L.PV + 2) * PART + (size_t)L.PK * L.Np * 128 + la;
+  const size_t la_tile = (size_t)MC * (s.dk + 4) * 4;
+  L.smem_out = 1024 + (size_t)(2 * L.PK + L.PV) * PART + (size_t)L.PK * L.Np * 128 +
+               (la_tile > 2 * PART ? la_tile : 2 * PART) + (size_t)s.dk * 4 + 16 + 16;
   return L;
 }
 
