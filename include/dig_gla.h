@@ -92,6 +92,37 @@ int gla_fwd_f32(const float* q, const float* k, const float* v, const float* log
                 int Hgrid, int Wgrid, int dk, int dv, int dir, float* out, cudaStream_t stream);
 
 /*
+ * gla_fwd_f32_noalloc -- gla_fwd_f32 without any device allocation.  The paper
+ * has no counterpart: this is a library convenience.
+ *
+ * For callers that cannot call cudaMalloc / cudaMallocAsync while they run the
+ * GLA: a host framework that owns every device allocation through its own pool
+ * and forbids foreign ones, a real-time or embedded program that allocates
+ * everything at start-up because allocating may block or synchronise the device,
+ * or work recorded into a CUDA graph that must not contain memory nodes.  The
+ * caller passes the inputs and the output exactly as for gla_fwd_f32 (same
+ * shapes, directions, arithmetic and result); the scratch lives in a fixed
+ * array of DIG_GLA_NOALLOC_SCRATCH_BYTES (8 MiB) of device memory inside the
+ * library, which every GPU that loads the library holds until the process exits.
+ *
+ *   - Capacity: the call needs 2*ceil(T/64)*B*H*dk*dv*4 + ceil(T/64)*B*H*(dk+1)*4
+ *     bytes of scratch (each term rounded up to 256); a larger problem returns
+ *     GLA_ERR_UNSUPPORTED and launches nothing.  (c1: B=2, H=6, T=256, d=64 needs
+ *     about 1.6 MB.)
+ *   - First call per device: it looks up the array's device address with
+ *     cudaGetSymbolAddress (with that device current) and caches it.  Make this
+ *     first call before any stream capture.
+ *   - Sharing: every call uses the same array, which keeps the last call's
+ *     contents; nothing in it needs to start at zero.  Calls that overlap on the
+ *     GPU (concurrent streams, or host threads launching at the same time) race on
+ *     the array and corrupt each other's results: serialise them.
+ *   - Allocates nothing and frees nothing, on the host or the device.
+ */
+#define DIG_GLA_NOALLOC_SCRATCH_BYTES (8u << 20)
+int gla_fwd_f32_noalloc(const float* q, const float* k, const float* v, const float* log_alpha, int B, int H,
+                        int Hgrid, int Wgrid, int dk, int dv, int dir, float* out, cudaStream_t stream);
+
+/*
  * srem_reorient -- SREM's change of scan direction as an explicit row gather
  * (DiG paper notes, SREM: the block ends by transposing the 2D token matrix and
  * flipping the sequence, both O(T) operations; DiG Block step (5)).
