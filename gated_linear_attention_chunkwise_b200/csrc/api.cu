@@ -121,7 +121,7 @@ struct GlaCall {
 };
 cudaError_t run_tc(void* ws, void* ctx) {
   const GlaCall* c = static_cast<const GlaCall*>(ctx);
-  return dig::gla_fused_forward(c->q, c->k, c->v, c->la, c->out, c->s, ws, c->st);
+  return dig::gla_ws_forward(c->q, c->k, c->v, c->la, c->out, c->s, ws, c->st);
 }
 cudaError_t run_f32(void* ws, void* ctx) {
   const GlaCall* c = static_cast<const GlaCall*>(ctx);
@@ -138,7 +138,7 @@ int gla_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
   if (rc != GLA_OK) return rc;
   if ((rc = dig::check_device()) != GLA_OK) return rc;
   GlaCall c{q, k, v, log_alpha, out, GlaShape{B, H, Hgrid, Wgrid, dk, dv, dir}, stream};
-  return dig::run_with_workspace(dig::gla_fused_workspace_bytes(c.s), stream, run_tc, &c);
+  return dig::run_with_workspace(dig::gla_ws_workspace_bytes(c.s), stream, run_tc, &c);
 }
 
 int gla_fwd_f32(const float* q, const float* k, const float* v, const float* log_alpha, int B, int H, int Hgrid,

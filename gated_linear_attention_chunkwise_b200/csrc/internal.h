@@ -25,6 +25,11 @@ size_t gla_fused_workspace_bytes(const GlaShape& s);
 cudaError_t gla_fused_forward(const void* q, const void* k, const void* v, const float* la, void* out,
                               const GlaShape& s, void* workspace, cudaStream_t st);
 
+// ---- bf16 warp-specialised single-kernel path ----
+size_t gla_ws_workspace_bytes(const GlaShape& s);
+cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const float* la, void* out, const GlaShape& s,
+                           void* workspace, cudaStream_t st);
+
 // ---- fp32 SIMT path (chunks of 64 scan positions) ----
 constexpr int kChunkF32 = 64;
 size_t gla_f32_workspace_bytes(const GlaShape& s);
