@@ -16,6 +16,9 @@
 
 namespace dig {
 
+// First error a kernel recorded on this device (GLA_OK while none).
+__device__ int g_device_status = 0;
+
 namespace {
 
 std::mutex g_mu;

@@ -18,16 +18,24 @@
 //
 // Roles (14 warps, 448 threads), connected by mbarriers:
 //   warp 0      producer: TMA loads of each chunk's q, k, v (32-byte-swizzled 16-channel
-//               boxes, the UMMA operand layout) and log-gates into a ring of stages
-//               (cp.async by the whole warp for column scans of grids whose height is
-//               not a multiple of 8);
+//               boxes, the UMMA operand layout) and log-gates into a ring of stages;
 //   warp 1      MMA issuer (tcgen05, one thread) and TMEM owner;
 //   warps 2-5   suffix sums of the log-gates, one thread per key channel;
 //   warps 6-9   gates applied in place (K^, Q~), one thread per row;
 //   warps 10-13 TMEM-side work, one thread per TMEM lane: G = Diag(gamma) S, score
-//               masking to the bf16 P tile, output epilogue, look-back, serial path.
-// TMEM (512 columns): scores [0,128), O buffer 0 [128,256), running state [256,384),
+//               masking to bf16 P, output epilogue, look-back, serial path.
+// TMEM (512 columns): scores [0,128) -- overwritten by the bf16 P matrix (two keys per
+// column, the A operand of P V) --, O buffer 0 [128,256), running state [256,384),
 // segment aggregate [384,512) -- reused as O buffer 1 once the look-back is done.
+// A stage is free once the MMAs that read it complete, so loads run ahead of the
+// output epilogue.
+//
+// Chunks follow the direction's base order (raster rows, or grid columns for T->B /
+// B->T) and are always cut in forward order; reversed scans visit them backwards and
+// walk each chunk's rows backwards.  Each chunk is one TMA box per tensor: 128
+// consecutive raster positions; 128/Hgrid whole columns when Hgrid divides 128;
+// otherwise one column cut into pieces of at most 128 rows.  Rows past the grid are
+// zero-filled by the TMA and contribute nothing.
 #include <math.h>
 #include <string.h>
 
@@ -44,7 +52,6 @@ constexpr int MC = kChunkTC;
 constexpr int NT = 448;
 constexpr int kWarpProd = 0, kWarpMma = 1, kWarpSuf = 2, kWarpGate = 6, kWarpEpi = 10;
 constexpr uint32_t ATOM32 = MC * 32u;    // one 16-channel block of a 32B-swizzled 128-row tile
-constexpr uint32_t PART128 = MC * 128u;  // one 64-key part of the 128B-swizzled P tile
 constexpr float kMaxGateRange = 80.0f;
 constexpr uint32_t kColS = 0, kColO0 = 128, kColState = 256, kColSeg = 384;
 constexpr uint32_t kLayoutSW32 = 6;
@@ -55,7 +62,7 @@ enum {
   kBarFull = 0,                          // [S]  tiles landed
   kBarSuf = kBarFull + kMaxStages,       // [S]  suffix sums done (128 arrivals)
   kBarGate = kBarSuf + kMaxStages,       // [S]  gates applied (128 arrivals)
-  kBarEmpty = kBarGate + kMaxStages,     // [S]  stage free (MMA commit + 128 arrivals)
+  kBarEmpty = kBarGate + kMaxStages,     // [S]  stage free (MMA commit, or the serial path)
   kBarScFull = kBarEmpty + kMaxStages,   // score MMA done
   kBarScEmpty,                           // scores read (128 arrivals)
   kBarPReady,                            // P and G written (128 arrivals)
@@ -78,7 +85,8 @@ struct WsArgs {
   int* flags;     // [BH][NS]               0 nothing, 1 aggregate, 2 inclusive
   int* ticket;
   int H, BH, dk, dv, NC, NS, G;
-  int Kp, Np, nstage, box_rows;
+  int Kp, Np, nstage;
+  int mode, rpc, ppr;  // chunk geometry: 0 raster, 1 whole columns (rpc per chunk), 2 column pieces (ppr per column)
   uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oMisc, oBar, oTm;
   ScanGeom g;
 };
@@ -128,12 +136,11 @@ __device__ __forceinline__ bool group_and(uint32_t id, uint32_t n, bool v) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+__device__ __forceinline__ void mbar_arrive_cnt(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-// cp.async completion of this thread triggers one arrival (counted in the init count).
-__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
   asm volatile(
@@ -148,6 +155,57 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
       : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 16-column TMEM load without the wait: the registers hold the columns only after
+// tmem_ld_cols' wait (several loads then share one round trip).
+__device__ __forceinline__ void tmem_ld16_issue(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+// Orders every later use of r after the preceding tcgen05.wait::ld.
+__device__ __forceinline__ void reg_tie16(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]));
+}
+// Columns [0, n) of this warp's lanes from taddr (n <= 16 P, multiple of 16), one wait.
+template <int P>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, int n, uint32_t (&r)[P][16]) {
+#pragma unroll
+  for (int q = 0; q < P; ++q)
+    if (16 * q < n) tmem_ld16_issue(taddr + (uint32_t)(16 * q), r[q]);
+  tmem_ld_wait();
+#pragma unroll
+  for (int q = 0; q < P; ++q) reg_tie16(r[q]);
+}
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+// D (+)= A * B with A read from TMEM (lane = row, two bf16 of K per column) and B
+// described in shared memory.
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ uint32_t pack_u2(uint32_t x, uint32_t y) {
+  return pack_bf16x2(__uint_as_float(x), __uint_as_float(y));
+}
 
 __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
                                             int c4, uint32_t bar) {
@@ -189,13 +247,35 @@ __device__ int wait_flag(const int* flags, int64_t idx) {
   return (int)f;
 }
 
-__device__ __forceinline__ void run_coords(const ScanGeom& g, int f, int& y, int& x) {
-  if (!g.column_base) {
-    y = f;
+// Forward chunk index of scan-order chunk c.
+__device__ __forceinline__ int fwd_chunk(const WsArgs& a, int c) { return a.g.reverse ? a.NC - 1 - c : c; }
+
+// Raster token of tile row r of forward chunk cf, or -1 for a padding row.
+__device__ __forceinline__ int row_token(const WsArgs& a, int cf, int r) {
+  if (a.mode == 0) {
+    const int f = cf * MC + r;
+    return f < a.g.T ? f : -1;
+  }
+  if (a.mode == 1) {
+    const int xl = r / a.g.Hg;
+    const int x = cf * a.rpc + xl, y = r - xl * a.g.Hg;
+    return x < a.g.Wg ? y * a.g.Wg + x : -1;
+  }
+  const int x = cf / a.ppr, y = (cf - x * a.ppr) * MC + r;
+  return y < a.g.Hg ? y * a.g.Wg + x : -1;
+}
+
+// TMA coordinates (run position, run index) of forward chunk cf's box.
+__device__ __forceinline__ void chunk_box(const WsArgs& a, int cf, int& y, int& x) {
+  if (a.mode == 0) {
+    y = cf * MC;
     x = 0;
+  } else if (a.mode == 1) {
+    y = 0;
+    x = cf * a.rpc;
   } else {
-    x = (f >= 0) ? f / g.Hg : -((-f + g.Hg - 1) / g.Hg);
-    y = f - x * g.Hg;
+    x = cf / a.ppr;
+    y = (cf - x * a.ppr) * MC;
   }
 }
 
@@ -204,53 +284,19 @@ __device__ __forceinline__ int job_chunk(int j, int c0, int n) { return j < n ? 
 // ---------------------------------------------------------------------------
 // Producer
 // ---------------------------------------------------------------------------
-__device__ void tma_job(const WsArgs& a, const TensorMaps& tm, uint32_t st, uint32_t bar, int f0, bool with_q, int b,
+__device__ void tma_job(const WsArgs& a, const TensorMaps& tm, uint32_t st, uint32_t bar, int cf, bool with_q, int b,
                         int h) {
-  const int R = a.box_rows;
   const uint32_t bytes = (uint32_t)(with_q ? 2 : 1) * (uint32_t)a.Kp * 256u + (uint32_t)a.Np * 256u +
                          (uint32_t)MC * (uint32_t)(a.dk + 4) * 4u;
   mbar_expect_tx(bar, bytes);
-  for (int m = 0; m < MC / R; ++m) {
-    int y, x;
-    run_coords(a.g, f0 + m * R, y, x);
-    const uint32_t roff = (uint32_t)(m * R) * 32u;
-    for (int cb = 0; cb < (a.Kp >> 4); ++cb) {
-      tma_load_5d(st + a.oK + (uint32_t)cb * ATOM32 + roff, &tm.k, cb * 16, h, y, x, b, bar);
-      if (with_q) tma_load_5d(st + a.oQ + (uint32_t)cb * ATOM32 + roff, &tm.q, cb * 16, h, y, x, b, bar);
-    }
-    for (int cb = 0; cb < (a.Np >> 4); ++cb)
-      tma_load_5d(st + a.oV + (uint32_t)cb * ATOM32 + roff, &tm.v, cb * 16, h, y, x, b, bar);
-    tma_load_5d(st + a.oLA + (uint32_t)(m * R) * (uint32_t)(a.dk + 4) * 4u, &tm.la, 0, h, y, x, b, bar);
+  int y, x;
+  chunk_box(a, cf, y, x);
+  for (int cb = 0; cb < (a.Kp >> 4); ++cb) {
+    tma_load_5d(st + a.oK + (uint32_t)cb * ATOM32, &tm.k, cb * 16, h, y, x, b, bar);
+    if (with_q) tma_load_5d(st + a.oQ + (uint32_t)cb * ATOM32, &tm.q, cb * 16, h, y, x, b, bar);
   }
-}
-
-// cp.async variant, issued by the 32 lanes of the producer warp.
-__device__ void cpasync_job(const WsArgs& a, uint32_t st, uint32_t bar, int f0, bool with_q, int b, int h, int lane) {
-  auto rows_sw32 = [&](uint32_t tile, const __nv_bfloat16* base, int d, int W) {
-    const int cpr = W >> 3;
-    for (int idx = lane; idx < MC * cpr; idx += 32) {
-      const int r = idx / cpr, cc = idx - r * cpr;
-      const int f = f0 + r;
-      const bool valid = (f >= 0) && (f < a.g.T) && (cc * 8 < d);
-      const __nv_bfloat16* src = base;
-      if (valid) src = base + (((int64_t)b * a.g.T + base_pos_to_token(a.g, f)) * a.H + h) * d + cc * 8;
-      cp_async16(tile + sw32_off((uint32_t)r, (uint32_t)cc * 8u), src, valid);
-    }
-  };
-  rows_sw32(st + a.oK, a.k, a.dk, a.Kp);
-  if (with_q) rows_sw32(st + a.oQ, a.q, a.dk, a.Kp);
-  rows_sw32(st + a.oV, a.v, a.dv, a.Np);
-  const int cpr = (a.dk + 4) >> 2;
-  const uint32_t pitch = (uint32_t)(a.dk + 4) * 4u;
-  for (int idx = lane; idx < MC * cpr; idx += 32) {
-    const int r = idx / cpr, cc = idx - r * cpr;
-    const int f = f0 + r;
-    const bool valid = (f >= 0) && (f < a.g.T) && (cc * 4 < a.dk);
-    const float* src = a.la;
-    if (valid) src = a.la + (((int64_t)b * a.g.T + base_pos_to_token(a.g, f)) * a.H + h) * a.dk + cc * 4;
-    cp_async16(st + a.oLA + (uint32_t)r * pitch + (uint32_t)cc * 16u, src, valid);
-  }
-  cp_async_mbar_arrive(bar);
+  for (int cb = 0; cb < (a.Np >> 4); ++cb) tma_load_5d(st + a.oV + (uint32_t)cb * ATOM32, &tm.v, cb * 16, h, y, x, b, bar);
+  tma_load_5d(st + a.oLA, &tm.la, 0, h, y, x, b, bar);
 }
 
 // ---------------------------------------------------------------------------
@@ -259,7 +305,7 @@ __device__ void cpasync_job(const WsArgs& a, uint32_t st, uint32_t bar, int f0, 
 // q, k are still the raw (unscaled) swizzled tiles.
 // ---------------------------------------------------------------------------
 __device__ void chunk_serial(const WsArgs& a, const uint8_t* st, float* red, uint32_t tstate, uint32_t lane_base,
-                             int i, int f0, int b, int h) {
+                             int i, int cf, int b, int h) {
   const int lane = threadIdx.x & 31, ew = (threadIdx.x >> 5) - kWarpEpi;  // 0..3
   for (int cb = 0; cb < (a.Np >> 4); ++cb) {
     float s[16];
@@ -269,9 +315,8 @@ __device__ void chunk_serial(const WsArgs& a, const uint8_t* st, float* red, uin
       for (int q = 0; q < 16; ++q) s[q] = 0.f;
     for (int step = 0; step < MC; ++step) {
       const int r = a.g.reverse ? (MC - 1 - step) : step;
-      const int f = f0 + r;
-      if (f < 0 || f >= a.g.T) continue;  // padding row: uniform
-      const int t = base_pos_to_token(a.g, f);
+      const int t = row_token(a, cf, r);
+      if (t < 0) continue;  // padding row: uniform
       float alpha = 1.f, kq = 0.f, qi = 0.f;
       if (i < a.dk) {
         alpha = __expf(__ldg(a.la + (((int64_t)b * a.g.T + t) * a.H + h) * a.dk + i));
@@ -318,7 +363,6 @@ __device__ __forceinline__ uint32_t align1024(uint32_t x) { return (x + 1023u) &
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
-template <bool TMA>
 __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid_constant__ TensorMaps tm) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -341,10 +385,10 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
   }
   if (tid == 0) {
     for (int s = 0; s < a.nstage; ++s) {
-      mbar_init(BAR(kBarFull + s), TMA ? 1 : 32);
+      mbar_init(BAR(kBarFull + s), 1);
       mbar_init(BAR(kBarSuf + s), 128);
       mbar_init(BAR(kBarGate + s), 128);
-      mbar_init(BAR(kBarEmpty + s), 129);
+      mbar_init(BAR(kBarEmpty + s), 1);
     }
     mbar_init(BAR(kBarScFull), 1);
     mbar_init(BAR(kBarScEmpty), 128);
@@ -378,17 +422,13 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
 
   if (warp == kWarpProd) {
     // ------------------------------------------------------------ producer
-    if (TMA ? lane == 0 : true) {
+    if (lane == 0) {
       for (int j = 0; j < njob; ++j) {
         const int s = j % S, k = j / S;
         if (k > 0 && !wait_bar(BAR(kBarEmpty + s), (uint32_t)((k - 1) & 1), abort_flag)) break;
         const uint32_t st = sbase + (uint32_t)s * a.stage_bytes;
-        const int f0 = chunk_first_base_pos(a.g, job_chunk(j, c0, n), MC);
-        if (TMA)
-          tma_job(a, tm, st, BAR(kBarFull + s), f0, j >= n, b, h);
-        else
-          cpasync_job(a, st, BAR(kBarFull + s), f0, j >= n, b, h, lane);
-        if (lane == 0) sMisc[3] = j + 1;
+        tma_job(a, tm, st, BAR(kBarFull + s), fwd_chunk(a, job_chunk(j, c0, n)), j >= n, b, h);
+        sMisc[3] = j + 1;
       }
     }
   } else if (warp == kWarpMma) {
@@ -410,10 +450,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
           if (j == n - 1) umma_commit(BAR(kBarSegDone));
           continue;
         }
-        if (sWide[s]) {  // evaluated serially by the TMEM-side warps
-          umma_commit(BAR(kBarEmpty + s));
-          continue;
-        }
+        if (sWide[s]) continue;  // evaluated serially by the TMEM-side warps, which free the stage
         if (kb > 0 && !wait_bar(BAR(kBarScEmpty), (uint32_t)((kb - 1) & 1), abort_flag)) break;
         tc_fence_after();
         {
@@ -432,8 +469,8 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
           const uint32_t tO = tbase + (ob ? kColSeg : kColO0);
           const uint32_t id_pv = idesc_bf16_f32(MC, a.Np, false, true);
 #pragma unroll 1
-          for (int kk = 0; kk < MC / 16; ++kk)
-            umma_ss(tO, desc_kmajor(st + a.oLA, PART128, kk), desc_sw32(st + a.oV + (uint32_t)kk * 512u, ATOM32, 256u),
+          for (int kk = 0; kk < MC / 16; ++kk)  // P is bf16 in the score columns
+            umma_ts(tO, tbase + kColS + (uint32_t)(kk * 8), desc_sw32(st + a.oV + (uint32_t)kk * 512u, ATOM32, 256u),
                     id_pv, kk > 0 ? 1u : 0u);
 #pragma unroll 1
           for (int kk = 0; kk < (a.Kp >> 4); ++kk)
@@ -473,14 +510,20 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
         const int step = a.g.reverse ? pw : -pw;
         const float base = pass1 ? off : 0.f;
         float acc = 0.f, ab = 0.f, po = 0.f;
-#pragma unroll 8
-        for (int p = 0; p < MC; ++p) {
-          const float x = *ptr;
-          *ptr = acc + base;
-          acc += x;
-          ab += fabsf(x);
-          po += fmaxf(x, 0.f);
-          ptr += step;
+        // Sixteen loads are issued before their stores so that they overlap.
+#pragma unroll 1
+        for (int p0 = 0; p0 < MC; p0 += 16) {
+          float x[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) x[q] = ptr[q * step];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            ptr[q * step] = acc + base;
+            acc += x[q];
+            ab += fabsf(x[q]);
+            po += fmaxf(x[q], 0.f);
+          }
+          ptr += 16 * step;
         }
         sBL[s * 128 + i] = acc;
         if (pass1) {
@@ -512,32 +555,45 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
       uint8_t* st = smem + (uint32_t)s * a.stage_bytes;
       if (pass1 || !sWide[s]) {
         const float* urow = reinterpret_cast<const float*>(st + a.oLA) + r * (a.dk + 4);
-        for (int c0c = 0; c0c < a.dk; c0c += 8) {
-          const uint32_t o = sw32_off((uint32_t)r, (uint32_t)c0c);
-          const float4 u0 = *reinterpret_cast<const float4*>(urow + c0c);
-          const float4 u1 = *reinterpret_cast<const float4*>(urow + c0c + 4);
-          const float e[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-          {
-            uint4* pk = reinterpret_cast<uint4*>(st + a.oK + o);
-            uint4 w = *pk;
-            uint32_t* u = reinterpret_cast<uint32_t*>(&w);
+        // Three 8-channel groups per round: all loads first, then gates, then stores.
+        for (int cbase = 0; cbase < a.dk; cbase += 24) {
+          float4 u[3][2];
+          uint4 kw[3], qw[3];
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              const float2 x = unpack_bf16x2(u[jj]);
-              u[jj] = pack_bf16x2(x.x * __expf(e[2 * jj]), x.y * __expf(e[2 * jj + 1]));
+          for (int g3 = 0; g3 < 3; ++g3) {
+            const int c = cbase + 8 * g3;
+            if (c < a.dk) {
+              const uint32_t o = sw32_off((uint32_t)r, (uint32_t)c);
+              u[g3][0] = *reinterpret_cast<const float4*>(urow + c);
+              u[g3][1] = *reinterpret_cast<const float4*>(urow + c + 4);
+              kw[g3] = *reinterpret_cast<const uint4*>(st + a.oK + o);
+              if (!pass1) qw[g3] = *reinterpret_cast<const uint4*>(st + a.oQ + o);
             }
-            *pk = w;
           }
-          if (!pass1) {
-            uint4* pq = reinterpret_cast<uint4*>(st + a.oQ + o);
-            uint4 w = *pq;
-            uint32_t* u = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              const float2 x = unpack_bf16x2(u[jj]);
-              u[jj] = pack_bf16x2(x.x * __expf(-e[2 * jj]), x.y * __expf(-e[2 * jj + 1]));
+          for (int g3 = 0; g3 < 3; ++g3) {
+            const int c = cbase + 8 * g3;
+            if (c < a.dk) {
+              const uint32_t o = sw32_off((uint32_t)r, (uint32_t)c);
+              const float e[8] = {u[g3][0].x, u[g3][0].y, u[g3][0].z, u[g3][0].w,
+                                  u[g3][1].x, u[g3][1].y, u[g3][1].z, u[g3][1].w};
+              uint32_t* uk = reinterpret_cast<uint32_t*>(&kw[g3]);
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj) {
+                const float2 xx = unpack_bf16x2(uk[jj]);
+                uk[jj] = pack_bf16x2(xx.x * __expf(e[2 * jj]), xx.y * __expf(e[2 * jj + 1]));
+              }
+              *reinterpret_cast<uint4*>(st + a.oK + o) = kw[g3];
+              if (!pass1) {
+                uint32_t* uq = reinterpret_cast<uint32_t*>(&qw[g3]);
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                  const float2 xx = unpack_bf16x2(uq[jj]);
+                  uq[jj] = pack_bf16x2(xx.x * __expf(-e[2 * jj]), xx.y * __expf(-e[2 * jj + 1]));
+                }
+                *reinterpret_cast<uint4*>(st + a.oQ + o) = qw[g3];
+              }
             }
-            *pq = w;
           }
         }
         fence_proxy_async_smem();
@@ -551,7 +607,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
     const int e = tid - 32 * kWarpEpi;
     int kb = 0;
     bool prev_pending = false;
-    int prev_s = 0, prev_f0 = 0;
+    int prev_cf = 0;
     bool ok = true;
 
     // Epilogue of the previous output buffer: O -> bf16 -> out[b][token][h][:].
@@ -561,31 +617,131 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
       if (!group_and(2, 128, wait_bar(BAR(kBarBatch0 + ob), (uint32_t)(((kb - 1) >> 1) & 1), abort_flag)))
         return false;
       tc_fence_after();
-      const int f = prev_f0 + i;
-      const bool valid = (f >= 0) && (f < a.g.T);
+      const int t = row_token(a, prev_cf, i);
+      const bool valid = t >= 0;
       __nv_bfloat16* orow = a.out;
-      if (valid) orow = a.out + (((int64_t)b * a.g.T + base_pos_to_token(a.g, f)) * a.H + h) * a.dv;
+      if (valid) orow = a.out + (((int64_t)b * a.g.T + t) * a.H + h) * a.dv;
       const uint32_t tO = tbase + (ob ? kColSeg : kColO0) + lane_base;
-      for (int cb = 0; cb < a.Np; cb += 16) {
-        float o[16];
-        tmem_ld16(tO + (uint32_t)cb, o);
+      for (int c0 = 0; c0 < a.Np; c0 += 32) {
+        uint32_t o[2][16];
+        tmem_ld_cols<2>(tO + (uint32_t)c0, a.Np - c0, o);
         if (valid) {
 #pragma unroll
-          for (int q = 0; q < 16; q += 8)
-            if (cb + q < a.dv)
-              *reinterpret_cast<uint4*>(orow + cb + q) =
-                  make_uint4(pack_bf16x2(o[q], o[q + 1]), pack_bf16x2(o[q + 2], o[q + 3]),
-                             pack_bf16x2(o[q + 4], o[q + 5]), pack_bf16x2(o[q + 6], o[q + 7]));
+          for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int hh = 0; hh < 16; hh += 8)
+              if (c0 + 16 * q + hh < a.dv)
+                *reinterpret_cast<uint4*>(orow + c0 + 16 * q + hh) =
+                    make_uint4(pack_u2(o[q][hh], o[q][hh + 1]), pack_u2(o[q][hh + 2], o[q][hh + 3]),
+                               pack_u2(o[q][hh + 4], o[q][hh + 5]), pack_u2(o[q][hh + 6], o[q][hh + 7]));
         }
       }
       tc_fence_before();
       mbar_arrive(BAR(kBarOEmpty0 + ob));
-      mbar_arrive(BAR(kBarEmpty + prev_s));
       prev_pending = false;
       return true;
     };
 
-    for (int j = 0; j < njob && ok; ++j) {
+    // ---- end of pass 1: publish the segment aggregate and look back ----
+    // (this group takes no part in pass 1 itself)
+    if (!group_and(2, 128, wait_bar(BAR(kBarSegDone), 0u, abort_flag))) ok = false;
+    if (ok) {
+      tc_fence_after();
+      const int DQ = a.dv >> 2;
+      const uint32_t tSeg = tbase + kColSeg + lane_base, tSt = tbase + kColState + lane_base;
+      const float gs = sGam[i];
+      if (i < a.dk) a.agg_g[seg_id * a.dk + i] = gs;
+      for (int c0 = 0; c0 < a.Np; c0 += 64) {
+        uint32_t t[4][16];
+        tmem_ld_cols<4>(tSeg + (uint32_t)c0, a.Np - c0, t);
+        if (i < a.dk) {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const int jq = c0 / 4 + q;
+            if (jq < DQ)
+              *reinterpret_cast<float4*>(a.agg_S + ((seg_id * DQ + jq) * a.dk + i) * 4) =
+                  make_float4(__uint_as_float(t[q >> 2][4 * (q & 3)]), __uint_as_float(t[q >> 2][4 * (q & 3) + 1]),
+                              __uint_as_float(t[q >> 2][4 * (q & 3) + 2]), __uint_as_float(t[q >> 2][4 * (q & 3) + 3]));
+          }
+        }
+      }
+      __threadfence();
+      named_sync(2, 128);
+      if (e == 0) st_release(a.flags + seg_id, 1);
+      {
+        float z[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) z[q] = 0.f;
+        for (int cb = 0; cb < a.Np; cb += 16) tmem_st16(tSt + (uint32_t)cb, z);
+        tmem_st_wait();
+      }
+      float gam = 1.f;
+      for (int p = seg - 1; p >= 0; --p) {
+        const int64_t pid = (int64_t)bh * a.NS + p;
+        if (e == 0) sMisc[2] = wait_flag(a.flags, pid);
+        named_sync(2, 128);
+        const int fl = sMisc[2];
+        named_sync(2, 128);
+        if (fl == 0) break;  // timed out (recorded)
+        const float* src = (fl == 2 ? a.incl_S : a.agg_S);
+        // 32 columns of the predecessor's rows are loaded before the TMEM round trip.
+        for (int c0 = 0; c0 < a.Np; c0 += 32) {
+          float4 x[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int jq = c0 / 4 + q;
+            x[q] = (i < a.dk && jq < DQ)
+                       ? __ldcg(reinterpret_cast<const float4*>(src + ((pid * DQ + jq) * a.dk + i) * 4))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          uint32_t t[2][16];
+          tmem_ld_cols<2>(tSt + (uint32_t)c0, a.Np - c0, t);
+#pragma unroll
+          for (int c4 = 0; c4 < 2; ++c4) {
+            if (c0 + 16 * c4 < a.Np) {
+              float t16[16];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                t16[4 * q] = fmaf(gam, x[4 * c4 + q].x, __uint_as_float(t[c4][4 * q]));
+                t16[4 * q + 1] = fmaf(gam, x[4 * c4 + q].y, __uint_as_float(t[c4][4 * q + 1]));
+                t16[4 * q + 2] = fmaf(gam, x[4 * c4 + q].z, __uint_as_float(t[c4][4 * q + 2]));
+                t16[4 * q + 3] = fmaf(gam, x[4 * c4 + q].w, __uint_as_float(t[c4][4 * q + 3]));
+              }
+              tmem_st16(tSt + (uint32_t)(c0 + 16 * c4), t16);
+            }
+          }
+        }
+        tmem_st_wait();
+        if (fl == 1 && i < a.dk) gam *= __ldcg(a.agg_g + pid * a.dk + i);
+        if (fl == 2) break;
+      }
+      // Inclusive state of this segment: Diag(gamma_seg) S_in + aggregate.
+      for (int c0 = 0; c0 < a.Np; c0 += 32) {
+        uint32_t sin[2][16], sg[2][16];
+        tmem_ld_cols<2>(tSt + (uint32_t)c0, a.Np - c0, sin);
+        tmem_ld_cols<2>(tSeg + (uint32_t)c0, a.Np - c0, sg);
+        if (i < a.dk) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int jq = c0 / 4 + q;
+            const int pc = q >> 2, o4 = 4 * (q & 3);
+            if (jq < DQ)
+              *reinterpret_cast<float4*>(a.incl_S + ((seg_id * DQ + jq) * a.dk + i) * 4) = make_float4(
+                  fmaf(gs, __uint_as_float(sin[pc][o4]), __uint_as_float(sg[pc][o4])),
+                  fmaf(gs, __uint_as_float(sin[pc][o4 + 1]), __uint_as_float(sg[pc][o4 + 1])),
+                  fmaf(gs, __uint_as_float(sin[pc][o4 + 2]), __uint_as_float(sg[pc][o4 + 2])),
+                  fmaf(gs, __uint_as_float(sin[pc][o4 + 3]), __uint_as_float(sg[pc][o4 + 3])));
+          }
+        }
+      }
+      __threadfence();
+      tc_fence_before();
+      named_sync(2, 128);
+      if (e == 0) st_release(a.flags + seg_id, 2);
+      tc_fence_after();
+    }
+
+    for (int j = n; j < njob && ok; ++j) {
       const int s = j % S, k = j / S;
       // The previous chunk's epilogue releases its stage; it must not wait behind this
       // chunk's gates (with one stage, those need that very stage).
@@ -598,124 +754,45 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
         break;
       }
       uint8_t* st = smem + (uint32_t)s * a.stage_bytes;
-      const int f0 = chunk_first_base_pos(a.g, job_chunk(j, c0, n), MC);
-      if (j < n) {
-        mbar_arrive(BAR(kBarEmpty + s));
-        if (j < n - 1) continue;
-        // ---- end of pass 1: publish the aggregate and look back ----
-        if (!group_and(2, 128, wait_bar(BAR(kBarSegDone), 0u, abort_flag))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int DQ = a.dv >> 2;
-        const float gs = sGam[i];
-        if (i < a.dk) a.agg_g[seg_id * a.dk + i] = gs;
-        for (int cb = 0; cb < a.Np; cb += 16) {
-          float t16[16];
-          tmem_ld16(tbase + kColSeg + lane_base + (uint32_t)cb, t16);
-          if (i < a.dk) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int jq = cb / 4 + q;
-              if (jq < DQ)
-                *reinterpret_cast<float4*>(a.agg_S + ((seg_id * DQ + jq) * a.dk + i) * 4) =
-                    make_float4(t16[4 * q], t16[4 * q + 1], t16[4 * q + 2], t16[4 * q + 3]);
-            }
-          }
-        }
-        __threadfence();
-        named_sync(2, 128);
-        if (e == 0) st_release(a.flags + seg_id, 1);
-        {
-          float z[16];
-#pragma unroll
-          for (int q = 0; q < 16; ++q) z[q] = 0.f;
-          for (int cb = 0; cb < a.Np; cb += 16) tmem_st16(tbase + kColState + lane_base + (uint32_t)cb, z);
-          tmem_st_wait();
-        }
-        float gam = 1.f;
-        for (int p = seg - 1; p >= 0; --p) {
-          const int64_t pid = (int64_t)bh * a.NS + p;
-          if (e == 0) sMisc[2] = wait_flag(a.flags, pid);
-          named_sync(2, 128);
-          const int fl = sMisc[2];
-          named_sync(2, 128);
-          if (fl == 0) break;  // timed out (recorded)
-          const float* src = (fl == 2 ? a.incl_S : a.agg_S);
-          for (int cb = 0; cb < a.Np; cb += 16) {
-            float t16[16];
-            tmem_ld16(tbase + kColState + lane_base + (uint32_t)cb, t16);
-            if (i < a.dk) {
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int jq = cb / 4 + q;
-                if (jq < DQ) {
-                  const float4 x = __ldcg(reinterpret_cast<const float4*>(src + ((pid * DQ + jq) * a.dk + i) * 4));
-                  t16[4 * q] = fmaf(gam, x.x, t16[4 * q]);
-                  t16[4 * q + 1] = fmaf(gam, x.y, t16[4 * q + 1]);
-                  t16[4 * q + 2] = fmaf(gam, x.z, t16[4 * q + 2]);
-                  t16[4 * q + 3] = fmaf(gam, x.w, t16[4 * q + 3]);
-                }
-              }
-            }
-            tmem_st16(tbase + kColState + lane_base + (uint32_t)cb, t16);
-          }
-          tmem_st_wait();
-          if (fl == 1 && i < a.dk) gam *= __ldcg(a.agg_g + pid * a.dk + i);
-          if (fl == 2) break;
-        }
-        for (int cb = 0; cb < a.Np; cb += 16) {
-          float sin[16], sg[16];
-          tmem_ld16(tbase + kColState + lane_base + (uint32_t)cb, sin);
-          tmem_ld16(tbase + kColSeg + lane_base + (uint32_t)cb, sg);
-          if (i < a.dk) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int jq = cb / 4 + q;
-              if (jq < DQ)
-                *reinterpret_cast<float4*>(a.incl_S + ((seg_id * DQ + jq) * a.dk + i) * 4) =
-                    make_float4(fmaf(gs, sin[4 * q], sg[4 * q]), fmaf(gs, sin[4 * q + 1], sg[4 * q + 1]),
-                                fmaf(gs, sin[4 * q + 2], sg[4 * q + 2]), fmaf(gs, sin[4 * q + 3], sg[4 * q + 3]));
-            }
-          }
-        }
-        __threadfence();
-        tc_fence_before();
-        named_sync(2, 128);
-        if (e == 0) st_release(a.flags + seg_id, 2);
-        tc_fence_after();
-        continue;
-      }
+      const int cf = fwd_chunk(a, job_chunk(j, c0, n));
 
       // ---- pass 2 ----
       if (sWide[s]) {
-        chunk_serial(a, st, red, tbase + kColState, lane_base, i, f0, b, h);
+        chunk_serial(a, st, red, tbase + kColState, lane_base, i, cf, b, h);
         tc_fence_before();
-        mbar_arrive(BAR(kBarEmpty + s));
+        named_sync(2, 128);
+        if (e == 0) mbar_arrive(BAR(kBarEmpty + s));
         continue;
       }
       // G = Diag(gamma) S (state -> state, bf16 copy into the G tile)
       {
         const float gm = __expf(sBL[s * 128 + i]);
-        for (int cb = 0; cb < a.Np; cb += 16) {
-          float t16[16];
-          tmem_ld16(tbase + kColState + lane_base + (uint32_t)cb, t16);
+        const uint32_t tSt = tbase + kColState + lane_base;
+        for (int c0 = 0; c0 < a.Np; c0 += 32) {
+          uint32_t t[2][16];
+          tmem_ld_cols<2>(tSt + (uint32_t)c0, a.Np - c0, t);
 #pragma unroll
-          for (int q = 0; q < 16; ++q) t16[q] *= gm;
-          tmem_st16(tbase + kColState + lane_base + (uint32_t)cb, t16);
-          if (i < a.Kp) {
-            const uint4 w0 = make_uint4(pack_bf16x2(t16[0], t16[1]), pack_bf16x2(t16[2], t16[3]),
-                                        pack_bf16x2(t16[4], t16[5]), pack_bf16x2(t16[6], t16[7]));
-            const uint4 w1 = make_uint4(pack_bf16x2(t16[8], t16[9]), pack_bf16x2(t16[10], t16[11]),
-                                        pack_bf16x2(t16[12], t16[13]), pack_bf16x2(t16[14], t16[15]));
-            *reinterpret_cast<uint4*>(smem + a.oG + g_off((uint32_t)i, (uint32_t)cb, (uint32_t)a.Kp)) = w0;
-            *reinterpret_cast<uint4*>(smem + a.oG + g_off((uint32_t)i, (uint32_t)cb + 8u, (uint32_t)a.Kp)) = w1;
+          for (int c4 = 0; c4 < 2; ++c4) {
+            const int cb = c0 + 16 * c4;
+            if (cb < a.Np) {
+              float t16[16];
+#pragma unroll
+              for (int q = 0; q < 16; ++q) t16[q] = __uint_as_float(t[c4][q]) * gm;
+              tmem_st16(tSt + (uint32_t)cb, t16);
+              if (i < a.Kp) {
+                const uint4 w0 = make_uint4(pack_bf16x2(t16[0], t16[1]), pack_bf16x2(t16[2], t16[3]),
+                                            pack_bf16x2(t16[4], t16[5]), pack_bf16x2(t16[6], t16[7]));
+                const uint4 w1 = make_uint4(pack_bf16x2(t16[8], t16[9]), pack_bf16x2(t16[10], t16[11]),
+                                            pack_bf16x2(t16[12], t16[13]), pack_bf16x2(t16[14], t16[15]));
+                *reinterpret_cast<uint4*>(smem + a.oG + g_off((uint32_t)i, (uint32_t)cb, (uint32_t)a.Kp)) = w0;
+                *reinterpret_cast<uint4*>(smem + a.oG + g_off((uint32_t)i, (uint32_t)cb + 8u, (uint32_t)a.Kp)) = w1;
+              }
+            }
           }
         }
         tmem_st_wait();
       }
-      // scores -> mask (keys scanned no later than the row) -> bf16 P in the log-gate area
+      // scores -> mask (keys scanned no later than the row) -> bf16 P in TMEM
       if (!group_and(2, 128, wait_bar(BAR(kBarScFull), (uint32_t)(kb & 1), abort_flag))) {
         ok = false;
         break;
@@ -727,41 +804,36 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
         for (int cb = 0; cb < MC; cb += 32) {
           const bool none = a.g.reverse ? (cb + 31 < rlo) : (cb > rhi);
           const bool all = a.g.reverse ? (cb >= rhi) : (cb + 31 <= rlo);
+          uint32_t sc[2][16];
+          if (!none) tmem_ld_cols<2>(tbase + kColS + lane_base + (uint32_t)cb, 32, sc);
           uint32_t pk[16];
           if (none) {
 #pragma unroll
             for (int q = 0; q < 16; ++q) pk[q] = 0u;
+          } else if (all) {
+#pragma unroll
+            for (int q = 0; q < 32; q += 2) pk[q >> 1] = pack_u2(sc[q >> 4][q & 15], sc[q >> 4][(q & 15) + 1]);
           } else {
-            float sc[32];
-            tmem_ld32(tbase + kColS + lane_base + (uint32_t)cb, sc);
-            if (all) {
 #pragma unroll
-              for (int q = 0; q < 32; q += 2) pk[q >> 1] = pack_bf16x2(sc[q], sc[q + 1]);
-            } else {
-#pragma unroll
-              for (int q = 0; q < 32; q += 2) {
-                const int s0 = cb + q, s1 = cb + q + 1;
-                const bool k0 = a.g.reverse ? (s0 >= i) : (s0 <= i);
-                const bool k1 = a.g.reverse ? (s1 >= i) : (s1 <= i);
-                pk[q >> 1] = pack_bf16x2(k0 ? sc[q] : 0.f, k1 ? sc[q + 1] : 0.f);
-              }
+            for (int q = 0; q < 32; q += 2) {
+              const int s0 = cb + q, s1 = cb + q + 1;
+              const bool k0 = a.g.reverse ? (s0 >= i) : (s0 <= i);
+              const bool k1 = a.g.reverse ? (s1 >= i) : (s1 <= i);
+              const float v0 = __uint_as_float(sc[q >> 4][q & 15]);
+              const float v1 = __uint_as_float(sc[q >> 4][(q & 15) + 1]);
+              pk[q >> 1] = pack_bf16x2(k0 ? v0 : 0.f, k1 ? v1 : 0.f);
             }
           }
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int key = cb + q4 * 8;
-            const uint32_t o = a.oLA + (uint32_t)(key >> 6) * PART128 + sw128((uint32_t)i, (uint32_t)(key & 63) * 2u);
-            *reinterpret_cast<uint4*>(st + o) = make_uint4(pk[q4 * 4], pk[q4 * 4 + 1], pk[q4 * 4 + 2], pk[q4 * 4 + 3]);
-          }
+          // bf16 pairs of keys overwrite score columns this thread has already read.
+          tmem_st16u(tbase + kColS + lane_base + (uint32_t)(cb >> 1), pk);
         }
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(BAR(kBarScEmpty));
       mbar_arrive(BAR(kBarPReady));
       prev_pending = true;
-      prev_s = s;
-      prev_f0 = f0;
+      prev_cf = cf;
       ++kb;
     }
     if (ok) finish_prev();
@@ -783,7 +855,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
 }
 
 struct WsLayout {
-  int NC, NS, G, Kp, Np, nstage;
+  int NC, NS, G, Kp, Np, nstage, mode, rpc, ppr;
   uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oMisc, oBar, oTm;
   size_t smem;
   size_t flag_bytes, agg_bytes, aggg_bytes;
@@ -797,7 +869,21 @@ size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 
 WsLayout ws_layout(const GlaShape& s) {
   WsLayout L;
-  L.NC = (s.T() + MC - 1) / MC;
+  // Chunk geometry (see the kernel's header comment).
+  L.rpc = 1;
+  L.ppr = 1;
+  if (s.dir < 2) {
+    L.mode = 0;
+    L.NC = (s.T() + MC - 1) / MC;
+  } else if (MC % s.Hg == 0) {
+    L.mode = 1;
+    L.rpc = MC / s.Hg;
+    L.NC = (s.Wg + L.rpc - 1) / L.rpc;
+  } else {
+    L.mode = 2;
+    L.ppr = (s.Hg + MC - 1) / MC;
+    L.NC = s.Wg * L.ppr;
+  }
   L.G = kSegChunks;
   L.NS = (L.NC + L.G - 1) / L.G;
   L.Kp = (s.dk + 15) / 16 * 16;
@@ -807,9 +893,9 @@ WsLayout ws_layout(const GlaShape& s) {
   L.oQ = L.oV + (uint32_t)(L.Np / 16) * ATOM32;
   L.oLA = al1024(L.oQ + (uint32_t)(L.Kp / 16) * ATOM32);
   const uint32_t la = (uint32_t)MC * (uint32_t)(s.dk + 4) * 4u;
-  // The score MMA's A operand (K^ as MN-major, M = 128 key channels) reads 8 channel
-  // blocks from oK; the stage is at least that large.
-  L.stage_bytes = al1024(L.oLA + (la > 2 * PART128 ? la : 2 * PART128));
+  // The state MMA's A operand (K^ transposed, MN-major, M = 128 key channels) reads 8
+  // channel blocks from oK; the stage is at least that large.
+  L.stage_bytes = al1024(L.oLA + la > 8 * ATOM32 ? L.oLA + la : 8 * ATOM32);
   const uint32_t gtile = al1024((uint32_t)L.Kp * (uint32_t)L.Np * 2u);
   const uint32_t fixed = gtile + kMaxStages * 512 + 256 + 512 + 256 + 64 + 8 * kNumBars + 16;
   L.nstage = (1024 + 2 * (size_t)L.stage_bytes + fixed <= kMaxSmem) ? 2 : 1;
@@ -853,7 +939,7 @@ EncodeTiledFn encode_fn() {
 // 5-D map over a [B][T][H][d] tensor viewed as (d, H, run position, run, B):
 // raster scans have one run of T positions, column scans Wg runs of Hg.
 bool encode_map(CUtensorMap* m, const void* base, bool f32, int d, int box0, CUtensorMapSwizzle sw, const GlaShape& s,
-                bool column, int box_rows) {
+                bool column, int box_rows, int box_runs) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t e = f32 ? 4 : 2;
@@ -875,20 +961,11 @@ bool encode_map(CUtensorMap* m, const void* base, bool f32, int d, int box0, CUt
   dims[4] = (cuuint64_t)s.B;
   strides[0] = (cuuint64_t)d * e;
   strides[3] = T * H * d * e;
-  const cuuint32_t box[5] = {(cuuint32_t)box0, 1, (cuuint32_t)box_rows, 1, 1};
+  const cuuint32_t box[5] = {(cuuint32_t)box0, 1, (cuuint32_t)box_rows, (cuuint32_t)box_runs, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base),
             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int gcd_int(int x, int y) {
-  while (y) {
-    const int t = x % y;
-    x = y;
-    y = t;
-  }
-  return x;
 }
 
 }  // namespace
@@ -941,29 +1018,24 @@ cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const fl
   a.g = make_geom(s.Hg, s.Wg, s.dir);
 
   const bool column = s.dir >= 2;
-  a.box_rows = column ? gcd_int(s.Hg, MC) : MC;
+  a.mode = L.mode;
+  a.rpc = L.rpc;
+  a.ppr = L.ppr;
+  const int box_rows = L.mode == 1 ? s.Hg : MC, box_runs = L.mode == 1 ? L.rpc : 1;
   TensorMaps tm;
   memset(&tm, 0, sizeof(tm));
-  bool use_tma = a.box_rows >= 8;
-  if (use_tma) {
-    // 16-channel boxes with the 32-byte swizzle land directly in the operand layout;
-    // the kernel's expected transaction bytes assume exactly these boxes.
-    use_tma = encode_map(&tm.q, q, false, s.dk, 16, CU_TENSOR_MAP_SWIZZLE_32B, s, column, a.box_rows) &&
-              encode_map(&tm.k, k, false, s.dk, 16, CU_TENSOR_MAP_SWIZZLE_32B, s, column, a.box_rows) &&
-              encode_map(&tm.v, v, false, s.dv, 16, CU_TENSOR_MAP_SWIZZLE_32B, s, column, a.box_rows) &&
-              encode_map(&tm.la, la, true, s.dk, s.dk + 4, CU_TENSOR_MAP_SWIZZLE_NONE, s, column, a.box_rows);
-  }
+  // 16-channel boxes with the 32-byte swizzle land directly in the operand layout;
+  // the kernel's expected transaction bytes assume exactly these boxes.
+  if (!(encode_map(&tm.q, q, false, s.dk, 16, CU_TENSOR_MAP_SWIZZLE_32B, s, column, box_rows, box_runs) &&
+        encode_map(&tm.k, k, false, s.dk, 16, CU_TENSOR_MAP_SWIZZLE_32B, s, column, box_rows, box_runs) &&
+        encode_map(&tm.v, v, false, s.dv, 16, CU_TENSOR_MAP_SWIZZLE_32B, s, column, box_rows, box_runs) &&
+        encode_map(&tm.la, la, true, s.dk, s.dk + 4, CU_TENSOR_MAP_SWIZZLE_NONE, s, column, box_rows, box_runs)))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(ws, 0, L.flag_bytes, st);  // flags and the ticket counter
   if (e != cudaSuccess) return e;
-  if (use_tma) {
-    e = cudaFuncSetAttribute(gla_ws_fwd<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
-    if (e != cudaSuccess) return e;
-    gla_ws_fwd<true><<<(unsigned)(BH * L.NS), NT, L.smem, st>>>(a, tm);
-  } else {
-    e = cudaFuncSetAttribute(gla_ws_fwd<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
-    if (e != cudaSuccess) return e;
-    gla_ws_fwd<false><<<(unsigned)(BH * L.NS), NT, L.smem, st>>>(a, tm);
-  }
+  e = cudaFuncSetAttribute(gla_ws_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
+  if (e != cudaSuccess) return e;
+  gla_ws_fwd<<<(unsigned)(BH * L.NS), NT, L.smem, st>>>(a, tm);
   return cudaGetLastError();
 }
 

@@ -16,14 +16,6 @@ struct GlaShape {
 
 // ---- bf16 tensor-core path (chunks of 128 scan positions) ----
 constexpr int kChunkTC = 128;
-size_t gla_tc_workspace_bytes(const GlaShape& s);
-cudaError_t gla_tc_forward(const void* q, const void* k, const void* v, const float* la, void* out,
-                           const GlaShape& s, void* workspace, cudaStream_t st);
-
-// ---- bf16 fused single-kernel path (segments of 4 chunks of 128, decoupled look-back) ----
-size_t gla_fused_workspace_bytes(const GlaShape& s);
-cudaError_t gla_fused_forward(const void* q, const void* k, const void* v, const float* la, void* out,
-                              const GlaShape& s, void* workspace, cudaStream_t st);
 
 // ---- bf16 warp-specialised single-kernel path ----
 size_t gla_ws_workspace_bytes(const GlaShape& s);
