@@ -4,7 +4,8 @@
 // o_t = q_t S_t, evaluated chunk-wise in on-chip memory (DiG paper notes,
 // "硬件友好的效率设计": chunks of M tokens computed in SRAM, O(T M D + T D^2)).
 //
-// One CTA per (head, segment of G chunks of 128 scan positions), in ticket order.
+// Work items are (head, segment of G chunks of 128 scan positions), taken in ticket
+// order by persistent CTAs.  Per item:
 //   pass 1  (chunks in reverse scan order)  u_s = log-gates scanned after s up to the
 //           segment end; K^ = k exp(u) (<= 1 for decaying gates); S_seg += K^T V.
 //   look-back  publish (exp(segment gate sum), S_seg); fold earlier segments of the
@@ -16,19 +17,22 @@
 // Chunks whose gates decay by more than e^80 inside the chunk are evaluated token by
 // token from the running state instead (exact).
 //
-// Roles (14 warps, 448 threads), connected by mbarriers:
-//   warp 0      producer: TMA loads of each chunk's q, k, v (32-byte-swizzled 16-channel
-//               boxes, the UMMA operand layout) and log-gates into a ring of stages;
+// Roles (16 warps, 512 threads), connected by mbarriers:
+//   warp 0      producer: takes tickets and posts jobs (pass 1 of the next item, then
+//               pass 2 of the current one); TMA loads of each chunk's q, k, v
+//               (32-byte-swizzled 16-channel boxes, the UMMA operand layout) and
+//               log-gates into a ring of stages;
 //   warp 1      MMA issuer (tcgen05, one thread) and TMEM owner;
-//   warps 2-5   suffix sums of the log-gates, one thread per key channel;
-//   warps 6-9   gates applied in place (K^, Q~), one thread per row;
-//   warps 10-13 TMEM-side work, one thread per TMEM lane: G = Diag(gamma) S, score
-//               masking to bf16 P, output epilogue, look-back, serial path.
+//   warps 2-3   suffix sums of the log-gates, one thread per pair of key channels,
+//               released to the gate warps 32 rows at a time;
+//   warps 4-7   gates applied in place (K^, Q~), one thread per row;
+//   warps 8-11  output group, one thread per TMEM lane: score masking to bf16 P,
+//               G = Diag(gamma) S, output epilogue, serial path;
+//   warps 12-15 look-back group, one thread per TMEM lane.
 // TMEM (512 columns): scores [0,128) -- overwritten by the bf16 P matrix (two keys per
-// column, the A operand of P V) --, O buffer 0 [128,256), running state [256,384),
-// segment aggregate [384,512) -- reused as O buffer 1 once the look-back is done.
-// A stage is free once the MMAs that read it complete, so loads run ahead of the
-// output epilogue.
+// column, the A operand of P V) --, O (two buffers when dv <= 96), and two buffers
+// that each hold an item's segment aggregate, then its incoming state, then its
+// running state.  A stage is free once the MMAs that read it complete.
 //
 // Chunks follow the direction's base order (raster rows, or grid columns for T->B /
 // B->T) and are always cut in forward order; reversed scans visit them backwards and
@@ -49,29 +53,36 @@ namespace dig {
 namespace {
 
 constexpr int MC = kChunkTC;
-constexpr int NT = 448;
-constexpr int kWarpProd = 0, kWarpMma = 1, kWarpSuf = 2, kWarpGate = 6, kWarpEpi = 10;
+constexpr int NT = 512;
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpSuf = 2, kWarpGate = 4, kWarpEpi = 8, kWarpLb = 12;
 constexpr uint32_t ATOM32 = MC * 32u;    // one 16-channel block of a 32B-swizzled 128-row tile
 constexpr float kMaxGateRange = 80.0f;
-constexpr uint32_t kColS = 0, kColO0 = 128, kColState = 256, kColSeg = 384;
+constexpr uint32_t kColS = 0;
 constexpr uint32_t kLayoutSW32 = 6;
 constexpr int kMaxStages = 2;
 
 // mbarrier indices (8 bytes each)
 enum {
-  kBarFull = 0,                          // [S]  tiles landed
-  kBarSuf = kBarFull + kMaxStages,       // [S]  suffix sums done (128 arrivals)
-  kBarGate = kBarSuf + kMaxStages,       // [S]  gates applied (128 arrivals)
-  kBarEmpty = kBarGate + kMaxStages,     // [S]  stage free (MMA commit, or the serial path)
-  kBarScFull = kBarEmpty + kMaxStages,   // score MMA done
-  kBarScEmpty,                           // scores read (128 arrivals)
-  kBarPReady,                            // P and G written (128 arrivals)
-  kBarBatch0,                            // [2] output MMAs done
-  kBarOEmpty0 = kBarBatch0 + 2,          // [2] output buffer read (128 arrivals)
-  kBarSegDone = kBarOEmpty0 + 2,         // pass-1 MMAs done
-  kBarDrain,                             // all MMAs of the CTA done (teardown)
+  kBarFull = 0,                       // [S]  tiles landed (or an end-of-stream job posted)
+  kBarSuf = kBarFull + kMaxStages,    // [S][4] suffix sums of a 32-row quarter done (64 arrivals)
+  kBarGate = kBarSuf + 4 * kMaxStages,  // [S]  gates applied (128 arrivals)
+  kBarEmpty = kBarGate + kMaxStages,  // [S]  stage free (MMA commit, or the serial path)
+  kBarMail = kBarEmpty + kMaxStages,  // pass-2 job handed to the output group
+  kBarScFull,                         // score MMA done
+  kBarScEmpty,                        // job taken and scores read (128 arrivals)
+  kBarPReady,                         // P written (128 arrivals)
+  kBarGReady,                         // state scaled and G written (128 arrivals)
+  kBarBatch,                          // [2] output and state MMAs done, per O buffer
+  kBarOFree = kBarBatch + 2,          // [2] O buffer read (128 arrivals)
+  kBarSegDone = kBarOFree + 2,        // [2] pass-1 MMAs of an item done (or end of stream)
+  kBarSinReady = kBarSegDone + 2,     // [2] look-back done: incoming state in the buffer
+  kBarSegFree = kBarSinReady + 2,     // [2] pass 2 done with the buffer
+  kBarDrain = kBarSegFree + 2,        // all MMAs of the CTA done (teardown)
   kNumBars
 };
+
+// Jobs posted by the producer, one per stage use.
+enum { kJobP1 = 1, kJobP2 = 2, kJobEnd = 3 };
 
 struct WsArgs {
   const __nv_bfloat16* q;
@@ -84,12 +95,32 @@ struct WsArgs {
   float* incl_S;  // [BH][NS][dv/4][dk][4]  state after the segment
   int* flags;     // [BH][NS]               0 nothing, 1 aggregate, 2 inclusive
   int* ticket;
-  int H, BH, dk, dv, NC, NS, G;
-  int Kp, Np, nstage;
+  int H, BH, dk, dv, NC, NS, G, items;
+  int Kp, Np, nstage, nO;
+  uint32_t colO0, colO1, colSeg0, colSeg1;
   int mode, rpc, ppr;  // chunk geometry: 0 raster, 1 whole columns (rpc per chunk), 2 column pieces (ppr per column)
-  uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oMisc, oBar, oTm;
+  uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oMisc, oJob, oMail, oItem, oBar, oTm;
   ScanGeom g;
+  __device__ __forceinline__ uint32_t col_seg(int buf) const { return buf ? colSeg1 : colSeg0; }
+  __device__ __forceinline__ uint32_t col_o(int ob) const { return ob ? colO1 : colO0; }
 };
+
+// One work item: a segment of G chunks of one (batch, head).
+struct Item {
+  int seg, bh, b, h, c0, n;
+  int64_t seg_id;
+};
+__device__ __forceinline__ Item decode_item(const WsArgs& a, int item) {
+  Item it;
+  it.seg = item / a.BH;
+  it.bh = item - it.seg * a.BH;
+  it.b = it.bh / a.H;
+  it.h = it.bh - it.b * a.H;
+  it.c0 = it.seg * a.G;
+  it.n = min(a.G, a.NC - it.c0);
+  it.seg_id = (int64_t)it.bh * a.NS + it.seg;
+  return it;
+}
 
 struct TensorMaps {
   CUtensorMap q, k, v, la;
@@ -133,11 +164,21 @@ __device__ __forceinline__ bool group_and(uint32_t id, uint32_t n, bool v) {
       : "memory");
   return r != 0;
 }
+// Group-wide OR over a named barrier.
+__device__ __forceinline__ bool group_or(uint32_t id, uint32_t n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_cnt(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
@@ -207,13 +248,24 @@ __device__ __forceinline__ uint32_t pack_u2(uint32_t x, uint32_t y) {
   return pack_bf16x2(__uint_as_float(x), __uint_as_float(y));
 }
 
+// TMA tile load with an L2 eviction-priority policy (from createpolicy).
 __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
-                                            int c4, uint32_t bar) {
+                                            int c4, uint32_t bar, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], "
-      "[%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar)
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3, "
+      "%4, %5, %6}], [%7], %8;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar), "l"(policy)
       : "memory");
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 
 // Bounded wait on an mbarrier phase that also gives up when another role has
@@ -279,8 +331,6 @@ __device__ __forceinline__ void chunk_box(const WsArgs& a, int cf, int& y, int& 
   }
 }
 
-__device__ __forceinline__ int job_chunk(int j, int c0, int n) { return j < n ? c0 + n - 1 - j : c0 + (j - n); }
-
 // ---------------------------------------------------------------------------
 // Producer
 // ---------------------------------------------------------------------------
@@ -291,18 +341,22 @@ __device__ void tma_job(const WsArgs& a, const TensorMaps& tm, uint32_t st, uint
   mbar_expect_tx(bar, bytes);
   int y, x;
   chunk_box(a, cf, y, x);
+  // Pass 2 is the last use of every tile: mark its lines first to go, so that the
+  // pass-1 tiles waiting for their second read stay in L2.
+  const uint64_t pol = with_q ? l2_policy_evict_first() : l2_policy_evict_normal();
   for (int cb = 0; cb < (a.Kp >> 4); ++cb) {
-    tma_load_5d(st + a.oK + (uint32_t)cb * ATOM32, &tm.k, cb * 16, h, y, x, b, bar);
-    if (with_q) tma_load_5d(st + a.oQ + (uint32_t)cb * ATOM32, &tm.q, cb * 16, h, y, x, b, bar);
+    tma_load_5d(st + a.oK + (uint32_t)cb * ATOM32, &tm.k, cb * 16, h, y, x, b, bar, pol);
+    if (with_q) tma_load_5d(st + a.oQ + (uint32_t)cb * ATOM32, &tm.q, cb * 16, h, y, x, b, bar, pol);
   }
-  for (int cb = 0; cb < (a.Np >> 4); ++cb) tma_load_5d(st + a.oV + (uint32_t)cb * ATOM32, &tm.v, cb * 16, h, y, x, b, bar);
-  tma_load_5d(st + a.oLA, &tm.la, 0, h, y, x, b, bar);
+  for (int cb = 0; cb < (a.Np >> 4); ++cb)
+    tma_load_5d(st + a.oV + (uint32_t)cb * ATOM32, &tm.v, cb * 16, h, y, x, b, bar, pol);
+  tma_load_5d(st + a.oLA, &tm.la, 0, h, y, x, b, bar, pol);
 }
 
 // ---------------------------------------------------------------------------
 // Serial path (wide chunks), run by the 128 TMEM-side threads: lane i owns state
 // row i; 16 value columns at a time, outputs reduced over lanes with shuffles.
-// q, k are still the raw (unscaled) swizzled tiles.
+// The stage's q, k tiles may already be gated, so raw q, k come from global memory.
 // ---------------------------------------------------------------------------
 __device__ void chunk_serial(const WsArgs& a, const uint8_t* st, float* red, uint32_t tstate, uint32_t lane_base,
                              int i, int cf, int b, int h) {
@@ -313,16 +367,29 @@ __device__ void chunk_serial(const WsArgs& a, const uint8_t* st, float* red, uin
     if (i >= a.dk)
 #pragma unroll
       for (int q = 0; q < 16; ++q) s[q] = 0.f;
-    for (int step = 0; step < MC; ++step) {
+    // alpha, k and q of the next row are fetched one step ahead.
+    auto fetch = [&](int step, float& al, float& kq, float& qi) -> int {
       const int r = a.g.reverse ? (MC - 1 - step) : step;
       const int t = row_token(a, cf, r);
-      if (t < 0) continue;  // padding row: uniform
-      float alpha = 1.f, kq = 0.f, qi = 0.f;
-      if (i < a.dk) {
-        alpha = __expf(__ldg(a.la + (((int64_t)b * a.g.T + t) * a.H + h) * a.dk + i));
-        kq = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(st + a.oK + sw32_off((uint32_t)r, (uint32_t)i)));
-        qi = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(st + a.oQ + sw32_off((uint32_t)r, (uint32_t)i)));
+      al = 1.f;
+      kq = 0.f;
+      qi = 0.f;
+      if (t >= 0 && i < a.dk) {
+        const int64_t o = (((int64_t)b * a.g.T + t) * a.H + h) * a.dk + i;
+        al = __expf(__ldg(a.la + o));
+        kq = __bfloat162float(a.k[o]);
+        qi = __bfloat162float(a.q[o]);
       }
+      return t;
+    };
+    float n_al, n_kq, n_qi;
+    int n_t = fetch(0, n_al, n_kq, n_qi);
+    for (int step = 0; step < MC; ++step) {
+      const int r = a.g.reverse ? (MC - 1 - step) : step;
+      const int t = n_t;
+      const float alpha = n_al, kq = n_kq, qi = n_qi;
+      if (step + 1 < MC) n_t = fetch(step + 1, n_al, n_kq, n_qi);
+      if (t < 0) continue;  // padding row: uniform
       float vv[16];
       {
         const uint4 w0 = *reinterpret_cast<const uint4*>(st + a.oV + sw32_off((uint32_t)r, (uint32_t)(cb * 16)));
@@ -358,12 +425,173 @@ __device__ void chunk_serial(const WsArgs& a, const uint8_t* st, float* red, uin
   tmem_st_wait();
 }
 
+// Adds coef * src[pid] (an aggregate or inclusive state in the quad layout) to the
+// state rows this thread owns in TMEM (tSt), 80 columns per global round trip; also
+// returns coef * gamma[pid] when want_gam (the coefficient for the next predecessor).
+__device__ __forceinline__ float fold_state(const WsArgs& a, const float* src, int64_t pid, float coef, uint32_t tSt,
+                                            int i, bool want_gam) {
+  const int DQ = a.dv >> 2;
+  const float g = (want_gam && i < a.dk) ? __ldcg(a.agg_g + pid * a.dk + i) : 1.f;
+#pragma unroll 1
+  for (int c0 = 0; c0 < a.Np; c0 += 80) {
+    float4 x[20];
+#pragma unroll
+    for (int q = 0; q < 20; ++q) {
+      const int jq = c0 / 4 + q;
+      x[q] = (i < a.dk && jq < DQ) ? __ldcg(reinterpret_cast<const float4*>(src + ((pid * DQ + jq) * a.dk + i) * 4))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int c4 = 0; c4 < 5; ++c4) {
+      const int cb = c0 + 16 * c4;
+      if (cb < a.Np) {
+        uint32_t t[1][16];
+        tmem_ld_cols<1>(tSt + (uint32_t)cb, 16, t);
+        float t16[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          t16[4 * q] = fmaf(coef, x[4 * c4 + q].x, __uint_as_float(t[0][4 * q]));
+          t16[4 * q + 1] = fmaf(coef, x[4 * c4 + q].y, __uint_as_float(t[0][4 * q + 1]));
+          t16[4 * q + 2] = fmaf(coef, x[4 * c4 + q].z, __uint_as_float(t[0][4 * q + 2]));
+          t16[4 * q + 3] = fmaf(coef, x[4 * c4 + q].w, __uint_as_float(t[0][4 * q + 3]));
+        }
+        tmem_st16(tSt + (uint32_t)cb, t16);
+      }
+    }
+  }
+  tmem_st_wait();
+  return coef * g;
+}
+
+// Look-back of one item, run by the 128 look-back threads (lane i = key channel).
+// tSeg holds the item's segment aggregate when called and its incoming state on
+// return.  Steps: publish the aggregate and exp(segment gate sum) (flag 1); fold
+// earlier segments of the same head, nearest first, into the incoming state until an
+// inclusive state is found (decoupled look-back); publish this segment's inclusive
+// state Diag(gamma_seg) S_in + aggregate (flag 2).  Predecessor flags are read 32 at a
+// time by one warp; sLb is a small shared scratch.
+__device__ __forceinline__ void lookback(const WsArgs& a, int seg, int bh, int64_t seg_id, uint32_t tSeg, int i, int e,
+                                         float gs, volatile int* sLb) {
+  const int DQ = a.dv >> 2;
+  const int lane = e & 31;
+  if (i < a.dk) a.agg_g[seg_id * a.dk + i] = gs;
+#pragma unroll 1
+  for (int c0 = 0; c0 < a.Np; c0 += 32) {
+    uint32_t t[2][16];
+    tmem_ld_cols<2>(tSeg + (uint32_t)c0, a.Np - c0, t);
+    if (i < a.dk) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int jq = c0 / 4 + q;
+        if (jq < DQ)
+          *reinterpret_cast<float4*>(a.agg_S + ((seg_id * DQ + jq) * a.dk + i) * 4) =
+              make_float4(__uint_as_float(t[q >> 2][4 * (q & 3)]), __uint_as_float(t[q >> 2][4 * (q & 3) + 1]),
+                          __uint_as_float(t[q >> 2][4 * (q & 3) + 2]), __uint_as_float(t[q >> 2][4 * (q & 3) + 3]));
+      }
+    }
+    // The columns now accumulate the incoming state.
+    float z[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) z[q] = 0.f;
+    tmem_st16(tSeg + (uint32_t)c0, z);
+    if (c0 + 16 < a.Np) tmem_st16(tSeg + (uint32_t)(c0 + 16), z);
+  }
+  tmem_st_wait();
+  named_sync(3, 128);
+  if (e == 0) {
+    __threadfence();
+    st_release(a.flags + seg_id, 1);
+  }
+  float coef = 1.f;
+  int base = seg - 1;  // nearest predecessor not folded yet
+  while (base >= 0) {
+    if (e < 32) {
+      // Wait until the window [base-31, base] shows an inclusive state (or the start of
+      // the sequence) with aggregates everywhere before it, or 32 aggregates.
+      int nagg = -1, incl = 0;
+      const long long t0 = clock64();
+      for (;;) {
+        const int p = base - lane;
+        const int fl = p >= 0 ? (int)ld_acquire(a.flags + (int64_t)bh * a.NS + p) : 2;
+        const uint32_t m2 = __ballot_sync(0xffffffffu, fl == 2);
+        const uint32_t m0 = __ballot_sync(0xffffffffu, fl == 0);
+        const int first2 = m2 ? __ffs(m2) - 1 : 32;
+        const uint32_t before = first2 == 32 ? 0xffffffffu : ((1u << first2) - 1u);
+        if ((m0 & before) == 0) {
+          nagg = first2;
+          incl = first2 < 32 && base - first2 >= 0;
+          break;
+        }
+        if (clock64() - t0 > kWaitCycles) {
+          if (lane == 0) report_status(GLA_ERR_TIMEOUT);
+          break;
+        }
+        __nanosleep(32);
+      }
+      if (lane == 0) {
+        sLb[0] = nagg;
+        sLb[1] = incl;
+      }
+    }
+    named_sync(3, 128);
+    const int nagg = sLb[0], incl = sLb[1];
+    named_sync(3, 128);
+    if (nagg < 0) break;  // timed out (recorded)
+    for (int m = 0; m < nagg; ++m) {
+      const int64_t pid = (int64_t)bh * a.NS + base - m;
+      coef = fold_state(a, a.agg_S, pid, coef, tSeg, i, true);
+    }
+    if (incl) {
+      fold_state(a, a.incl_S, (int64_t)bh * a.NS + base - nagg, coef, tSeg, i, false);
+      break;
+    }
+    base -= nagg;
+  }
+  // Inclusive state of this segment: Diag(gamma_seg) S_in + aggregate (re-read from
+  // the copy this thread published above).
+#pragma unroll 1
+  for (int c0 = 0; c0 < a.Np; c0 += 32) {
+    float4 g[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int jq = c0 / 4 + q;
+      g[q] = (i < a.dk && jq < DQ) ? __ldcg(reinterpret_cast<const float4*>(a.agg_S + ((seg_id * DQ + jq) * a.dk + i) * 4))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    uint32_t sin[2][16];
+    tmem_ld_cols<2>(tSeg + (uint32_t)c0, a.Np - c0, sin);
+    if (i < a.dk) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int jq = c0 / 4 + q;
+        if (jq < DQ) {
+          const uint32_t* v = &sin[q >> 2][4 * (q & 3)];
+          *reinterpret_cast<float4*>(a.incl_S + ((seg_id * DQ + jq) * a.dk + i) * 4) =
+              make_float4(fmaf(gs, __uint_as_float(v[0]), g[q].x), fmaf(gs, __uint_as_float(v[1]), g[q].y),
+                          fmaf(gs, __uint_as_float(v[2]), g[q].z), fmaf(gs, __uint_as_float(v[3]), g[q].w));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  named_sync(3, 128);
+  if (e == 0) {
+    __threadfence();
+    st_release(a.flags + seg_id, 2);
+  }
+}
+
 __device__ __forceinline__ uint32_t align1024(uint32_t x) { return (x + 1023u) & ~1023u; }
 
 // ---------------------------------------------------------------------------
-// The kernel
+// The kernel (persistent: each CTA takes items from a ticket counter until none
+// are left).  The producer posts, per item, its pass-1 jobs and then the pass-2
+// jobs of the previous item; the look-back group works on an item while pass 1 of
+// the next one and pass 2 of the previous one proceed.  Item k uses aggregate buffer
+// k % 2, which holds its aggregate after pass 1, its incoming state after the
+// look-back and its running state during pass 2.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid_constant__ TensorMaps tm) {
+__global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsArgs a, const __grid_constant__ TensorMaps tm) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t sbase = align1024(raw_u32);
@@ -371,10 +599,14 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* sBL = reinterpret_cast<float*>(smem + a.oBL);      // [S][128] chunk gate sums
-  volatile int* sWide = reinterpret_cast<volatile int*>(smem + a.oWide);  // [S] + [S][4] per-warp flags
-  float* sGam = reinterpret_cast<float*>(smem + a.oGam);    // [128] exp(segment gate sum)
+  volatile int* sWide = reinterpret_cast<volatile int*>(smem + a.oWide);  // [S] chunk evaluated serially
+  float* sGam = reinterpret_cast<float*>(smem + a.oGam);    // [2][128] exp(segment gate sum)
   float* red = reinterpret_cast<float*>(smem + a.oRed);     // serial-path reduction [4][16]
-  volatile int* sMisc = reinterpret_cast<volatile int*>(smem + a.oMisc);  // [0] item [1] abort [2] flag
+  // [0] first item [1] abort [2] look-back flag [3] jobs posted [4] jobs taken [5] end item index
+  volatile int* sMisc = reinterpret_cast<volatile int*>(smem + a.oMisc);
+  volatile int* sJob = reinterpret_cast<volatile int*>(smem + a.oJob);    // [S][4] kind, item, j, buf
+  volatile int* sMail = reinterpret_cast<volatile int*>(smem + a.oMail);  // [4]    stage, wide, item, j
+  volatile int* sItem = reinterpret_cast<volatile int*>(smem + a.oItem);  // [2] item per buffer, [2] same for pass 2
   const uint32_t bars = sbase + a.oBar;
   auto BAR = [&](int idx) -> uint32_t { return bars + 8u * (uint32_t)idx; };
   volatile int* abort_flag = sMisc + 1;
@@ -386,73 +618,172 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
   if (tid == 0) {
     for (int s = 0; s < a.nstage; ++s) {
       mbar_init(BAR(kBarFull + s), 1);
-      mbar_init(BAR(kBarSuf + s), 128);
+      for (int qd = 0; qd < 4; ++qd) mbar_init(BAR(kBarSuf + 4 * s + qd), 64);
       mbar_init(BAR(kBarGate + s), 128);
       mbar_init(BAR(kBarEmpty + s), 1);
     }
+    mbar_init(BAR(kBarMail), 1);
     mbar_init(BAR(kBarScFull), 1);
     mbar_init(BAR(kBarScEmpty), 128);
     mbar_init(BAR(kBarPReady), 128);
-    mbar_init(BAR(kBarBatch0), 1);
-    mbar_init(BAR(kBarBatch0 + 1), 1);
-    mbar_init(BAR(kBarOEmpty0), 128);
-    mbar_init(BAR(kBarOEmpty0 + 1), 128);
-    mbar_init(BAR(kBarSegDone), 1);
+    mbar_init(BAR(kBarGReady), 128);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(BAR(kBarBatch + q), 1);
+      mbar_init(BAR(kBarOFree + q), 128);
+      mbar_init(BAR(kBarSegDone + q), 1);
+      mbar_init(BAR(kBarSinReady + q), 1);
+      mbar_init(BAR(kBarSegFree + q), 1);
+    }
     mbar_init(BAR(kBarDrain), 1);
     fence_mbar_init();
     sMisc[0] = atomicAdd(a.ticket, 1);
-    sMisc[1] = 0;  // abort
-    sMisc[3] = 0;  // load jobs issued
-    sMisc[4] = 0;  // load jobs consumed
+    sMisc[1] = 0;
+    sMisc[3] = 0;
+    sMisc[4] = 0;
+    sMisc[5] = 0x7fffffff;
   }
   for (int x = tid; x < kMaxStages * 128; x += NT) sBL[x] = 0.f;  // rows >= dk: gamma = 1
-  for (int x = tid; x < 128; x += NT) sGam[x] = 1.f;
+  for (int x = tid; x < 2 * 128; x += NT) sGam[x] = 1.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(smem + a.oTm);
-  const int item = sMisc[0];
-  const int seg = item / a.BH, bh = item - seg * a.BH;
-  const int b = bh / a.H, h = bh - b * a.H;
-  const int c0 = seg * a.G;
-  const int n = min(a.G, a.NC - c0);
-  const int64_t seg_id = (int64_t)bh * a.NS + seg;
-  const int njob = 2 * n;
   const int S = a.nstage;
+  const bool has_work = sMisc[0] < a.items;
 
-  if (warp == kWarpProd) {
+  if (!has_work) {
+    // every ticket was taken by earlier CTAs
+  } else if (warp == kWarpProd) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      for (int j = 0; j < njob; ++j) {
-        const int s = j % S, k = j / S;
-        if (k > 0 && !wait_bar(BAR(kBarEmpty + s), (uint32_t)((k - 1) & 1), abort_flag)) break;
-        const uint32_t st = sbase + (uint32_t)s * a.stage_bytes;
-        tma_job(a, tm, st, BAR(kBarFull + s), fwd_chunk(a, job_chunk(j, c0, n)), j >= n, b, h);
-        sMisc[3] = j + 1;
+      int jc = 0;
+      auto post = [&](int kind, int item, int j, int buf) -> bool {
+        const int s = jc % S, use = jc / S;
+        if (use > 0 && !wait_bar(BAR(kBarEmpty + s), (uint32_t)((use - 1) & 1), abort_flag)) return false;
+        sJob[4 * s] = kind;
+        sJob[4 * s + 1] = item;
+        sJob[4 * s + 2] = j;
+        sJob[4 * s + 3] = buf;
+        if (kind == kJobEnd) {
+          mbar_arrive(BAR(kBarFull + s));
+        } else {
+          const Item it = decode_item(a, item);
+          const int c = kind == kJobP1 ? it.c0 + it.n - 1 - j : it.c0 + j;  // pass 1 walks backwards
+          tma_job(a, tm, sbase + (uint32_t)s * a.stage_bytes, BAR(kBarFull + s), fwd_chunk(a, c), kind == kJobP2,
+                  it.b, it.h);
+        }
+        sMisc[3] = ++jc;
+        return true;
+      };
+      auto post_p1 = [&](int item, int k) -> bool {
+        const int buf = k & 1;
+        // sItem[buf] is rewritten once the look-back of item k - 2 has read it.
+        if (k >= 2 && !wait_bar(BAR(kBarSinReady + buf), (uint32_t)(((k >> 1) - 1) & 1), abort_flag)) return false;
+        sItem[buf] = item;
+        const int n = decode_item(a, item).n;
+        for (int j = 0; j < n; ++j)
+          if (!post(kJobP1, item, j, buf)) return false;
+        return true;
+      };
+      auto post_p2 = [&](int item, int k) -> bool {
+        const int n = decode_item(a, item).n;
+        for (int j = 0; j < n; ++j)
+          if (!post(kJobP2, item, j, k & 1)) return false;
+        return true;
+      };
+      int cur = sMisc[0];
+      bool ok = post_p1(cur, 0);
+      for (int k = 0; ok; ++k) {
+        const int nxt = atomicAdd(a.ticket, 1);
+        const bool more = nxt < a.items;
+        if (more) ok = post_p1(nxt, k + 1);
+        if (ok) ok = post_p2(cur, k);
+        if (!ok) break;
+        if (!more) {
+          post(kJobEnd, -1, 0, 0);
+          break;
+        }
+        cur = nxt;
       }
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
+    // Pass-2 order: S(j) ... P V(j), then S(j+1) when chunk j+1 is already gated, then
+    // Q~ G(j) and K^T V(j), so that the masking of chunk j+1 overlaps the state MMAs of
+    // chunk j.
     if (lane == 0) {
-      int kb = 0;
-      for (int j = 0; j < njob; ++j) {
-        const int s = j % S, k = j / S;
-        if (!wait_bar(BAR(kBarGate + s), (uint32_t)(k & 1), abort_flag)) break;
+      int kb = 0, jb = 0, km = 0;  // non-serial pass-2 jobs, pass-2 jobs, items through pass 1
+      bool tail = false;           // Q~ G and K^T V of the last non-serial job still to issue
+      int t_s = 0, t_buf = 0, t_kb = 0;
+      bool ok = true;
+      auto issue_tail = [&]() -> bool {
+        if (!tail) return true;
+        tail = false;
+        if (!wait_bar(BAR(kBarGReady), (uint32_t)(t_kb & 1), abort_flag)) return false;
         tc_fence_after();
+        const int ob = t_kb % a.nO;
+        const uint32_t st = sbase + (uint32_t)t_s * a.stage_bytes;
+        const uint32_t id_pv = idesc_bf16_f32(MC, a.Np, false, true);
+#pragma unroll 1
+        for (int kk = 0; kk < (a.Kp >> 4); ++kk)
+          umma_ss(tbase + a.col_o(ob), desc_sw32(st + a.oQ + (uint32_t)kk * ATOM32, 16u, 256u),
+                  desc_sw32(sbase + a.oG + (uint32_t)kk * 512u, (uint32_t)a.Kp * 32u, 256u), id_pv, 1u);
+        const uint32_t id_s = idesc_bf16_f32(MC, a.Np, true, true);
+#pragma unroll 1
+        for (int kk = 0; kk < MC / 16; ++kk)
+          umma_ss(tbase + a.col_seg(t_buf), desc_sw32(st + a.oK + (uint32_t)kk * 512u, ATOM32, 256u),
+                  desc_sw32(st + a.oV + (uint32_t)kk * 512u, ATOM32, 256u), id_s, 1u);
+        umma_commit(BAR(kBarBatch + ob));
+        umma_commit(BAR(kBarEmpty + t_s));
+        return true;
+      };
+      for (int jc = 0; ok; ++jc) {
+        const int s = jc % S, use = jc / S;
+        // The deferred MMAs go first unless this job is already gated: its stage may be
+        // waiting for them.
+        if (tail && !mbar_try_wait(BAR(kBarGate + s), (uint32_t)(use & 1)) && !issue_tail()) break;
+        if (!wait_bar(BAR(kBarGate + s), (uint32_t)(use & 1), abort_flag)) break;
+        tc_fence_after();
+        const int kind = sJob[4 * s], item = sJob[4 * s + 1], j = sJob[4 * s + 2], buf = sJob[4 * s + 3];
+        if (kind != kJobP2 && !issue_tail()) break;
+        if (kind == kJobEnd) {
+          sMisc[5] = km;  // the look-back and output groups stop at item km
+          mbar_arrive(BAR(kBarSegDone + (km & 1)));
+          break;
+        }
         const uint32_t st = sbase + (uint32_t)s * a.stage_bytes;
-        if (j < n) {
+        const int n = decode_item(a, item).n;
+        if (kind == kJobP1) {
+          // The buffer is free once pass 2 of item km - 2 is done with it.
+          if (j == 0 && km >= 2 && !wait_bar(BAR(kBarSegFree + buf), (uint32_t)(((km >> 1) - 1) & 1), abort_flag))
+            break;
+          tc_fence_after();
           const uint32_t id = idesc_bf16_f32(MC, a.Np, true, true);
 #pragma unroll 1
           for (int kk = 0; kk < MC / 16; ++kk)
-            umma_ss(tbase + kColSeg, desc_sw32(st + a.oK + (uint32_t)kk * 512u, ATOM32, 256u),
+            umma_ss(tbase + a.col_seg(buf), desc_sw32(st + a.oK + (uint32_t)kk * 512u, ATOM32, 256u),
                     desc_sw32(st + a.oV + (uint32_t)kk * 512u, ATOM32, 256u), id, (j > 0 || kk > 0) ? 1u : 0u);
           umma_commit(BAR(kBarEmpty + s));
-          if (j == n - 1) umma_commit(BAR(kBarSegDone));
+          if (j == n - 1) {
+            umma_commit(BAR(kBarSegDone + buf));
+            ++km;
+          }
           continue;
         }
-        if (sWide[s]) continue;  // evaluated serially by the TMEM-side warps, which free the stage
-        if (kb > 0 && !wait_bar(BAR(kBarScEmpty), (uint32_t)((kb - 1) & 1), abort_flag)) break;
+        // pass 2: hand the job to the output group once it has taken the previous one
+        if (jb > 0 && !wait_bar(BAR(kBarScEmpty), (uint32_t)((jb - 1) & 1), abort_flag)) break;
         tc_fence_after();
+        const int wide = sWide[s];
+        sMail[0] = s;
+        sMail[1] = wide;
+        sMail[2] = item;
+        sMail[3] = j;
+        mbar_arrive(BAR(kBarMail));
+        ++jb;
+        if (wide) {  // evaluated serially by the output group, which frees the stage
+          if (!issue_tail()) break;
+          continue;
+        }
         {
           const uint32_t id = idesc_bf16_f32(MC, MC, false, false);
 #pragma unroll 1
@@ -461,30 +792,25 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
                     desc_sw32(st + a.oK + (uint32_t)kk * ATOM32, 16u, 256u), id, kk > 0 ? 1u : 0u);
           umma_commit(BAR(kBarScFull));
         }
+        if (!issue_tail()) break;
         if (!wait_bar(BAR(kBarPReady), (uint32_t)(kb & 1), abort_flag)) break;
-        const int ob = kb & 1;
-        if (kb >= 2 && !wait_bar(BAR(kBarOEmpty0 + ob), (uint32_t)(((kb >> 1) - 1) & 1), abort_flag)) break;
+        const int ob = kb % a.nO;
+        if (kb >= a.nO && !wait_bar(BAR(kBarOFree + ob), (uint32_t)(((kb / a.nO) - 1) & 1), abort_flag)) break;
         tc_fence_after();
         {
-          const uint32_t tO = tbase + (ob ? kColSeg : kColO0);
           const uint32_t id_pv = idesc_bf16_f32(MC, a.Np, false, true);
 #pragma unroll 1
           for (int kk = 0; kk < MC / 16; ++kk)  // P is bf16 in the score columns
-            umma_ts(tO, tbase + kColS + (uint32_t)(kk * 8), desc_sw32(st + a.oV + (uint32_t)kk * 512u, ATOM32, 256u),
-                    id_pv, kk > 0 ? 1u : 0u);
-#pragma unroll 1
-          for (int kk = 0; kk < (a.Kp >> 4); ++kk)
-            umma_ss(tO, desc_sw32(st + a.oQ + (uint32_t)kk * ATOM32, 16u, 256u),
-                    desc_sw32(sbase + a.oG + (uint32_t)kk * 512u, (uint32_t)a.Kp * 32u, 256u), id_pv, 1u);
-          const uint32_t id_s = idesc_bf16_f32(MC, a.Np, true, true);
-#pragma unroll 1
-          for (int kk = 0; kk < MC / 16; ++kk)
-            umma_ss(tbase + kColState, desc_sw32(st + a.oK + (uint32_t)kk * 512u, ATOM32, 256u),
-                    desc_sw32(st + a.oV + (uint32_t)kk * 512u, ATOM32, 256u), id_s, 1u);
-          umma_commit(BAR(kBarBatch0 + ob));
-          umma_commit(BAR(kBarEmpty + s));
+            umma_ts(tbase + a.col_o(ob), tbase + kColS + (uint32_t)(kk * 8),
+                    desc_sw32(st + a.oV + (uint32_t)kk * 512u, ATOM32, 256u), id_pv, kk > 0 ? 1u : 0u);
         }
+        tail = true;
+        t_s = s;
+        t_buf = buf;
+        t_kb = kb;
         ++kb;
+        // With one stage, or at the end of an item, the next job cannot come first.
+        if ((S == 1 || j == n - 1) && !issue_tail()) break;
       }
       // Every MMA of this CTA completes before TMEM is released (bounded).
       umma_commit(BAR(kBarDrain));
@@ -494,66 +820,90 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
     }
   } else if (warp < kWarpGate) {
     // ------------------------------------------------------------ suffix sums
-    const int i = tid - 32 * kWarpSuf;  // key channel
-    const int sw = warp - kWarpSuf;
-    float off = 0.f, pos_seg = 0.f;
-    for (int j = 0; j < njob; ++j) {
-      const int s = j % S, k = j / S;
-      if (!group_and(1, 128, wait_bar(BAR(kBarFull + s), (uint32_t)(k & 1), abort_flag))) break;
-      if (i == 0) sMisc[4] = j + 1;
-      float* sLA = reinterpret_cast<float*>(smem + (uint32_t)s * a.stage_bytes + a.oLA);
-      const bool pass1 = j < n;
-      int wide = 0;
-      if (i < a.dk) {
-        const int pw = a.dk + 4;
-        float* ptr = sLA + (a.g.reverse ? 0 : (MC - 1)) * pw + i;  // last scanned row first
-        const int step = a.g.reverse ? pw : -pw;
-        const float base = pass1 ? off : 0.f;
-        float acc = 0.f, ab = 0.f, po = 0.f;
-        // Sixteen loads are issued before their stores so that they overlap.
-#pragma unroll 1
-        for (int p0 = 0; p0 < MC; p0 += 16) {
-          float x[16];
-#pragma unroll
-          for (int q = 0; q < 16; ++q) x[q] = ptr[q * step];
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            ptr[q * step] = acc + base;
-            acc += x[q];
-            ab += fabsf(x[q]);
-            po += fmaxf(x[q], 0.f);
-          }
-          ptr += 16 * step;
-        }
-        sBL[s * 128 + i] = acc;
-        if (pass1) {
-          off += acc;
-          pos_seg += po;
-          if (j == n - 1) {
-            if (!(pos_seg <= kMaxGateRange)) report_status(GLA_ERR_RANGE);
-            sGam[i] = __expf(off);
-          }
-        } else {
-          wide = !(ab <= kMaxGateRange);
-        }
+    // In place over the log-gate tile: u_r = base + sum of the log-gates scanned after
+    // row r (base = the later chunks of the segment in pass 1, 0 in pass 2).  Rows are
+    // walked from the last scanned one; each finished quarter of 32 rows is released
+    // to the gate warp that owns it.
+    const int c = 2 * (tid - 32 * kWarpSuf);  // key channels c, c + 1
+    float2 off = make_float2(0.f, 0.f);
+    int ks = 0;  // items through pass 1
+    for (int jc = 0;; ++jc) {
+      const int s = jc % S, use = jc / S;
+      if (!group_and(1, 64, wait_bar(BAR(kBarFull + s), (uint32_t)(use & 1), abort_flag))) break;
+      if (c == 0) sMisc[4] = jc + 1;
+      const int kind = sJob[4 * s], j = sJob[4 * s + 2], buf = sJob[4 * s + 3];
+      if (kind == kJobEnd) {
+        for (int qd = 0; qd < 4; ++qd) mbar_arrive(BAR(kBarSuf + 4 * s + qd));
+        break;
       }
-      const int any = __any_sync(0xffffffffu, wide);
-      if (lane == 0) sWide[kMaxStages + s * 4 + sw] = any;
-      named_sync(1, 128);
-      if (i == 0)
-        sWide[s] = sWide[kMaxStages + s * 4 + 0] | sWide[kMaxStages + s * 4 + 1] | sWide[kMaxStages + s * 4 + 2] |
-                   sWide[kMaxStages + s * 4 + 3];
-      mbar_arrive(BAR(kBarSuf + s));
+      const bool pass1 = kind == kJobP1;
+      const bool last1 = pass1 && j == decode_item(a, sJob[4 * s + 1]).n - 1;
+      // sGam[buf] is rewritten once the look-back of item ks - 2 has read it.
+      if (last1 && ks >= 2 &&
+          !group_and(1, 64, wait_bar(BAR(kBarSinReady + buf), (uint32_t)(((ks >> 1) - 1) & 1), abort_flag)))
+        break;
+      if (pass1 && j == 0) off = make_float2(0.f, 0.f);
+      const bool act = c < a.dk;
+      const int pw = (a.dk + 4) >> 1;  // row pitch in float2
+      float2* ptr = reinterpret_cast<float2*>(smem + (uint32_t)s * a.stage_bytes + a.oLA) +
+                    (a.g.reverse ? 0 : (MC - 1)) * pw + (c >> 1);  // last scanned row first
+      const int step = a.g.reverse ? pw : -pw;
+      const float2 base = pass1 ? off : make_float2(0.f, 0.f);
+      float2 acc = base;
+#pragma unroll 1
+      for (int m = 0; m < 4; ++m) {
+        if (act) {
+#pragma unroll 1
+          for (int h16 = 0; h16 < 2; ++h16) {
+            // Sixteen rows are loaded before their stores so that the loads overlap.
+            float2 x[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) x[q] = ptr[q * step];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              ptr[q * step] = acc;
+              acc.x += x[q].x;
+              acc.y += x[q].y;
+            }
+            ptr += 16 * step;
+          }
+        }
+        if (m == 3 && act) {  // chunk totals before the last quarter is released
+          sBL[s * 128 + c] = acc.x - base.x;
+          sBL[s * 128 + c + 1] = acc.y - base.y;
+          if (pass1) {
+            off = acc;
+            if (last1) {
+              // exp(segment gate sum) of growth gates must stay finite
+              if (!(off.x <= kMaxGateRange) || !(off.y <= kMaxGateRange)) report_status(GLA_ERR_RANGE);
+              sGam[buf * 128 + c] = __expf(off.x);
+              sGam[buf * 128 + c + 1] = __expf(off.y);
+            }
+          }
+        }
+        mbar_arrive(BAR(kBarSuf + 4 * s + (a.g.reverse ? m : 3 - m)));
+      }
+      if (last1) ++ks;
     }
   } else if (warp < kWarpEpi) {
     // ------------------------------------------------------------ gates (row r)
+    // K^ = k exp(u) (and Q~ = q exp(-u) in pass 2) in place.  A chunk whose |u| exceeds
+    // the fp32-safe range anywhere is evaluated serially instead (flagged here; the
+    // serial path reads the raw q and k from global memory).
     const int r = tid - 32 * kWarpGate;
-    for (int j = 0; j < njob; ++j) {
-      const int s = j % S, k = j / S;
-      if (!wait_bar(BAR(kBarSuf + s), (uint32_t)(k & 1), abort_flag)) break;
-      const bool pass1 = j < n;
+    const int quarter = warp - kWarpGate;
+    for (int jc = 0;; ++jc) {
+      const int s = jc % S, use = jc / S;
+      if (!wait_bar(BAR(kBarSuf + 4 * s + quarter), (uint32_t)(use & 1), abort_flag)) break;
+      const int kind = sJob[4 * s];
+      if (kind == kJobEnd) {
+        mbar_arrive(BAR(kBarGate + s));
+        break;
+      }
+      const bool pass1 = kind == kJobP1;
       uint8_t* st = smem + (uint32_t)s * a.stage_bytes;
-      if (pass1 || !sWide[s]) {
+      float umax = 0.f;  // pass 1: largest u; pass 2: largest |u|
+      {
         const float* urow = reinterpret_cast<const float*>(st + a.oLA) + r * (a.dk + 4);
         // Three 8-channel groups per round: all loads first, then gates, then stores.
         for (int cbase = 0; cbase < a.dk; cbase += 24) {
@@ -561,27 +911,29 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
           uint4 kw[3], qw[3];
 #pragma unroll
           for (int g3 = 0; g3 < 3; ++g3) {
-            const int c = cbase + 8 * g3;
-            if (c < a.dk) {
-              const uint32_t o = sw32_off((uint32_t)r, (uint32_t)c);
-              u[g3][0] = *reinterpret_cast<const float4*>(urow + c);
-              u[g3][1] = *reinterpret_cast<const float4*>(urow + c + 4);
+            const int cc = cbase + 8 * g3;
+            if (cc < a.dk) {
+              const uint32_t o = sw32_off((uint32_t)r, (uint32_t)cc);
+              u[g3][0] = *reinterpret_cast<const float4*>(urow + cc);
+              u[g3][1] = *reinterpret_cast<const float4*>(urow + cc + 4);
               kw[g3] = *reinterpret_cast<const uint4*>(st + a.oK + o);
               if (!pass1) qw[g3] = *reinterpret_cast<const uint4*>(st + a.oQ + o);
             }
           }
 #pragma unroll
           for (int g3 = 0; g3 < 3; ++g3) {
-            const int c = cbase + 8 * g3;
-            if (c < a.dk) {
-              const uint32_t o = sw32_off((uint32_t)r, (uint32_t)c);
-              const float e[8] = {u[g3][0].x, u[g3][0].y, u[g3][0].z, u[g3][0].w,
-                                  u[g3][1].x, u[g3][1].y, u[g3][1].z, u[g3][1].w};
+            const int cc = cbase + 8 * g3;
+            if (cc < a.dk) {
+              const uint32_t o = sw32_off((uint32_t)r, (uint32_t)cc);
+              const float ev[8] = {u[g3][0].x, u[g3][0].y, u[g3][0].z, u[g3][0].w,
+                                   u[g3][1].x, u[g3][1].y, u[g3][1].z, u[g3][1].w};
+#pragma unroll
+              for (int q = 0; q < 8; ++q) umax = fmaxf(umax, pass1 ? ev[q] : fabsf(ev[q]));
               uint32_t* uk = reinterpret_cast<uint32_t*>(&kw[g3]);
 #pragma unroll
               for (int jj = 0; jj < 4; ++jj) {
                 const float2 xx = unpack_bf16x2(uk[jj]);
-                uk[jj] = pack_bf16x2(xx.x * __expf(e[2 * jj]), xx.y * __expf(e[2 * jj + 1]));
+                uk[jj] = pack_bf16x2(xx.x * __expf(ev[2 * jj]), xx.y * __expf(ev[2 * jj + 1]));
               }
               *reinterpret_cast<uint4*>(st + a.oK + o) = kw[g3];
               if (!pass1) {
@@ -589,7 +941,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
                   const float2 xx = unpack_bf16x2(uq[jj]);
-                  uq[jj] = pack_bf16x2(xx.x * __expf(-e[2 * jj]), xx.y * __expf(-e[2 * jj + 1]));
+                  uq[jj] = pack_bf16x2(xx.x * __expf(-ev[2 * jj]), xx.y * __expf(-ev[2 * jj + 1]));
                 }
                 *reinterpret_cast<uint4*>(st + a.oQ + o) = qw[g3];
               }
@@ -598,30 +950,40 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
         }
         fence_proxy_async_smem();
       }
+      // NaN compares false: a NaN or infinite u also counts as out of range.
+      bool bad = !(umax <= kMaxGateRange);
+      if (!pass1 && quarter == (a.g.reverse ? 3 : 0))  // this quarter is released last
+        for (int cc = lane; cc < a.dk; cc += 32) bad |= !(sBL[s * 128 + cc] <= kMaxGateRange);  // exp(chunk sum)
+      if (pass1) {
+        if (bad) report_status(GLA_ERR_RANGE);  // exp(u) of growth gates overflows
+      } else {
+        const bool wide = group_or(4, 128, bad);
+        if (r == 0) sWide[s] = wide;
+      }
       mbar_arrive(BAR(kBarGate + s));
     }
-  } else {
-    // ------------------------------------------------------------ TMEM-side work
+  } else if (warp < kWarpLb) {
+    // ------------------------------------------------------------ output group (pass 2)
+    // Per non-serial chunk j: mask S(j) into P(j); epilogue of chunk j-1 (its MMAs also
+    // finished the state update); G = Diag(gamma_j) S; then the MMAs of chunk j run.
     const int i = 32 * (warp & 3) + lane;  // TMEM lane = row / key channel
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const int e = tid - 32 * kWarpEpi;
-    int kb = 0;
-    bool prev_pending = false;
-    int prev_cf = 0;
+    int kb = 0, jb = 0;
     bool ok = true;
 
-    // Epilogue of the previous output buffer: O -> bf16 -> out[b][token][h][:].
-    auto finish_prev = [&]() -> bool {
-      if (!prev_pending) return true;
-      const int ob = (kb - 1) & 1;
-      if (!group_and(2, 128, wait_bar(BAR(kBarBatch0 + ob), (uint32_t)(((kb - 1) >> 1) & 1), abort_flag)))
-        return false;
+    // Epilogue of non-serial job pkb: O -> bf16 -> out[b][token][h][:], then the O
+    // buffer is released.
+    auto finish = [&](int ib, int ih, int cf, int pkb) -> bool {
+      const int ob = pkb % a.nO;
+      if (!group_and(2, 128, wait_bar(BAR(kBarBatch + ob), (uint32_t)((pkb / a.nO) & 1), abort_flag))) return false;
       tc_fence_after();
-      const int t = row_token(a, prev_cf, i);
+      const int t = row_token(a, cf, i);
       const bool valid = t >= 0;
       __nv_bfloat16* orow = a.out;
-      if (valid) orow = a.out + (((int64_t)b * a.g.T + t) * a.H + h) * a.dv;
-      const uint32_t tO = tbase + (ob ? kColSeg : kColO0) + lane_base;
+      if (valid) orow = a.out + (((int64_t)ib * a.g.T + t) * a.H + ih) * a.dv;
+      const uint32_t tO = tbase + a.col_o(ob) + lane_base;
+#pragma unroll 1
       for (int c0 = 0; c0 < a.Np; c0 += 32) {
         uint32_t o[2][16];
         tmem_ld_cols<2>(tO + (uint32_t)c0, a.Np - c0, o);
@@ -637,206 +999,154 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
         }
       }
       tc_fence_before();
-      mbar_arrive(BAR(kBarOEmpty0 + ob));
-      prev_pending = false;
+      mbar_arrive(BAR(kBarOFree + ob));
       return true;
     };
 
-    // ---- end of pass 1: publish the segment aggregate and look back ----
-    // (this group takes no part in pass 1 itself)
-    if (!group_and(2, 128, wait_bar(BAR(kBarSegDone), 0u, abort_flag))) ok = false;
-    if (ok) {
+    for (int k = 0; ok; ++k) {
+      const int buf = k & 1;
+      if (!group_and(2, 128, wait_bar(BAR(kBarSinReady + buf), (uint32_t)((k >> 1) & 1), abort_flag))) break;
+      if (k >= sMisc[5]) break;  // end of the job stream
       tc_fence_after();
-      const int DQ = a.dv >> 2;
-      const uint32_t tSeg = tbase + kColSeg + lane_base, tSt = tbase + kColState + lane_base;
-      const float gs = sGam[i];
-      if (i < a.dk) a.agg_g[seg_id * a.dk + i] = gs;
-      for (int c0 = 0; c0 < a.Np; c0 += 64) {
-        uint32_t t[4][16];
-        tmem_ld_cols<4>(tSeg + (uint32_t)c0, a.Np - c0, t);
-        if (i < a.dk) {
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const int jq = c0 / 4 + q;
-            if (jq < DQ)
-              *reinterpret_cast<float4*>(a.agg_S + ((seg_id * DQ + jq) * a.dk + i) * 4) =
-                  make_float4(__uint_as_float(t[q >> 2][4 * (q & 3)]), __uint_as_float(t[q >> 2][4 * (q & 3) + 1]),
-                              __uint_as_float(t[q >> 2][4 * (q & 3) + 2]), __uint_as_float(t[q >> 2][4 * (q & 3) + 3]));
+      const Item it = decode_item(a, sItem[2 + buf]);
+      const uint32_t tSt = tbase + a.col_seg(buf) + lane_base;  // running state
+      bool pending = false;  // epilogue of the last non-serial chunk still to do
+      int p_cf = 0, p_kb = 0;
+      // j == n only finishes the last chunk.
+      for (int j = 0; j <= it.n; ++j) {
+        const bool last = j == it.n;
+        bool wide = false;
+        int s = 0, cf = 0;
+        if (!last) {
+          if (!group_and(2, 128, wait_bar(BAR(kBarMail), (uint32_t)(jb & 1), abort_flag))) {
+            ok = false;
+            break;
           }
-        }
-      }
-      __threadfence();
-      named_sync(2, 128);
-      if (e == 0) st_release(a.flags + seg_id, 1);
-      {
-        float z[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) z[q] = 0.f;
-        for (int cb = 0; cb < a.Np; cb += 16) tmem_st16(tSt + (uint32_t)cb, z);
-        tmem_st_wait();
-      }
-      float gam = 1.f;
-      for (int p = seg - 1; p >= 0; --p) {
-        const int64_t pid = (int64_t)bh * a.NS + p;
-        if (e == 0) sMisc[2] = wait_flag(a.flags, pid);
-        named_sync(2, 128);
-        const int fl = sMisc[2];
-        named_sync(2, 128);
-        if (fl == 0) break;  // timed out (recorded)
-        const float* src = (fl == 2 ? a.incl_S : a.agg_S);
-        // 32 columns of the predecessor's rows are loaded before the TMEM round trip.
-        for (int c0 = 0; c0 < a.Np; c0 += 32) {
-          float4 x[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int jq = c0 / 4 + q;
-            x[q] = (i < a.dk && jq < DQ)
-                       ? __ldcg(reinterpret_cast<const float4*>(src + ((pid * DQ + jq) * a.dk + i) * 4))
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-          uint32_t t[2][16];
-          tmem_ld_cols<2>(tSt + (uint32_t)c0, a.Np - c0, t);
-#pragma unroll
-          for (int c4 = 0; c4 < 2; ++c4) {
-            if (c0 + 16 * c4 < a.Np) {
-              float t16[16];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                t16[4 * q] = fmaf(gam, x[4 * c4 + q].x, __uint_as_float(t[c4][4 * q]));
-                t16[4 * q + 1] = fmaf(gam, x[4 * c4 + q].y, __uint_as_float(t[c4][4 * q + 1]));
-                t16[4 * q + 2] = fmaf(gam, x[4 * c4 + q].z, __uint_as_float(t[c4][4 * q + 2]));
-                t16[4 * q + 3] = fmaf(gam, x[4 * c4 + q].w, __uint_as_float(t[c4][4 * q + 3]));
-              }
-              tmem_st16(tSt + (uint32_t)(c0 + 16 * c4), t16);
-            }
-          }
-        }
-        tmem_st_wait();
-        if (fl == 1 && i < a.dk) gam *= __ldcg(a.agg_g + pid * a.dk + i);
-        if (fl == 2) break;
-      }
-      // Inclusive state of this segment: Diag(gamma_seg) S_in + aggregate.
-      for (int c0 = 0; c0 < a.Np; c0 += 32) {
-        uint32_t sin[2][16], sg[2][16];
-        tmem_ld_cols<2>(tSt + (uint32_t)c0, a.Np - c0, sin);
-        tmem_ld_cols<2>(tSeg + (uint32_t)c0, a.Np - c0, sg);
-        if (i < a.dk) {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int jq = c0 / 4 + q;
-            const int pc = q >> 2, o4 = 4 * (q & 3);
-            if (jq < DQ)
-              *reinterpret_cast<float4*>(a.incl_S + ((seg_id * DQ + jq) * a.dk + i) * 4) = make_float4(
-                  fmaf(gs, __uint_as_float(sin[pc][o4]), __uint_as_float(sg[pc][o4])),
-                  fmaf(gs, __uint_as_float(sin[pc][o4 + 1]), __uint_as_float(sg[pc][o4 + 1])),
-                  fmaf(gs, __uint_as_float(sin[pc][o4 + 2]), __uint_as_float(sg[pc][o4 + 2])),
-                  fmaf(gs, __uint_as_float(sin[pc][o4 + 3]), __uint_as_float(sg[pc][o4 + 3])));
-          }
-        }
-      }
-      __threadfence();
-      tc_fence_before();
-      named_sync(2, 128);
-      if (e == 0) st_release(a.flags + seg_id, 2);
-      tc_fence_after();
-    }
-
-    for (int j = n; j < njob && ok; ++j) {
-      const int s = j % S, k = j / S;
-      // The previous chunk's epilogue releases its stage; it must not wait behind this
-      // chunk's gates (with one stage, those need that very stage).
-      if (j > n && !finish_prev()) {
-        ok = false;
-        break;
-      }
-      if (!group_and(2, 128, wait_bar(BAR(kBarGate + s), (uint32_t)(k & 1), abort_flag))) {
-        ok = false;
-        break;
-      }
-      uint8_t* st = smem + (uint32_t)s * a.stage_bytes;
-      const int cf = fwd_chunk(a, job_chunk(j, c0, n));
-
-      // ---- pass 2 ----
-      if (sWide[s]) {
-        chunk_serial(a, st, red, tbase + kColState, lane_base, i, cf, b, h);
-        tc_fence_before();
-        named_sync(2, 128);
-        if (e == 0) mbar_arrive(BAR(kBarEmpty + s));
-        continue;
-      }
-      // G = Diag(gamma) S (state -> state, bf16 copy into the G tile)
-      {
-        const float gm = __expf(sBL[s * 128 + i]);
-        const uint32_t tSt = tbase + kColState + lane_base;
-        for (int c0 = 0; c0 < a.Np; c0 += 32) {
-          uint32_t t[2][16];
-          tmem_ld_cols<2>(tSt + (uint32_t)c0, a.Np - c0, t);
-#pragma unroll
-          for (int c4 = 0; c4 < 2; ++c4) {
-            const int cb = c0 + 16 * c4;
-            if (cb < a.Np) {
-              float t16[16];
-#pragma unroll
-              for (int q = 0; q < 16; ++q) t16[q] = __uint_as_float(t[c4][q]) * gm;
-              tmem_st16(tSt + (uint32_t)cb, t16);
-              if (i < a.Kp) {
-                const uint4 w0 = make_uint4(pack_bf16x2(t16[0], t16[1]), pack_bf16x2(t16[2], t16[3]),
-                                            pack_bf16x2(t16[4], t16[5]), pack_bf16x2(t16[6], t16[7]));
-                const uint4 w1 = make_uint4(pack_bf16x2(t16[8], t16[9]), pack_bf16x2(t16[10], t16[11]),
-                                            pack_bf16x2(t16[12], t16[13]), pack_bf16x2(t16[14], t16[15]));
-                *reinterpret_cast<uint4*>(smem + a.oG + g_off((uint32_t)i, (uint32_t)cb, (uint32_t)a.Kp)) = w0;
-                *reinterpret_cast<uint4*>(smem + a.oG + g_off((uint32_t)i, (uint32_t)cb + 8u, (uint32_t)a.Kp)) = w1;
-              }
-            }
-          }
-        }
-        tmem_st_wait();
-      }
-      // scores -> mask (keys scanned no later than the row) -> bf16 P in TMEM
-      if (!group_and(2, 128, wait_bar(BAR(kBarScFull), (uint32_t)(kb & 1), abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      {
-        const int rlo = 32 * (warp & 3), rhi = rlo + 31;
-#pragma unroll 1
-        for (int cb = 0; cb < MC; cb += 32) {
-          const bool none = a.g.reverse ? (cb + 31 < rlo) : (cb > rhi);
-          const bool all = a.g.reverse ? (cb >= rhi) : (cb + 31 <= rlo);
-          uint32_t sc[2][16];
-          if (!none) tmem_ld_cols<2>(tbase + kColS + lane_base + (uint32_t)cb, 32, sc);
-          uint32_t pk[16];
-          if (none) {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) pk[q] = 0u;
-          } else if (all) {
-#pragma unroll
-            for (int q = 0; q < 32; q += 2) pk[q >> 1] = pack_u2(sc[q >> 4][q & 15], sc[q >> 4][(q & 15) + 1]);
+          s = sMail[0];
+          wide = sMail[1] != 0;
+          ++jb;
+          cf = fwd_chunk(a, it.c0 + j);
+          if (wide) {
+            mbar_arrive(BAR(kBarScEmpty));  // no scores: the job is taken
           } else {
+            // scores -> mask (keys scanned no later than the row) -> bf16 P in TMEM
+            if (!group_and(2, 128, wait_bar(BAR(kBarScFull), (uint32_t)(kb & 1), abort_flag))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            {
+              const int rlo = 32 * (warp & 3), rhi = rlo + 31;
+#pragma unroll 1
+              for (int cb = 0; cb < MC; cb += 32) {
+                const bool none = a.g.reverse ? (cb + 31 < rlo) : (cb > rhi);
+                const bool all = a.g.reverse ? (cb >= rhi) : (cb + 31 <= rlo);
+                uint32_t sc[2][16];
+                if (!none) tmem_ld_cols<2>(tbase + kColS + lane_base + (uint32_t)cb, 32, sc);
+                uint32_t pk[16];
+                if (none) {
 #pragma unroll
-            for (int q = 0; q < 32; q += 2) {
-              const int s0 = cb + q, s1 = cb + q + 1;
-              const bool k0 = a.g.reverse ? (s0 >= i) : (s0 <= i);
-              const bool k1 = a.g.reverse ? (s1 >= i) : (s1 <= i);
-              const float v0 = __uint_as_float(sc[q >> 4][q & 15]);
-              const float v1 = __uint_as_float(sc[q >> 4][(q & 15) + 1]);
-              pk[q >> 1] = pack_bf16x2(k0 ? v0 : 0.f, k1 ? v1 : 0.f);
+                  for (int q = 0; q < 16; ++q) pk[q] = 0u;
+                } else if (all) {
+#pragma unroll
+                  for (int q = 0; q < 32; q += 2) pk[q >> 1] = pack_u2(sc[q >> 4][q & 15], sc[q >> 4][(q & 15) + 1]);
+                } else {
+#pragma unroll
+                  for (int q = 0; q < 32; q += 2) {
+                    const int s0 = cb + q, s1 = cb + q + 1;
+                    const bool k0 = a.g.reverse ? (s0 >= i) : (s0 <= i);
+                    const bool k1 = a.g.reverse ? (s1 >= i) : (s1 <= i);
+                    const float v0 = __uint_as_float(sc[q >> 4][q & 15]);
+                    const float v1 = __uint_as_float(sc[q >> 4][(q & 15) + 1]);
+                    pk[q >> 1] = pack_bf16x2(k0 ? v0 : 0.f, k1 ? v1 : 0.f);
+                  }
+                }
+                // bf16 pairs of keys overwrite score columns this thread has already read.
+                tmem_st16u(tbase + kColS + lane_base + (uint32_t)(cb >> 1), pk);
+              }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(BAR(kBarScEmpty));
+            mbar_arrive(BAR(kBarPReady));
+          }
+        }
+        // Epilogue of the previous chunk; its MMAs also completed the state update.
+        if (pending && !finish(it.b, it.h, p_cf, p_kb)) {
+          ok = false;
+          break;
+        }
+        pending = false;
+        if (last) break;
+        uint8_t* st = smem + (uint32_t)s * a.stage_bytes;
+        if (wide) {
+          chunk_serial(a, st, red, tbase + a.col_seg(buf), lane_base, i, cf, it.b, it.h);
+          tc_fence_before();
+          named_sync(2, 128);
+          if (e == 0) mbar_arrive(BAR(kBarEmpty + s));
+          continue;
+        }
+        // G = Diag(gamma) S (state -> state, bf16 copy into the G tile)
+        {
+          const float gm = __expf(sBL[s * 128 + i]);
+#pragma unroll 1
+          for (int c0 = 0; c0 < a.Np; c0 += 32) {
+            uint32_t t[2][16];
+            tmem_ld_cols<2>(tSt + (uint32_t)c0, a.Np - c0, t);
+#pragma unroll
+            for (int c4 = 0; c4 < 2; ++c4) {
+              const int cb = c0 + 16 * c4;
+              if (cb < a.Np) {
+                float t16[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) t16[q] = __uint_as_float(t[c4][q]) * gm;
+                tmem_st16(tSt + (uint32_t)cb, t16);
+                if (i < a.Kp) {
+                  const uint4 w0 = make_uint4(pack_bf16x2(t16[0], t16[1]), pack_bf16x2(t16[2], t16[3]),
+                                              pack_bf16x2(t16[4], t16[5]), pack_bf16x2(t16[6], t16[7]));
+                  const uint4 w1 = make_uint4(pack_bf16x2(t16[8], t16[9]), pack_bf16x2(t16[10], t16[11]),
+                                              pack_bf16x2(t16[12], t16[13]), pack_bf16x2(t16[14], t16[15]));
+                  *reinterpret_cast<uint4*>(smem + a.oG + g_off((uint32_t)i, (uint32_t)cb, (uint32_t)a.Kp)) = w0;
+                  *reinterpret_cast<uint4*>(smem + a.oG + g_off((uint32_t)i, (uint32_t)cb + 8u, (uint32_t)a.Kp)) = w1;
+                }
+              }
             }
           }
-          // bf16 pairs of keys overwrite score columns this thread has already read.
-          tmem_st16u(tbase + kColS + lane_base + (uint32_t)(cb >> 1), pk);
+          tmem_st_wait();
         }
+        tc_fence_before();
+        mbar_arrive(BAR(kBarGReady));
+        pending = true;
+        p_cf = cf;
+        p_kb = kb;
+        ++kb;
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(BAR(kBarScEmpty));
-      mbar_arrive(BAR(kBarPReady));
-      prev_pending = true;
-      prev_cf = cf;
-      ++kb;
+      if (!ok) break;
+      // pass 2 is done with the buffer
+      named_sync(2, 128);
+      if (e == 0) mbar_arrive(BAR(kBarSegFree + buf));
     }
-    if (ok) finish_prev();
+  } else {
+    // ------------------------------------------------------------ look-back group
+    const int i = 32 * (warp & 3) + lane;  // TMEM lane = key channel
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const int e = tid - 32 * kWarpLb;
+    for (int k = 0;; ++k) {
+      const int buf = k & 1;
+      if (!group_and(3, 128, wait_bar(BAR(kBarSegDone + buf), (uint32_t)((k >> 1) & 1), abort_flag))) break;
+      if (k >= sMisc[5]) {  // end of the job stream: pass it on to the output group
+        if (e == 0) mbar_arrive(BAR(kBarSinReady + buf));
+        break;
+      }
+      tc_fence_after();
+      const int item = sItem[buf];
+      const Item it = decode_item(a, item);
+      lookback(a, it.seg, it.bh, it.seg_id, tbase + a.col_seg(buf) + lane_base, i, e, sGam[buf * 128 + i], sMisc + 2);
+      if (e == 0) {
+        sItem[2 + buf] = item;
+        mbar_arrive(BAR(kBarSinReady + buf));
+      }
+    }
   }
 
   // ---------------------------------------------------------------- teardown
@@ -856,7 +1166,9 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const WsArgs a, const __grid
 
 struct WsLayout {
   int NC, NS, G, Kp, Np, nstage, mode, rpc, ppr;
-  uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oMisc, oBar, oTm;
+  uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oMisc, oJob, oMail, oItem, oBar, oTm;
+  int nO;
+  uint32_t colO0, colO1, colSeg0, colSeg1;
   size_t smem;
   size_t flag_bytes, agg_bytes, aggg_bytes;
 };
@@ -897,18 +1209,36 @@ WsLayout ws_layout(const GlaShape& s) {
   // channel blocks from oK; the stage is at least that large.
   L.stage_bytes = al1024(L.oLA + la > 8 * ATOM32 ? L.oLA + la : 8 * ATOM32);
   const uint32_t gtile = al1024((uint32_t)L.Kp * (uint32_t)L.Np * 2u);
-  const uint32_t fixed = gtile + kMaxStages * 512 + 256 + 512 + 256 + 64 + 8 * kNumBars + 16;
+  const uint32_t fixed = gtile + kMaxStages * 512 + 256 + 1024 + 256 + 64 + 16 * kMaxStages + 16 + 16 +
+                         8 * kNumBars + 16;
   L.nstage = (1024 + 2 * (size_t)L.stage_bytes + fixed <= kMaxSmem) ? 2 : 1;
   L.oG = (uint32_t)L.nstage * L.stage_bytes;
   L.oBL = L.oG + gtile;
   L.oWide = L.oBL + kMaxStages * 512;
   L.oGam = L.oWide + 256;
-  L.oRed = L.oGam + 512;
+  L.oRed = L.oGam + 1024;
   L.oMisc = L.oRed + 256;
-  L.oBar = L.oMisc + 64;
+  L.oJob = L.oMisc + 64;
+  L.oMail = L.oJob + 16 * kMaxStages;
+  L.oItem = L.oMail + 16;
+  L.oBar = L.oItem + 16;
   L.oTm = L.oBar + 8 * kNumBars;
   L.smem = 1024 + (size_t)L.oTm + 16;
   if (L.smem < 120 * 1024) L.smem = 120 * 1024;  // one CTA per SM: it owns all 512 TMEM columns
+  // TMEM columns: scores / P [0,128), O (two buffers when dv <= 96), then two
+  // aggregate / state buffers.
+  if (L.Np <= 96) {
+    L.nO = 2;
+    L.colO0 = 128;
+    L.colO1 = 224;
+    L.colSeg0 = 320;
+    L.colSeg1 = 416;
+  } else {
+    L.nO = 1;
+    L.colO0 = L.colO1 = 128;
+    L.colSeg0 = 256;
+    L.colSeg1 = 384;
+  }
   const size_t BH = (size_t)s.B * s.H;
   L.flag_bytes = al256((BH * L.NS + 1) * sizeof(int));
   L.agg_bytes = al256(BH * L.NS * s.dk * s.dv * sizeof(float));
@@ -1013,7 +1343,16 @@ cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const fl
   a.oGam = L.oGam;
   a.oRed = L.oRed;
   a.oMisc = L.oMisc;
+  a.oJob = L.oJob;
+  a.oMail = L.oMail;
+  a.oItem = L.oItem;
   a.oBar = L.oBar;
+  a.nO = L.nO;
+  a.colO0 = L.colO0;
+  a.colO1 = L.colO1;
+  a.colSeg0 = L.colSeg0;
+  a.colSeg1 = L.colSeg1;
+  a.items = (int)(BH * L.NS);
   a.oTm = L.oTm;
   a.g = make_geom(s.Hg, s.Wg, s.dir);
 
@@ -1035,7 +1374,13 @@ cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const fl
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(gla_ws_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
   if (e != cudaSuccess) return e;
-  gla_ws_fwd<<<(unsigned)(BH * L.NS), NT, L.smem, st>>>(a, tm);
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const size_t grid = (size_t)a.items < (size_t)sms ? (size_t)a.items : (size_t)sms;
+  gla_ws_fwd<<<(unsigned)grid, NT, L.smem, st>>>(a, tm);
   return cudaGetLastError();
 }
 
