@@ -25,7 +25,8 @@
 //   warp 1      MMA issuer (tcgen05, one thread) and TMEM owner;
 //   warps 2-3   suffix sums of the log-gates, one thread per pair of key channels,
 //               released to the gate warps 32 rows at a time;
-//   warps 4-7   gates applied in place (K^, Q~), one thread per row;
+//   warps 4-7   gates applied in place (K^, Q~): lane = row of the released quarter,
+//               warp = set of 8-channel blocks;
 //   warps 8-11  output group, one thread per TMEM lane: score masking to bf16 P,
 //               G = Diag(gamma) S, output epilogue, serial path;
 //   warps 12-15 look-back group, one thread per TMEM lane.
@@ -74,10 +75,10 @@ enum {
   kBarGReady,                         // state scaled and G written (128 arrivals)
   kBarBatch,                          // [2] output and state MMAs done, per O buffer
   kBarOFree = kBarBatch + 2,          // [2] O buffer read (128 arrivals)
-  kBarSegDone = kBarOFree + 2,        // [2] pass-1 MMAs of an item done (or end of stream)
-  kBarSinReady = kBarSegDone + 2,     // [2] look-back done: incoming state in the buffer
-  kBarSegFree = kBarSinReady + 2,     // [2] pass 2 done with the buffer
-  kBarDrain = kBarSegFree + 2,        // all MMAs of the CTA done (teardown)
+  kBarSegDone = kBarOFree + 2,        // [3] pass-1 MMAs of an item done (or end of stream)
+  kBarSinReady = kBarSegDone + 3,     // [3] look-back done: incoming state in the buffer
+  kBarSegFree = kBarSinReady + 3,     // [3] pass 2 done with the buffer
+  kBarDrain = kBarSegFree + 3,        // all MMAs of the CTA done (teardown)
   kNumBars
 };
 
@@ -96,12 +97,14 @@ struct WsArgs {
   int* flags;     // [BH][NS]               0 nothing, 1 aggregate, 2 inclusive
   int* ticket;
   int H, BH, dk, dv, NC, NS, G, items;
-  int Kp, Np, nstage, nO;
-  uint32_t colO0, colO1, colSeg0, colSeg1;
+  int Kp, Np, nstage, nO, nbuf;
+  uint32_t colO0, colO1, colSeg0, colSeg1, colSeg2;
   int mode, rpc, ppr;  // chunk geometry: 0 raster, 1 whole columns (rpc per chunk), 2 column pieces (ppr per column)
   uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oMisc, oJob, oMail, oItem, oBar, oTm;
   ScanGeom g;
-  __device__ __forceinline__ uint32_t col_seg(int buf) const { return buf ? colSeg1 : colSeg0; }
+  __device__ __forceinline__ uint32_t col_seg(int buf) const {
+    return buf == 0 ? colSeg0 : (buf == 1 ? colSeg1 : colSeg2);
+  }
   __device__ __forceinline__ uint32_t col_o(int ob) const { return ob ? colO1 : colO0; }
 };
 
@@ -123,7 +126,7 @@ __device__ __forceinline__ Item decode_item(const WsArgs& a, int item) {
 }
 
 struct TensorMaps {
-  CUtensorMap q, k, v, la;
+  CUtensorMap q, k, v, la;  // operand tiles (16-channel boxes, 32-byte swizzle) and log-gate tiles
 };
 
 // ---------------------------------------------------------------------------
@@ -244,6 +247,11 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Lane-wise product of two packed bf16 pairs, rounded to bf16.
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t x, uint32_t y) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&x), *reinterpret_cast<__nv_bfloat162*>(&y));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
 __device__ __forceinline__ uint32_t pack_u2(uint32_t x, uint32_t y) {
   return pack_bf16x2(__uint_as_float(x), __uint_as_float(y));
 }
@@ -282,21 +290,6 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     }
   }
   return true;
-}
-
-// Spin (one thread) until flags[idx] != 0; 0 on timeout.
-__device__ int wait_flag(const int* flags, int64_t idx) {
-  uint32_t f = ld_acquire(flags + idx);
-  if (f) return (int)f;
-  const long long t0 = clock64();
-  while ((f = ld_acquire(flags + idx)) == 0) {
-    if (clock64() - t0 > kWaitCycles) {
-      report_status(GLA_ERR_TIMEOUT);
-      return 0;
-    }
-    __nanosleep(64);
-  }
-  return (int)f;
 }
 
 // Forward chunk index of scan-order chunk c.
@@ -426,23 +419,23 @@ __device__ void chunk_serial(const WsArgs& a, const uint8_t* st, float* red, uin
 }
 
 // Adds coef * src[pid] (an aggregate or inclusive state in the quad layout) to the
-// state rows this thread owns in TMEM (tSt), 80 columns per global round trip; also
+// state rows this thread owns in TMEM (tSt), 32 columns per global round trip; also
 // returns coef * gamma[pid] when want_gam (the coefficient for the next predecessor).
 __device__ __forceinline__ float fold_state(const WsArgs& a, const float* src, int64_t pid, float coef, uint32_t tSt,
                                             int i, bool want_gam) {
   const int DQ = a.dv >> 2;
   const float g = (want_gam && i < a.dk) ? __ldcg(a.agg_g + pid * a.dk + i) : 1.f;
 #pragma unroll 1
-  for (int c0 = 0; c0 < a.Np; c0 += 80) {
-    float4 x[20];
+  for (int c0 = 0; c0 < a.Np; c0 += 32) {
+    float4 x[8];
 #pragma unroll
-    for (int q = 0; q < 20; ++q) {
+    for (int q = 0; q < 8; ++q) {
       const int jq = c0 / 4 + q;
       x[q] = (i < a.dk && jq < DQ) ? __ldcg(reinterpret_cast<const float4*>(src + ((pid * DQ + jq) * a.dk + i) * 4))
                                    : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int c4 = 0; c4 < 5; ++c4) {
+    for (int c4 = 0; c4 < 2; ++c4) {
       const int cb = c0 + 16 * c4;
       if (cb < a.Np) {
         uint32_t t[1][16];
@@ -600,13 +593,13 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* sBL = reinterpret_cast<float*>(smem + a.oBL);      // [S][128] chunk gate sums
   volatile int* sWide = reinterpret_cast<volatile int*>(smem + a.oWide);  // [S] chunk evaluated serially
-  float* sGam = reinterpret_cast<float*>(smem + a.oGam);    // [2][128] exp(segment gate sum)
+  float* sGam = reinterpret_cast<float*>(smem + a.oGam);    // [3][128] exp(segment gate sum)
   float* red = reinterpret_cast<float*>(smem + a.oRed);     // serial-path reduction [4][16]
   // [0] first item [1] abort [2] look-back flag [3] jobs posted [4] jobs taken [5] end item index
   volatile int* sMisc = reinterpret_cast<volatile int*>(smem + a.oMisc);
   volatile int* sJob = reinterpret_cast<volatile int*>(smem + a.oJob);    // [S][4] kind, item, j, buf
   volatile int* sMail = reinterpret_cast<volatile int*>(smem + a.oMail);  // [4]    stage, wide, item, j
-  volatile int* sItem = reinterpret_cast<volatile int*>(smem + a.oItem);  // [2] item per buffer, [2] same for pass 2
+  volatile int* sItem = reinterpret_cast<volatile int*>(smem + a.oItem);  // [3] item per buffer, [3] same for pass 2
   const uint32_t bars = sbase + a.oBar;
   auto BAR = [&](int idx) -> uint32_t { return bars + 8u * (uint32_t)idx; };
   volatile int* abort_flag = sMisc + 1;
@@ -630,6 +623,8 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     for (int q = 0; q < 2; ++q) {
       mbar_init(BAR(kBarBatch + q), 1);
       mbar_init(BAR(kBarOFree + q), 128);
+    }
+    for (int q = 0; q < 3; ++q) {
       mbar_init(BAR(kBarSegDone + q), 1);
       mbar_init(BAR(kBarSinReady + q), 1);
       mbar_init(BAR(kBarSegFree + q), 1);
@@ -643,7 +638,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     sMisc[5] = 0x7fffffff;
   }
   for (int x = tid; x < kMaxStages * 128; x += NT) sBL[x] = 0.f;  // rows >= dk: gamma = 1
-  for (int x = tid; x < 2 * 128; x += NT) sGam[x] = 1.f;
+  for (int x = tid; x < 3 * 128; x += NT) sGam[x] = 1.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -676,9 +671,10 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         return true;
       };
       auto post_p1 = [&](int item, int k) -> bool {
-        const int buf = k & 1;
-        // sItem[buf] is rewritten once the look-back of item k - 2 has read it.
-        if (k >= 2 && !wait_bar(BAR(kBarSinReady + buf), (uint32_t)(((k >> 1) - 1) & 1), abort_flag)) return false;
+        const int buf = k % a.nbuf;
+        // sItem[buf] is rewritten once the look-back of item k - nbuf has read it.
+        if (k >= a.nbuf && !wait_bar(BAR(kBarSinReady + buf), (uint32_t)(((k / a.nbuf) - 1) & 1), abort_flag))
+          return false;
         sItem[buf] = item;
         const int n = decode_item(a, item).n;
         for (int j = 0; j < n; ++j)
@@ -688,23 +684,30 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       auto post_p2 = [&](int item, int k) -> bool {
         const int n = decode_item(a, item).n;
         for (int j = 0; j < n; ++j)
-          if (!post(kJobP2, item, j, k & 1)) return false;
+          if (!post(kJobP2, item, j, k % a.nbuf)) return false;
         return true;
       };
-      int cur = sMisc[0];
-      bool ok = post_p1(cur, 0);
-      for (int k = 0; ok; ++k) {
-        const int nxt = atomicAdd(a.ticket, 1);
-        const bool more = nxt < a.items;
-        if (more) ok = post_p1(nxt, k + 1);
-        if (ok) ok = post_p2(cur, k);
-        if (!ok) break;
-        if (!more) {
-          post(kJobEnd, -1, 0, 0);
-          break;
+      // Pass 1 runs nbuf - 1 items ahead of pass 2.
+      int ring[4];
+      int have = 0;  // items claimed (their pass 1 posted)
+      bool ok = true, more = true;
+      auto claim = [&]() {
+        const int t = have == 0 ? sMisc[0] : atomicAdd(a.ticket, 1);
+        if (t >= a.items) {
+          more = false;
+          return;
         }
-        cur = nxt;
+        ring[have & 3] = t;
+        ok = post_p1(t, have);
+        ++have;
+      };
+      claim();
+      for (int l = 1; l < a.nbuf - 1 && ok && more; ++l) claim();
+      for (int k = 0; ok && k < have; ++k) {
+        if (more) claim();
+        if (ok) ok = post_p2(ring[k & 3], k);
       }
+      if (ok) post(kJobEnd, -1, 0, 0);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
@@ -748,14 +751,15 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         if (kind != kJobP2 && !issue_tail()) break;
         if (kind == kJobEnd) {
           sMisc[5] = km;  // the look-back and output groups stop at item km
-          mbar_arrive(BAR(kBarSegDone + (km & 1)));
+          mbar_arrive(BAR(kBarSegDone + km % a.nbuf));
           break;
         }
         const uint32_t st = sbase + (uint32_t)s * a.stage_bytes;
         const int n = decode_item(a, item).n;
         if (kind == kJobP1) {
           // The buffer is free once pass 2 of item km - 2 is done with it.
-          if (j == 0 && km >= 2 && !wait_bar(BAR(kBarSegFree + buf), (uint32_t)(((km >> 1) - 1) & 1), abort_flag))
+          if (j == 0 && km >= a.nbuf &&
+              !wait_bar(BAR(kBarSegFree + buf), (uint32_t)(((km / a.nbuf) - 1) & 1), abort_flag))
             break;
           tc_fence_after();
           const uint32_t id = idesc_bf16_f32(MC, a.Np, true, true);
@@ -838,9 +842,9 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       }
       const bool pass1 = kind == kJobP1;
       const bool last1 = pass1 && j == decode_item(a, sJob[4 * s + 1]).n - 1;
-      // sGam[buf] is rewritten once the look-back of item ks - 2 has read it.
-      if (last1 && ks >= 2 &&
-          !group_and(1, 64, wait_bar(BAR(kBarSinReady + buf), (uint32_t)(((ks >> 1) - 1) & 1), abort_flag)))
+      // sGam[buf] is rewritten once the look-back of item ks - nbuf has read it.
+      if (last1 && ks >= a.nbuf &&
+          !group_and(1, 64, wait_bar(BAR(kBarSinReady + buf), (uint32_t)(((ks / a.nbuf) - 1) & 1), abort_flag)))
         break;
       if (pass1 && j == 0) off = make_float2(0.f, 0.f);
       const bool act = c < a.dk;
@@ -886,79 +890,72 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       if (last1) ++ks;
     }
   } else if (warp < kWarpEpi) {
-    // ------------------------------------------------------------ gates (row r)
-    // K^ = k exp(u) (and Q~ = q exp(-u) in pass 2) in place.  A chunk whose |u| exceeds
-    // the fp32-safe range anywhere is evaluated serially instead (flagged here; the
-    // serial path reads the raw q and k from global memory).
-    const int r = tid - 32 * kWarpGate;
-    const int quarter = warp - kWarpGate;
+    // ------------------------------------------------------------ gates
+    // K^ = k exp(u) (and Q~ = q exp(-u) in pass 2) in place.  Lane l of gate warp w
+    // gates row 32q + l of each quarter q, in the order the suffix pass releases them,
+    // on the 8-channel blocks w, w + 4, w + 8, ...  A chunk whose |u| exceeds the
+    // fp32-safe range anywhere is evaluated serially instead (flagged here; the serial
+    // path reads the raw q and k from global memory).
+    const int gw = warp - kWarpGate;
     for (int jc = 0;; ++jc) {
       const int s = jc % S, use = jc / S;
-      if (!wait_bar(BAR(kBarSuf + 4 * s + quarter), (uint32_t)(use & 1), abort_flag)) break;
-      const int kind = sJob[4 * s];
+      int kind = kJobEnd;
+      bool ok_wait = true;
+      float umax = 0.f;  // pass 1: largest u; pass 2: largest |u|
+      uint8_t* st = smem + (uint32_t)s * a.stage_bytes;
+#pragma unroll 1
+      for (int m = 0; m < 4; ++m) {
+        const int quarter = a.g.reverse ? m : 3 - m;
+        if (!wait_bar(BAR(kBarSuf + 4 * s + quarter), (uint32_t)(use & 1), abort_flag)) {
+          ok_wait = false;
+          break;
+        }
+        kind = sJob[4 * s];
+        if (kind == kJobEnd) break;
+        const bool pass1 = kind == kJobP1;
+        const int r = 32 * quarter + lane;
+        const float* urow = reinterpret_cast<const float*>(st + a.oLA) + r * (a.dk + 4);
+        // exp(u) is rounded to bf16 pairs and applied with packed bf16 multiplies,
+        // exp(-u) as its reciprocal.
+#pragma unroll 1
+        for (int cc = 8 * gw; cc < a.dk; cc += 32) {
+          const uint32_t o = sw32_off((uint32_t)r, (uint32_t)cc);
+          const float4 u0 = *reinterpret_cast<const float4*>(urow + cc);
+          const float4 u1 = *reinterpret_cast<const float4*>(urow + cc + 4);
+          uint4 kw = *reinterpret_cast<const uint4*>(st + a.oK + o);
+          uint4 qw = make_uint4(0u, 0u, 0u, 0u);
+          if (!pass1) qw = *reinterpret_cast<const uint4*>(st + a.oQ + o);
+          const float ev[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+          uint32_t* uk = reinterpret_cast<uint32_t*>(&kw);
+          uint32_t* uq = reinterpret_cast<uint32_t*>(&qw);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const float a0 = ev[2 * jj], a1 = ev[2 * jj + 1];
+            umax = fmaxf(umax, pass1 ? fmaxf(a0, a1) : fmaxf(fabsf(a0), fabsf(a1)));
+            const float p0 = __expf(a0), p1 = __expf(a1);
+            uk[jj] = mul_bf16x2(uk[jj], pack_bf16x2(p0, p1));
+            if (!pass1) uq[jj] = mul_bf16x2(uq[jj], pack_bf16x2(__fdividef(1.f, p0), __fdividef(1.f, p1)));
+          }
+          *reinterpret_cast<uint4*>(st + a.oK + o) = kw;
+          if (!pass1) *reinterpret_cast<uint4*>(st + a.oQ + o) = qw;
+        }
+      }
+      if (!ok_wait) break;
       if (kind == kJobEnd) {
         mbar_arrive(BAR(kBarGate + s));
         break;
       }
+      fence_proxy_async_smem();
       const bool pass1 = kind == kJobP1;
-      uint8_t* st = smem + (uint32_t)s * a.stage_bytes;
-      float umax = 0.f;  // pass 1: largest u; pass 2: largest |u|
-      {
-        const float* urow = reinterpret_cast<const float*>(st + a.oLA) + r * (a.dk + 4);
-        // Three 8-channel groups per round: all loads first, then gates, then stores.
-        for (int cbase = 0; cbase < a.dk; cbase += 24) {
-          float4 u[3][2];
-          uint4 kw[3], qw[3];
-#pragma unroll
-          for (int g3 = 0; g3 < 3; ++g3) {
-            const int cc = cbase + 8 * g3;
-            if (cc < a.dk) {
-              const uint32_t o = sw32_off((uint32_t)r, (uint32_t)cc);
-              u[g3][0] = *reinterpret_cast<const float4*>(urow + cc);
-              u[g3][1] = *reinterpret_cast<const float4*>(urow + cc + 4);
-              kw[g3] = *reinterpret_cast<const uint4*>(st + a.oK + o);
-              if (!pass1) qw[g3] = *reinterpret_cast<const uint4*>(st + a.oQ + o);
-            }
-          }
-#pragma unroll
-          for (int g3 = 0; g3 < 3; ++g3) {
-            const int cc = cbase + 8 * g3;
-            if (cc < a.dk) {
-              const uint32_t o = sw32_off((uint32_t)r, (uint32_t)cc);
-              const float ev[8] = {u[g3][0].x, u[g3][0].y, u[g3][0].z, u[g3][0].w,
-                                   u[g3][1].x, u[g3][1].y, u[g3][1].z, u[g3][1].w};
-#pragma unroll
-              for (int q = 0; q < 8; ++q) umax = fmaxf(umax, pass1 ? ev[q] : fabsf(ev[q]));
-              uint32_t* uk = reinterpret_cast<uint32_t*>(&kw[g3]);
-#pragma unroll
-              for (int jj = 0; jj < 4; ++jj) {
-                const float2 xx = unpack_bf16x2(uk[jj]);
-                uk[jj] = pack_bf16x2(xx.x * __expf(ev[2 * jj]), xx.y * __expf(ev[2 * jj + 1]));
-              }
-              *reinterpret_cast<uint4*>(st + a.oK + o) = kw[g3];
-              if (!pass1) {
-                uint32_t* uq = reinterpret_cast<uint32_t*>(&qw[g3]);
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                  const float2 xx = unpack_bf16x2(uq[jj]);
-                  uq[jj] = pack_bf16x2(xx.x * __expf(-ev[2 * jj]), xx.y * __expf(-ev[2 * jj + 1]));
-                }
-                *reinterpret_cast<uint4*>(st + a.oQ + o) = qw[g3];
-              }
-            }
-          }
-        }
-        fence_proxy_async_smem();
-      }
       // NaN compares false: a NaN or infinite u also counts as out of range.
       bool bad = !(umax <= kMaxGateRange);
-      if (!pass1 && quarter == (a.g.reverse ? 3 : 0))  // this quarter is released last
+      if (!pass1 && gw == 0)
         for (int cc = lane; cc < a.dk; cc += 32) bad |= !(sBL[s * 128 + cc] <= kMaxGateRange);  // exp(chunk sum)
       if (pass1) {
         if (bad) report_status(GLA_ERR_RANGE);  // exp(u) of growth gates overflows
       } else {
         const bool wide = group_or(4, 128, bad);
-        if (r == 0) sWide[s] = wide;
+        if (gw == 0 && lane == 0) sWide[s] = wide;
       }
       mbar_arrive(BAR(kBarGate + s));
     }
@@ -1004,11 +1001,11 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     };
 
     for (int k = 0; ok; ++k) {
-      const int buf = k & 1;
-      if (!group_and(2, 128, wait_bar(BAR(kBarSinReady + buf), (uint32_t)((k >> 1) & 1), abort_flag))) break;
+      const int buf = k % a.nbuf;
+      if (!group_and(2, 128, wait_bar(BAR(kBarSinReady + buf), (uint32_t)((k / a.nbuf) & 1), abort_flag))) break;
       if (k >= sMisc[5]) break;  // end of the job stream
       tc_fence_after();
-      const Item it = decode_item(a, sItem[2 + buf]);
+      const Item it = decode_item(a, sItem[3 + buf]);
       const uint32_t tSt = tbase + a.col_seg(buf) + lane_base;  // running state
       bool pending = false;  // epilogue of the last non-serial chunk still to do
       int p_cf = 0, p_kb = 0;
@@ -1132,8 +1129,8 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const int e = tid - 32 * kWarpLb;
     for (int k = 0;; ++k) {
-      const int buf = k & 1;
-      if (!group_and(3, 128, wait_bar(BAR(kBarSegDone + buf), (uint32_t)((k >> 1) & 1), abort_flag))) break;
+      const int buf = k % a.nbuf;
+      if (!group_and(3, 128, wait_bar(BAR(kBarSegDone + buf), (uint32_t)((k / a.nbuf) & 1), abort_flag))) break;
       if (k >= sMisc[5]) {  // end of the job stream: pass it on to the output group
         if (e == 0) mbar_arrive(BAR(kBarSinReady + buf));
         break;
@@ -1143,7 +1140,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       const Item it = decode_item(a, item);
       lookback(a, it.seg, it.bh, it.seg_id, tbase + a.col_seg(buf) + lane_base, i, e, sGam[buf * 128 + i], sMisc + 2);
       if (e == 0) {
-        sItem[2 + buf] = item;
+        sItem[3 + buf] = item;
         mbar_arrive(BAR(kBarSinReady + buf));
       }
     }
@@ -1167,8 +1164,8 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
 struct WsLayout {
   int NC, NS, G, Kp, Np, nstage, mode, rpc, ppr;
   uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oMisc, oJob, oMail, oItem, oBar, oTm;
-  int nO;
-  uint32_t colO0, colO1, colSeg0, colSeg1;
+  int nO, nbuf;
+  uint32_t colO0, colO1, colSeg0, colSeg1, colSeg2;
   size_t smem;
   size_t flag_bytes, agg_bytes, aggg_bytes;
 };
@@ -1209,35 +1206,35 @@ WsLayout ws_layout(const GlaShape& s) {
   // channel blocks from oK; the stage is at least that large.
   L.stage_bytes = al1024(L.oLA + la > 8 * ATOM32 ? L.oLA + la : 8 * ATOM32);
   const uint32_t gtile = al1024((uint32_t)L.Kp * (uint32_t)L.Np * 2u);
-  const uint32_t fixed = gtile + kMaxStages * 512 + 256 + 1024 + 256 + 64 + 16 * kMaxStages + 16 + 16 +
+  const uint32_t fixed = gtile + kMaxStages * 512 + 256 + 1536 + 256 + 64 + 16 * kMaxStages + 16 + 32 +
                          8 * kNumBars + 16;
   L.nstage = (1024 + 2 * (size_t)L.stage_bytes + fixed <= kMaxSmem) ? 2 : 1;
   L.oG = (uint32_t)L.nstage * L.stage_bytes;
   L.oBL = L.oG + gtile;
   L.oWide = L.oBL + kMaxStages * 512;
   L.oGam = L.oWide + 256;
-  L.oRed = L.oGam + 1024;
+  L.oRed = L.oGam + 1536;
   L.oMisc = L.oRed + 256;
   L.oJob = L.oMisc + 64;
   L.oMail = L.oJob + 16 * kMaxStages;
   L.oItem = L.oMail + 16;
-  L.oBar = L.oItem + 16;
+  L.oBar = L.oItem + 32;
   L.oTm = L.oBar + 8 * kNumBars;
   L.smem = 1024 + (size_t)L.oTm + 16;
   if (L.smem < 120 * 1024) L.smem = 120 * 1024;  // one CTA per SM: it owns all 512 TMEM columns
-  // TMEM columns: scores / P [0,128), O (two buffers when dv <= 96), then two
-  // aggregate / state buffers.
+  // TMEM columns: scores / P [0,128), one O buffer, then the aggregate / state
+  // buffers: three when dv <= 96 (pass 1 two items ahead), else two.
+  L.nO = 1;
+  L.colO0 = L.colO1 = 128;
   if (L.Np <= 96) {
-    L.nO = 2;
-    L.colO0 = 128;
-    L.colO1 = 224;
-    L.colSeg0 = 320;
-    L.colSeg1 = 416;
+    L.nbuf = 3;
+    L.colSeg0 = 224;
+    L.colSeg1 = 320;
+    L.colSeg2 = 416;
   } else {
-    L.nO = 1;
-    L.colO0 = L.colO1 = 128;
+    L.nbuf = 2;
     L.colSeg0 = 256;
-    L.colSeg1 = 384;
+    L.colSeg1 = L.colSeg2 = 384;
   }
   const size_t BH = (size_t)s.B * s.H;
   L.flag_bytes = al256((BH * L.NS + 1) * sizeof(int));
@@ -1352,6 +1349,8 @@ cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const fl
   a.colO1 = L.colO1;
   a.colSeg0 = L.colSeg0;
   a.colSeg1 = L.colSeg1;
+  a.colSeg2 = L.colSeg2;
+  a.nbuf = L.nbuf;
   a.items = (int)(BH * L.NS);
   a.oTm = L.oTm;
   a.g = make_geom(s.Hg, s.Wg, s.dir);
