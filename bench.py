@@ -240,7 +240,7 @@ def run_gpu(args):
     convs = [torch.empty((w.B, w.Hgrid, w.Wgrid, w.C), dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
     reor = [torch.empty((w.B, w.T, w.C), dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
     stream = torch.cuda.current_stream(dev)
-    launches_per_layer = 3 + 1 + 1  # gla_fwd (chunk state, prefix, output) + dwconv3x3 + srem_reorient
+    launches_per_layer = 1 + 1 + 1  # gla_ws_fwd + dwconv3x3 + srem_reorient (the flag reset is a memset)
 
     def layer(l, ev=None):
         q, k, v, la = dev_in[l]
@@ -346,7 +346,7 @@ def run_gpu(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_dict({"parallelism": f"replicas x{world}" if world > 1 else "single GPU"}),
             "roofline": {
-                "bound": "hbm", "kernel": "gla_fwd (chunk state + prefix + output)",
+                "bound": "hbm", "kernel": "gla_ws_fwd (persistent warp-specialised GLA forward)",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "peak_source": f"{peak_kind} hbm_gbs", "traffic": traffic,
                 "algorithmic_bytes_per_launch": gla_bytes, "avg_launch_us": gla_avg_s * 1e6,
