@@ -70,8 +70,8 @@ enum {
   kBarEmpty = kBarGate + kMaxStages,  // [S]  stage free (MMA commit, or the serial path)
   kBarMail = kBarEmpty + kMaxStages,  // pass-2 job handed to the output group
   kBarScFull,                         // score MMA done
-  kBarScEmpty,                        // job taken and scores read (128 arrivals)
-  kBarPReady,                         // P written (128 arrivals)
+  kBarScEmpty,                        // pass-2 job taken by the output group (128 arrivals)
+  kBarPReady,                         // P written by the gate warps (128 arrivals)
   kBarGReady,                         // state scaled and G written (128 arrivals)
   kBarBatch,                          // [2] output and state MMAs done, per O buffer
   kBarOFree = kBarBatch + 2,          // [2] O buffer read (128 arrivals)
@@ -897,6 +897,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     // fp32-safe range anywhere is evaluated serially instead (flagged here; the serial
     // path reads the raw q and k from global memory).
     const int gw = warp - kWarpGate;
+    int kbg = 0;  // non-serial pass-2 jobs masked so far
     for (int jc = 0;; ++jc) {
       const int s = jc % S, use = jc / S;
       int kind = kJobEnd;
@@ -956,6 +957,50 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       } else {
         const bool wide = group_or(4, 128, bad);
         if (gw == 0 && lane == 0) sWide[s] = wide;
+        mbar_arrive(BAR(kBarGate + s));
+        if (!wide) {
+          // scores -> mask (keys scanned no later than the row) -> bf16 P in TMEM.
+          // Warp w owns TMEM lanes (rows) 32w..32w+31.
+          if (!group_and(4, 128, wait_bar(BAR(kBarScFull), (uint32_t)(kbg & 1), abort_flag))) break;
+          ++kbg;
+          tc_fence_after();
+          const int i = 32 * gw + lane;
+          const uint32_t lane_base = (uint32_t)(32 * gw) << 16;
+          {
+            const int rlo = 32 * (warp & 3), rhi = rlo + 31;
+#pragma unroll 1
+            for (int cb = 0; cb < MC; cb += 32) {
+              const bool none = a.g.reverse ? (cb + 31 < rlo) : (cb > rhi);
+              const bool all = a.g.reverse ? (cb >= rhi) : (cb + 31 <= rlo);
+              uint32_t sc[2][16];
+              if (!none) tmem_ld_cols<2>(tbase + kColS + lane_base + (uint32_t)cb, 32, sc);
+              uint32_t pk[16];
+              if (none) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q) pk[q] = 0u;
+              } else if (all) {
+#pragma unroll
+                for (int q = 0; q < 32; q += 2) pk[q >> 1] = pack_u2(sc[q >> 4][q & 15], sc[q >> 4][(q & 15) + 1]);
+              } else {
+#pragma unroll
+                for (int q = 0; q < 32; q += 2) {
+                  const int s0 = cb + q, s1 = cb + q + 1;
+                  const bool k0 = a.g.reverse ? (s0 >= i) : (s0 <= i);
+                  const bool k1 = a.g.reverse ? (s1 >= i) : (s1 <= i);
+                  const float v0 = __uint_as_float(sc[q >> 4][q & 15]);
+                  const float v1 = __uint_as_float(sc[q >> 4][(q & 15) + 1]);
+                  pk[q >> 1] = pack_bf16x2(k0 ? v0 : 0.f, k1 ? v1 : 0.f);
+                }
+              }
+              // bf16 pairs of keys overwrite score columns this thread has already read.
+              tmem_st16u(tbase + kColS + lane_base + (uint32_t)(cb >> 1), pk);
+            }
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(BAR(kBarPReady));
+        }
+        continue;
       }
       mbar_arrive(BAR(kBarGate + s));
     }
@@ -1023,50 +1068,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
           wide = sMail[1] != 0;
           ++jb;
           cf = fwd_chunk(a, it.c0 + j);
-          if (wide) {
-            mbar_arrive(BAR(kBarScEmpty));  // no scores: the job is taken
-          } else {
-            // scores -> mask (keys scanned no later than the row) -> bf16 P in TMEM
-            if (!group_and(2, 128, wait_bar(BAR(kBarScFull), (uint32_t)(kb & 1), abort_flag))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            {
-              const int rlo = 32 * (warp & 3), rhi = rlo + 31;
-#pragma unroll 1
-              for (int cb = 0; cb < MC; cb += 32) {
-                const bool none = a.g.reverse ? (cb + 31 < rlo) : (cb > rhi);
-                const bool all = a.g.reverse ? (cb >= rhi) : (cb + 31 <= rlo);
-                uint32_t sc[2][16];
-                if (!none) tmem_ld_cols<2>(tbase + kColS + lane_base + (uint32_t)cb, 32, sc);
-                uint32_t pk[16];
-                if (none) {
-#pragma unroll
-                  for (int q = 0; q < 16; ++q) pk[q] = 0u;
-                } else if (all) {
-#pragma unroll
-                  for (int q = 0; q < 32; q += 2) pk[q >> 1] = pack_u2(sc[q >> 4][q & 15], sc[q >> 4][(q & 15) + 1]);
-                } else {
-#pragma unroll
-                  for (int q = 0; q < 32; q += 2) {
-                    const int s0 = cb + q, s1 = cb + q + 1;
-                    const bool k0 = a.g.reverse ? (s0 >= i) : (s0 <= i);
-                    const bool k1 = a.g.reverse ? (s1 >= i) : (s1 <= i);
-                    const float v0 = __uint_as_float(sc[q >> 4][q & 15]);
-                    const float v1 = __uint_as_float(sc[q >> 4][(q & 15) + 1]);
-                    pk[q >> 1] = pack_bf16x2(k0 ? v0 : 0.f, k1 ? v1 : 0.f);
-                  }
-                }
-                // bf16 pairs of keys overwrite score columns this thread has already read.
-                tmem_st16u(tbase + kColS + lane_base + (uint32_t)(cb >> 1), pk);
-              }
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(BAR(kBarScEmpty));
-            mbar_arrive(BAR(kBarPReady));
-          }
+          mbar_arrive(BAR(kBarScEmpty));  // the job is taken (the gate warps mask its scores)
         }
         // Epilogue of the previous chunk; its MMAs also completed the state update.
         if (pending && !finish(it.b, it.h, p_cf, p_kb)) {
