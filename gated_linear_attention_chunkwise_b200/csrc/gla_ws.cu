@@ -1014,12 +1014,17 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     int kb = 0, jb = 0;
     bool ok = true;
 
-    // Epilogue of non-serial job pkb: O -> bf16 -> out[b][token][h][:], then the O
-    // buffer is released.
-    auto finish = [&](int ib, int ih, int cf, int pkb) -> bool {
-      const int ob = pkb % a.nO;
-      if (!group_and(2, 128, wait_bar(BAR(kBarBatch + ob), (uint32_t)((pkb / a.nO) & 1), abort_flag))) return false;
+    // MMAs of non-serial job pkb complete (output and state update).
+    auto wait_batch = [&](int pkb) -> bool {
+      if (!group_and(2, 128, wait_bar(BAR(kBarBatch + pkb % a.nO), (uint32_t)((pkb / a.nO) & 1), abort_flag)))
+        return false;
       tc_fence_after();
+      return true;
+    };
+    // Epilogue of non-serial job pkb (after wait_batch): O -> bf16 -> out[b][token][h][:],
+    // then the O buffer is released.
+    auto epilogue = [&](int ib, int ih, int cf, int pkb) {
+      const int ob = pkb % a.nO;
       const int t = row_token(a, cf, i);
       const bool valid = t >= 0;
       __nv_bfloat16* orow = a.out;
@@ -1042,7 +1047,6 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       }
       tc_fence_before();
       mbar_arrive(BAR(kBarOFree + ob));
-      return true;
     };
 
     for (int k = 0; ok; ++k) {
@@ -1070,14 +1074,48 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
           cf = fwd_chunk(a, it.c0 + j);
           mbar_arrive(BAR(kBarScEmpty));  // the job is taken (the gate warps mask its scores)
         }
-        // Epilogue of the previous chunk; its MMAs also completed the state update.
-        if (pending && !finish(it.b, it.h, p_cf, p_kb)) {
+        // The previous chunk's MMAs complete: they updated the state and wrote its O.
+        if (pending && !wait_batch(p_kb)) {
           ok = false;
           break;
         }
+        uint8_t* st = smem + (uint32_t)s * a.stage_bytes;
+        if (!last && !wide) {
+          // G = Diag(gamma) S (state -> state, bf16 copy into the G tile)
+          {
+            const float gm = __expf(sBL[s * 128 + i]);
+#pragma unroll 1
+            for (int c0 = 0; c0 < a.Np; c0 += 32) {
+              uint32_t t[2][16];
+              tmem_ld_cols<2>(tSt + (uint32_t)c0, a.Np - c0, t);
+#pragma unroll
+              for (int c4 = 0; c4 < 2; ++c4) {
+                const int cb = c0 + 16 * c4;
+                if (cb < a.Np) {
+                  float t16[16];
+#pragma unroll
+                  for (int q = 0; q < 16; ++q) t16[q] = __uint_as_float(t[c4][q]) * gm;
+                  tmem_st16(tSt + (uint32_t)cb, t16);
+                  if (i < a.Kp) {
+                    const uint4 w0 = make_uint4(pack_bf16x2(t16[0], t16[1]), pack_bf16x2(t16[2], t16[3]),
+                                                pack_bf16x2(t16[4], t16[5]), pack_bf16x2(t16[6], t16[7]));
+                    const uint4 w1 = make_uint4(pack_bf16x2(t16[8], t16[9]), pack_bf16x2(t16[10], t16[11]),
+                                                pack_bf16x2(t16[12], t16[13]), pack_bf16x2(t16[14], t16[15]));
+                    *reinterpret_cast<uint4*>(smem + a.oG + g_off((uint32_t)i, (uint32_t)cb, (uint32_t)a.Kp)) = w0;
+                    *reinterpret_cast<uint4*>(smem + a.oG + g_off((uint32_t)i, (uint32_t)cb + 8u, (uint32_t)a.Kp)) = w1;
+                  }
+                }
+              }
+            }
+            tmem_st_wait();
+          }
+          tc_fence_before();
+          mbar_arrive(BAR(kBarGReady));
+        }
+        // The previous chunk's epilogue runs while this chunk's state MMAs do.
+        if (pending) epilogue(it.b, it.h, p_cf, p_kb);
         pending = false;
         if (last) break;
-        uint8_t* st = smem + (uint32_t)s * a.stage_bytes;
         if (wide) {
           chunk_serial(a, st, red, tbase + a.col_seg(buf), lane_base, i, cf, it.b, it.h);
           tc_fence_before();
@@ -1085,36 +1123,6 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
           if (e == 0) mbar_arrive(BAR(kBarEmpty + s));
           continue;
         }
-        // G = Diag(gamma) S (state -> state, bf16 copy into the G tile)
-        {
-          const float gm = __expf(sBL[s * 128 + i]);
-#pragma unroll 1
-          for (int c0 = 0; c0 < a.Np; c0 += 32) {
-            uint32_t t[2][16];
-            tmem_ld_cols<2>(tSt + (uint32_t)c0, a.Np - c0, t);
-#pragma unroll
-            for (int c4 = 0; c4 < 2; ++c4) {
-              const int cb = c0 + 16 * c4;
-              if (cb < a.Np) {
-                float t16[16];
-#pragma unroll
-                for (int q = 0; q < 16; ++q) t16[q] = __uint_as_float(t[c4][q]) * gm;
-                tmem_st16(tSt + (uint32_t)cb, t16);
-                if (i < a.Kp) {
-                  const uint4 w0 = make_uint4(pack_bf16x2(t16[0], t16[1]), pack_bf16x2(t16[2], t16[3]),
-                                              pack_bf16x2(t16[4], t16[5]), pack_bf16x2(t16[6], t16[7]));
-                  const uint4 w1 = make_uint4(pack_bf16x2(t16[8], t16[9]), pack_bf16x2(t16[10], t16[11]),
-                                              pack_bf16x2(t16[12], t16[13]), pack_bf16x2(t16[14], t16[15]));
-                  *reinterpret_cast<uint4*>(smem + a.oG + g_off((uint32_t)i, (uint32_t)cb, (uint32_t)a.Kp)) = w0;
-                  *reinterpret_cast<uint4*>(smem + a.oG + g_off((uint32_t)i, (uint32_t)cb + 8u, (uint32_t)a.Kp)) = w1;
-                }
-              }
-            }
-          }
-          tmem_st_wait();
-        }
-        tc_fence_before();
-        mbar_arrive(BAR(kBarGReady));
         pending = true;
         p_cf = cf;
         p_kb = kb;
@@ -1224,17 +1232,18 @@ WsLayout ws_layout(const GlaShape& s) {
   L.oTm = L.oBar + 8 * kNumBars;
   L.smem = 1024 + (size_t)L.oTm + 16;
   if (L.smem < 120 * 1024) L.smem = 120 * 1024;  // one CTA per SM: it owns all 512 TMEM columns
-  // TMEM columns: scores / P [0,128), one O buffer, then the aggregate / state
-  // buffers: three when dv <= 96 (pass 1 two items ahead), else two.
-  L.nO = 1;
-  L.colO0 = L.colO1 = 128;
+  // TMEM columns: scores / P [0,128), O, then the aggregate / state buffers: two O
+  // buffers and two aggregate buffers when dv <= 96, else one O and two aggregates.
+  L.nbuf = 2;
   if (L.Np <= 96) {
-    L.nbuf = 3;
-    L.colSeg0 = 224;
-    L.colSeg1 = 320;
-    L.colSeg2 = 416;
+    L.nO = 2;
+    L.colO0 = 128;
+    L.colO1 = 224;
+    L.colSeg0 = 320;
+    L.colSeg1 = L.colSeg2 = 416;
   } else {
-    L.nbuf = 2;
+    L.nO = 1;
+    L.colO0 = L.colO1 = 128;
     L.colSeg0 = 256;
     L.colSeg1 = L.colSeg2 = 384;
   }
