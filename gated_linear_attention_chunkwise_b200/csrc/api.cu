@@ -98,6 +98,19 @@ int run_with_workspace(size_t bytes, cudaStream_t st, cudaError_t (*fn)(void*, v
 
 }  // namespace
 
+EncodeTiledFn tensor_map_encoder() {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {  // initialised once, thread-safe
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<EncodeTiledFn>(p);
+    cudaGetLastError();
+    return nullptr;
+  }();
+  return fn;
+}
+
 cudaError_t read_and_clear_device_status(int* status, cudaStream_t st) {
   cudaError_t e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return e;

@@ -1254,31 +1254,11 @@ WsLayout ws_layout(const GlaShape& s) {
   return L;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-    else
-      cudaGetLastError();
-  }
-  return fn;
-}
-
 // 5-D map over a [B][T][H][d] tensor viewed as (d, H, run position, run, B):
 // raster scans have one run of T positions, column scans Wg runs of Hg.
 bool encode_map(CUtensorMap* m, const void* base, bool f32, int d, int box0, CUtensorMapSwizzle sw, const GlaShape& s,
                 bool column, int box_rows, int box_runs) {
-  EncodeTiledFn fn = encode_fn();
+  EncodeTiledFn fn = tensor_map_encoder();
   if (!fn) return false;
   const cuuint64_t e = f32 ? 4 : 2;
   const cuuint64_t T = (cuuint64_t)s.T(), H = (cuuint64_t)s.H;

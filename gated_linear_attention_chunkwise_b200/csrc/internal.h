@@ -2,6 +2,7 @@
 // assumes its arguments were validated by api.cu and only enqueues work.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -27,6 +28,13 @@ constexpr int kChunkF32 = 64;
 size_t gla_f32_workspace_bytes(const GlaShape& s);
 cudaError_t gla_f32_forward(const float* q, const float* k, const float* v, const float* la, float* out,
                             const GlaShape& s, void* workspace, cudaStream_t st);
+
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point
+// (nullptr when the driver does not provide it).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder();
 
 // ---- SREM ----
 cudaError_t srem_reorient_launch(const void* x, void* y, int dir, int inverse, int B, int Hg, int Wg,

@@ -4,7 +4,8 @@
 //                     sequence), bit-exact.
 //   dwconv3x3_k     : 3x3 depthwise convolution on the channels-last token grid,
 //                     zero padding, fp32 accumulation.
-// Both are pure HBM streams: 128-bit loads and stores, no tensor cores.
+// Both are pure HBM streams, no tensor cores.  The conv streams haloed tiles
+// through shared memory with TMA; the reorientation copies 16-byte vectors.
 #include "dev_common.cuh"
 #include "internal.h"
 
@@ -29,95 +30,160 @@ __global__ void __launch_bounds__(256) srem_reorient_k(const uint4* __restrict__
   }
 }
 
+// ---------------------------------------------------------------------------
+// dwconv3x3_k: persistent blocks walk tiles of 16 x 16 pixels x one 128-byte channel
+// slice.  Each tile arrives with a one-pixel halo (18 x 18 pixels) by one TMA load
+// into a double-buffered shared-memory ring; pixels outside the image read as zero
+// (the TMA fills out-of-bounds elements), which is the zero padding.  Lane = 4
+// bytes of channels (two bf16 or one fp32 channel), warp = two output columns; each
+// thread walks the 16 rows with a 3-row x 4-column register window.
+// ---------------------------------------------------------------------------
+constexpr int kTile = 16;                          // output rows and columns per tile
+constexpr int kHalo = kTile + 2;                   // input rows and columns per tile
+constexpr uint32_t kTileBytes = kHalo * kHalo * 128u;                 // one haloed tile
+constexpr uint32_t kBufBytes = (kTileBytes + 1023u) / 1024u * 1024u;  // buffer stride (1024-aligned)
+constexpr size_t kConvSmem = 1024 + 2 * (size_t)kBufBytes + 64;      // + alignment slack and barriers
+constexpr int kConvThreads = 32 * (kTile / 2);
+
 template <typename T>
-struct VecTraits;
+struct Lane4;  // the 4 bytes of channels a lane owns
 template <>
-struct VecTraits<__nv_bfloat16> {
-  static constexpr int kVec = 8;
-  __device__ static void unpack(const uint4& u, float (&f)[8]) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+struct Lane4<__nv_bfloat16> {
+  static constexpr int kCh = 2;
+  __device__ static float2 get(uint32_t v) { return unpack_bf16x2(v); }
+  __device__ static uint32_t put(float2 f) { return pack_bf16x2(f.x, f.y); }
+};
+template <>
+struct Lane4<float> {
+  static constexpr int kCh = 1;
+  __device__ static float2 get(uint32_t v) { return make_float2(__uint_as_float(v), 0.f); }
+  __device__ static uint32_t put(float2 f) { return __float_as_uint(f.x); }
+};
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      : "memory");
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kConvThreads) dwconv3x3_k(const __grid_constant__ CUtensorMap xmap,
+                                                            const float* __restrict__ w, T* __restrict__ y, int Hg,
+                                                            int Wg, int C, int ntx, int nty, int nct, int ntiles) {
+  constexpr int kCh = Lane4<T>::kCh;
+  constexpr int kTC = 32 * kCh;  // channels per tile slice
+  extern __shared__ uint8_t sm_raw[];
+  // Tile buffers start on a 1024-byte boundary (TMA destinations); the two mbarriers
+  // follow them.
+  const uint32_t raw = smem_u32(sm_raw);
+  const uint32_t sbuf = (raw + 1023u) & ~1023u;
+  uint8_t* sm = sm_raw + (sbuf - raw);
+  const uint32_t bar0 = sbuf + 2u * kBufBytes;
+  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+  auto tile_coords = [&](int tile, int& b, int& ty, int& tx, int& ct) {
+    ct = tile % nct;
+    int r = tile / nct;
+    tx = r % ntx;
+    r /= ntx;
+    ty = r % nty;
+    b = r / nty;
+  };
+  auto issue = [&](int tile, int buf) {
+    int b, ty, tx, ct;
+    tile_coords(tile, b, ty, tx, ct);
+    mbar_expect_tx(bar0 + 8u * buf, kTileBytes);
+    tma_load_4d(sbuf + (uint32_t)buf * kBufBytes, &xmap, ct * kTC, tx * kTile - 1, ty * kTile - 1, b, bar0 + 8u * buf);
+  };
+  if (threadIdx.x == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar0 + 8, 1);
+    fence_mbar_init();
+    if ((int)blockIdx.x < ntiles) issue(blockIdx.x, 0);
+    if ((int)(blockIdx.x + gridDim.x) < ntiles) issue(blockIdx.x + gridDim.x, 1);
+  }
+  __syncthreads();
+  int ct_w = -1;
+  float2 wt[9];
+  for (int k = 0;; ++k) {
+    const int tile = blockIdx.x + k * gridDim.x;
+    if (tile >= ntiles) break;
+    const int buf = k & 1;
+    int b, ty, tx, ct;
+    tile_coords(tile, b, ty, tx, ct);
+    const int c = ct * kTC + kCh * lane;  // first channel of this lane
+    if (ct != ct_w) {  // weights of this lane's channels (zero past C)
+      ct_w = ct;
+#pragma unroll
+      for (int t = 0; t < 9; ++t) {
+        wt[t].x = c < C ? __ldg(w + (int64_t)c * 9 + t) : 0.f;
+        wt[t].y = (kCh == 2 && c + 1 < C) ? __ldg(w + (int64_t)(c + 1) * 9 + t) : 0.f;
+      }
+    }
+    // Bounded wait for the tile; the block leaves together if it expires.
+    bool late = false;
+    if (!mbar_try_wait(bar0 + 8u * buf, (uint32_t)((k >> 1) & 1))) {
+      const long long t0 = clock64();
+      while (!mbar_try_wait(bar0 + 8u * buf, (uint32_t)((k >> 1) & 1)))
+        if (clock64() - t0 > kWaitCycles) {
+          late = true;
+          break;
+        }
+    }
+    if (__syncthreads_or(late)) {
+      if (threadIdx.x == 0) {
+        report_status(GLA_ERR_TIMEOUT);
+        // Let the loads already issued into either buffer land before leaving (bounded).
+        for (int kk = k; kk < k + 2 && (int)(blockIdx.x + kk * gridDim.x) < ntiles; ++kk) {
+          const long long t0 = clock64();
+          while (!mbar_try_wait(bar0 + 8u * (kk & 1), (uint32_t)((kk >> 1) & 1)) && clock64() - t0 < kWaitCycles) {
+          }
+        }
+      }
+      return;
+    }
+    const uint32_t* tl = reinterpret_cast<const uint32_t*>(sm + (uint32_t)buf * kBufBytes);
+    auto at = [&](int r, int cc) -> uint32_t { return tl[(r * kHalo + cc) * 32 + lane]; };
+    const int x0 = tx * kTile + 2 * wp, y0 = ty * kTile;
+    uint32_t win[3][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float2 p = unpack_bf16x2(w[j]);
-      f[2 * j] = p.x;
-      f[2 * j + 1] = p.y;
+      win[0][j] = at(0, 2 * wp + j);
+      win[1][j] = at(1, 2 * wp + j);
     }
-  }
-  __device__ static uint4 pack(const float (&f)[8]) {
-    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                      pack_bf16x2(f[6], f[7]));
-  }
-};
-template <>
-struct VecTraits<float> {
-  static constexpr int kVec = 4;
-  __device__ static void unpack(const uint4& u, float (&f)[4]) {
-    f[0] = __uint_as_float(u.x);
-    f[1] = __uint_as_float(u.y);
-    f[2] = __uint_as_float(u.z);
-    f[3] = __uint_as_float(u.w);
-  }
-  __device__ static uint4 pack(const float (&f)[4]) {
-    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3]));
-  }
-};
-
-constexpr int kConvCols = 4;   // pixel columns per block (threadIdx.y)
-constexpr int kConvRows = 16;  // output rows per block, walked with a rolling 3-row window
-
-// Thread (cv, col): channel vector cv (16 bytes) of pixel column `col`, rows
-// y0 .. y0+kConvRows-1 of one image.  The 3x3 window of input vectors is kept in
-// registers and shifted down one row per output row.
-template <typename T>
-__global__ void __launch_bounds__(32 * kConvCols) dwconv3x3_k(const uint4* __restrict__ x, const float* __restrict__ w,
-                                                              uint4* __restrict__ y, int Hg, int Wg, int nvec,
-                                                              int nbands) {
-  constexpr int V = VecTraits<T>::kVec;
-  const int cv = blockIdx.x * 32 + threadIdx.x;
-  const int col = blockIdx.y * kConvCols + threadIdx.y;
-  const int b = blockIdx.z / nbands;
-  const int y0 = (blockIdx.z - b * nbands) * kConvRows;
-  if (cv >= nvec || col >= Wg) return;
-
-  float wr[9][V];
+    T* out = y + ((int64_t)b * Hg * Wg) * C + c;
+#pragma unroll 4
+    for (int r = 0; r < kTile; ++r) {
 #pragma unroll
-  for (int c = 0; c < V; ++c)
+      for (int j = 0; j < 4; ++j) win[2][j] = at(r + 2, 2 * wp + j);
 #pragma unroll
-    for (int t = 0; t < 9; ++t) wr[t][c] = __ldg(w + (int64_t)(cv * V + c) * 9 + t);
-
-  const int64_t img = (int64_t)b * Hg * Wg;
-  auto load = [&](int yy, int xx) -> uint4 {
-    if (yy < 0 || yy >= Hg || xx < 0 || xx >= Wg) return make_uint4(0u, 0u, 0u, 0u);
-    return __ldg(x + ((img + (int64_t)yy * Wg + xx) * nvec + cv));
-  };
-  uint4 win[3][3];
+      for (int oc = 0; oc < 2; ++oc) {
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int dj = 0; dj < 3; ++dj) {
-    win[0][dj] = load(y0 - 1, col + dj - 1);
-    win[1][dj] = load(y0, col + dj - 1);
-  }
-  const int yend = min(y0 + kConvRows, Hg);
-  for (int yy = y0; yy < yend; ++yy) {
+        for (int di = 0; di < 3; ++di)
 #pragma unroll
-    for (int dj = 0; dj < 3; ++dj) win[2][dj] = load(yy + 1, col + dj - 1);
-    float acc[V];
-#pragma unroll
-    for (int c = 0; c < V; ++c) acc[c] = 0.f;
-#pragma unroll
-    for (int di = 0; di < 3; ++di)
-#pragma unroll
-      for (int dj = 0; dj < 3; ++dj) {
-        float f[V];
-        VecTraits<T>::unpack(win[di][dj], f);
-#pragma unroll
-        for (int c = 0; c < V; ++c) acc[c] = fmaf(wr[di * 3 + dj][c], f[c], acc[c]);
+          for (int dj = 0; dj < 3; ++dj) {
+            const float2 v = Lane4<T>::get(win[di][oc + dj]);
+            acc.x = fmaf(wt[di * 3 + dj].x, v.x, acc.x);
+            acc.y = fmaf(wt[di * 3 + dj].y, v.y, acc.y);
+          }
+        const int yy = y0 + r, xx = x0 + oc;
+        if (yy < Hg && xx < Wg && c < C)
+          *reinterpret_cast<uint32_t*>(out + ((int64_t)yy * Wg + xx) * C) = Lane4<T>::put(acc);
       }
-    y[(img + (int64_t)yy * Wg + col) * nvec + cv] = VecTraits<T>::pack(acc);
 #pragma unroll
-    for (int dj = 0; dj < 3; ++dj) {
-      win[0][dj] = win[1][dj];
-      win[1][dj] = win[2][dj];
+      for (int j = 0; j < 4; ++j) {
+        win[0][j] = win[1][j];
+        win[1][j] = win[2][j];
+      }
     }
+    __syncthreads();  // the buffer is read out before it is refilled
+    if (threadIdx.x == 0 && tile + 2 * (int)gridDim.x < ntiles) issue(tile + 2 * gridDim.x, buf);
   }
 }
 
@@ -139,17 +205,40 @@ cudaError_t srem_reorient_launch(const void* x, void* y, int dir, int inverse, i
 
 cudaError_t dwconv3x3_launch(const void* x, const float* w, void* y, int B, int Hg, int Wg, int C, int dtype,
                              cudaStream_t st) {
-  const int V = (dtype == GLA_BF16) ? 8 : 4;
-  const int nvec = C / V;
-  const int nbands = (Hg + kConvRows - 1) / kConvRows;
-  const dim3 block(32, kConvCols);
-  const dim3 grid((nvec + 31) / 32, (Wg + kConvCols - 1) / kConvCols, B * nbands);
-  if (dtype == GLA_BF16)
-    dwconv3x3_k<__nv_bfloat16><<<grid, block, 0, st>>>(static_cast<const uint4*>(x), w, static_cast<uint4*>(y), Hg, Wg,
-                                                       nvec, nbands);
-  else
-    dwconv3x3_k<float><<<grid, block, 0, st>>>(static_cast<const uint4*>(x), w, static_cast<uint4*>(y), Hg, Wg, nvec,
-                                               nbands);
+  const bool bf = dtype == GLA_BF16;
+  const int esz = bf ? 2 : 4;
+  const int tc = 128 / esz;  // channels per tile slice
+  EncodeTiledFn fn = tensor_map_encoder();
+  if (!fn) return cudaErrorNotSupported;
+  // 4-D view (channel, column, row, image); the box is one haloed tile.
+  CUtensorMap map;
+  const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)Wg, (cuuint64_t)Hg, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)C * esz, (cuuint64_t)Wg * C * esz, (cuuint64_t)Hg * Wg * C * esz};
+  const cuuint32_t box[4] = {(cuuint32_t)tc, (cuuint32_t)kHalo, (cuuint32_t)kHalo, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  if (fn(&map, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(x), dims,
+         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const int ntx = (Wg + kTile - 1) / kTile, nty = (Hg + kTile - 1) / kTile, nct = (C + tc - 1) / tc;
+  const int ntiles = B * nty * ntx * nct;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = ntiles < 2 * sms ? ntiles : 2 * sms;  // two blocks per SM, each double-buffered
+  const size_t smem = kConvSmem;
+  cudaError_t e;
+  if (bf) {
+    e = cudaFuncSetAttribute(dwconv3x3_k<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dwconv3x3_k<__nv_bfloat16><<<grid, kConvThreads, smem, st>>>(map, w, static_cast<__nv_bfloat16*>(y), Hg, Wg, C,
+                                                                   ntx, nty, nct, ntiles);
+  } else {
+    e = cudaFuncSetAttribute(dwconv3x3_k<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dwconv3x3_k<float><<<grid, kConvThreads, smem, st>>>(map, w, static_cast<float*>(y), Hg, Wg, C, ntx, nty, nct,
+                                                         ntiles);
+  }
   return cudaGetLastError();
 }
 
