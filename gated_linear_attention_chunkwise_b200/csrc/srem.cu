@@ -31,19 +31,21 @@ __global__ void __launch_bounds__(256) srem_reorient_k(const uint4* __restrict__
 }
 
 // ---------------------------------------------------------------------------
-// dwconv3x3_k: persistent blocks walk tiles of 16 x 16 pixels x one 128-byte channel
-// slice.  Each tile arrives with a one-pixel halo (18 x 18 pixels) by one TMA load
-// into a double-buffered shared-memory ring; pixels outside the image read as zero
-// (the TMA fills out-of-bounds elements), which is the zero padding.  Lane = 4
-// bytes of channels (two bf16 or one fp32 channel), warp = two output columns; each
-// thread walks the 16 rows with a 3-row x 4-column register window.
+// dwconv3x3_k: persistent blocks walk tiles of 8 x 16 pixels (rows x columns) x one
+// 128-byte channel slice.  Each tile arrives with a one-pixel halo (10 x 18 pixels)
+// by one TMA load into a 4-deep shared-memory ring, so three loads are in flight
+// while a tile is computed; pixels outside the image read as zero (the TMA fills
+// out-of-bounds elements), which is the zero padding.  Lane = 4 bytes of channels
+// (two bf16 or one fp32 channel), warp = two output columns; each thread walks the
+// tile's rows with a 3-row x 4-column register window.
 // ---------------------------------------------------------------------------
-constexpr int kTile = 16;                          // output rows and columns per tile
-constexpr int kHalo = kTile + 2;                   // input rows and columns per tile
-constexpr uint32_t kTileBytes = kHalo * kHalo * 128u;                 // one haloed tile
+constexpr int kTileR = 8, kTileC = 16;            // output rows, columns per tile
+constexpr int kHaloR = kTileR + 2, kHaloC = kTileC + 2;
+constexpr int kConvBufs = 4;                       // TMA ring depth per block
+constexpr uint32_t kTileBytes = kHaloR * kHaloC * 128u;               // one haloed tile
 constexpr uint32_t kBufBytes = (kTileBytes + 1023u) / 1024u * 1024u;  // buffer stride (1024-aligned)
-constexpr size_t kConvSmem = 1024 + 2 * (size_t)kBufBytes + 64;      // + alignment slack and barriers
-constexpr int kConvThreads = 32 * (kTile / 2);
+constexpr size_t kConvSmem = 1024 + kConvBufs * (size_t)kBufBytes + 64;  // + alignment slack and barriers
+constexpr int kConvThreads = 32 * (kTileC / 2);
 
 template <typename T>
 struct Lane4;  // the 4 bytes of channels a lane owns
@@ -75,7 +77,7 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
 template <typename T>
 __global__ void __launch_bounds__(kConvThreads) dwconv3x3_k(const __grid_constant__ CUtensorMap xmap,
                                                             const float* __restrict__ w, T* __restrict__ y, int Hg,
-                                                            int Wg, int C, int ntx, int nty, int nct, int ntiles) {
+                                                            int Wg, int C, int ntx, int nty, int nct, int nsp) {
   constexpr int kCh = Lane4<T>::kCh;
   constexpr int kTC = 32 * kCh;  // channels per tile slice
   extern __shared__ uint8_t sm_raw[];
@@ -84,52 +86,49 @@ __global__ void __launch_bounds__(kConvThreads) dwconv3x3_k(const __grid_constan
   const uint32_t raw = smem_u32(sm_raw);
   const uint32_t sbuf = (raw + 1023u) & ~1023u;
   uint8_t* sm = sm_raw + (sbuf - raw);
-  const uint32_t bar0 = sbuf + 2u * kBufBytes;
+  const uint32_t bar0 = sbuf + (uint32_t)kConvBufs * kBufBytes;
   const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-  auto tile_coords = [&](int tile, int& b, int& ty, int& tx, int& ct) {
-    ct = tile % nct;
-    int r = tile / nct;
-    tx = r % ntx;
-    r /= ntx;
+  // Every block keeps one channel slice (its weights stay in registers) and walks the
+  // spatial tiles sp = blockIdx.x / nct + k * (gridDim.x / nct).
+  const int ct = blockIdx.x % nct, bpc = gridDim.x / nct, sp0 = blockIdx.x / nct;
+  auto spatial = [&](int sp, int& b, int& ty, int& tx) {
+    tx = sp % ntx;
+    const int r = sp / ntx;
     ty = r % nty;
     b = r / nty;
   };
-  auto issue = [&](int tile, int buf) {
-    int b, ty, tx, ct;
-    tile_coords(tile, b, ty, tx, ct);
+  auto issue = [&](int k, int buf) {
+    int b, ty, tx;
+    spatial(sp0 + k * bpc, b, ty, tx);
     mbar_expect_tx(bar0 + 8u * buf, kTileBytes);
-    tma_load_4d(sbuf + (uint32_t)buf * kBufBytes, &xmap, ct * kTC, tx * kTile - 1, ty * kTile - 1, b, bar0 + 8u * buf);
+    tma_load_4d(sbuf + (uint32_t)buf * kBufBytes, &xmap, ct * kTC, tx * kTileC - 1, ty * kTileR - 1, b, bar0 + 8u * buf);
   };
   if (threadIdx.x == 0) {
-    mbar_init(bar0, 1);
-    mbar_init(bar0 + 8, 1);
+    for (int q = 0; q < kConvBufs; ++q) mbar_init(bar0 + 8u * q, 1);
     fence_mbar_init();
-    if ((int)blockIdx.x < ntiles) issue(blockIdx.x, 0);
-    if ((int)(blockIdx.x + gridDim.x) < ntiles) issue(blockIdx.x + gridDim.x, 1);
+    for (int q = 0; q < kConvBufs; ++q)
+      if (sp0 + q * bpc < nsp) issue(q, q);
   }
   __syncthreads();
-  int ct_w = -1;
-  float2 wt[9];
-  for (int k = 0;; ++k) {
-    const int tile = blockIdx.x + k * gridDim.x;
-    if (tile >= ntiles) break;
-    const int buf = k & 1;
-    int b, ty, tx, ct;
-    tile_coords(tile, b, ty, tx, ct);
-    const int c = ct * kTC + kCh * lane;  // first channel of this lane
-    if (ct != ct_w) {  // weights of this lane's channels (zero past C)
-      ct_w = ct;
+  const int c = ct * kTC + kCh * lane;  // first channel of this lane
+  float2 wt[9];  // weights of this lane's channels (zero past C)
 #pragma unroll
-      for (int t = 0; t < 9; ++t) {
-        wt[t].x = c < C ? __ldg(w + (int64_t)c * 9 + t) : 0.f;
-        wt[t].y = (kCh == 2 && c + 1 < C) ? __ldg(w + (int64_t)(c + 1) * 9 + t) : 0.f;
-      }
-    }
+  for (int t = 0; t < 9; ++t) {
+    wt[t].x = c < C ? __ldg(w + (int64_t)c * 9 + t) : 0.f;
+    wt[t].y = (kCh == 2 && c + 1 < C) ? __ldg(w + (int64_t)(c + 1) * 9 + t) : 0.f;
+  }
+  for (int k = 0;; ++k) {
+    const int sp = sp0 + k * bpc;
+    if (sp >= nsp) break;
+    const int buf = k % kConvBufs;
+    const uint32_t par = (uint32_t)((k / kConvBufs) & 1);
+    int b, ty, tx;
+    spatial(sp, b, ty, tx);
     // Bounded wait for the tile; the block leaves together if it expires.
     bool late = false;
-    if (!mbar_try_wait(bar0 + 8u * buf, (uint32_t)((k >> 1) & 1))) {
+    if (!mbar_try_wait(bar0 + 8u * buf, par)) {
       const long long t0 = clock64();
-      while (!mbar_try_wait(bar0 + 8u * buf, (uint32_t)((k >> 1) & 1)))
+      while (!mbar_try_wait(bar0 + 8u * buf, par))
         if (clock64() - t0 > kWaitCycles) {
           late = true;
           break;
@@ -138,44 +137,52 @@ __global__ void __launch_bounds__(kConvThreads) dwconv3x3_k(const __grid_constan
     if (__syncthreads_or(late)) {
       if (threadIdx.x == 0) {
         report_status(GLA_ERR_TIMEOUT);
-        // Let the loads already issued into either buffer land before leaving (bounded).
-        for (int kk = k; kk < k + 2 && (int)(blockIdx.x + kk * gridDim.x) < ntiles; ++kk) {
+        // Let the loads already issued into the ring land before leaving (bounded).
+        for (int kk = k; kk < k + kConvBufs && sp0 + kk * bpc < nsp; ++kk) {
           const long long t0 = clock64();
-          while (!mbar_try_wait(bar0 + 8u * (kk & 1), (uint32_t)((kk >> 1) & 1)) && clock64() - t0 < kWaitCycles) {
+          while (!mbar_try_wait(bar0 + 8u * (kk % kConvBufs), (uint32_t)((kk / kConvBufs) & 1)) &&
+                 clock64() - t0 < kWaitCycles) {
           }
         }
       }
       return;
     }
     const uint32_t* tl = reinterpret_cast<const uint32_t*>(sm + (uint32_t)buf * kBufBytes);
-    auto at = [&](int r, int cc) -> uint32_t { return tl[(r * kHalo + cc) * 32 + lane]; };
-    const int x0 = tx * kTile + 2 * wp, y0 = ty * kTile;
-    uint32_t win[3][4];
+    auto at = [&](int r, int cc) -> uint32_t { return tl[(r * kHaloC + cc) * 32 + lane]; };
+    const int x0 = tx * kTileC + 2 * wp, y0 = ty * kTileR;
+    // Window of input values as fp32 (converted once, when a row enters it).
+    float2 win[3][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      win[0][j] = at(0, 2 * wp + j);
-      win[1][j] = at(1, 2 * wp + j);
+      win[0][j] = Lane4<T>::get(at(0, 2 * wp + j));
+      win[1][j] = Lane4<T>::get(at(1, 2 * wp + j));
     }
-    T* out = y + ((int64_t)b * Hg * Wg) * C + c;
-#pragma unroll 4
-    for (int r = 0; r < kTile; ++r) {
+    // Output pointer of (row y0, column x0) for this lane; rows advance by Wg * C.
+    T* out = y + (((int64_t)b * Hg + y0) * Wg + x0) * C + c;
+    const int64_t rstride = (int64_t)Wg * C;
+    const bool ok0 = c < C && x0 < Wg, ok1 = c < C && x0 + 1 < Wg;
+    const int rows = min(kTileR, Hg - y0);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) win[2][j] = at(r + 2, 2 * wp + j);
+    for (int r = 0; r < kTileR; ++r) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) win[2][j] = Lane4<T>::get(at(r + 2, 2 * wp + j));
+      float2 acc[2];
 #pragma unroll
       for (int oc = 0; oc < 2; ++oc) {
-        float2 acc = make_float2(0.f, 0.f);
+        acc[oc] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int di = 0; di < 3; ++di)
 #pragma unroll
           for (int dj = 0; dj < 3; ++dj) {
-            const float2 v = Lane4<T>::get(win[di][oc + dj]);
-            acc.x = fmaf(wt[di * 3 + dj].x, v.x, acc.x);
-            acc.y = fmaf(wt[di * 3 + dj].y, v.y, acc.y);
+            acc[oc].x = fmaf(wt[di * 3 + dj].x, win[di][oc + dj].x, acc[oc].x);
+            if (kCh == 2) acc[oc].y = fmaf(wt[di * 3 + dj].y, win[di][oc + dj].y, acc[oc].y);
           }
-        const int yy = y0 + r, xx = x0 + oc;
-        if (yy < Hg && xx < Wg && c < C)
-          *reinterpret_cast<uint32_t*>(out + ((int64_t)yy * Wg + xx) * C) = Lane4<T>::put(acc);
       }
+      if (r < rows) {
+        if (ok0) *reinterpret_cast<uint32_t*>(out) = Lane4<T>::put(acc[0]);
+        if (ok1) *reinterpret_cast<uint32_t*>(out + C) = Lane4<T>::put(acc[1]);
+      }
+      out += rstride;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         win[0][j] = win[1][j];
@@ -183,7 +190,7 @@ __global__ void __launch_bounds__(kConvThreads) dwconv3x3_k(const __grid_constan
       }
     }
     __syncthreads();  // the buffer is read out before it is refilled
-    if (threadIdx.x == 0 && tile + 2 * (int)gridDim.x < ntiles) issue(tile + 2 * gridDim.x, buf);
+    if (threadIdx.x == 0 && sp + kConvBufs * bpc < nsp) issue(k + kConvBufs, buf);
   }
 }
 
@@ -214,30 +221,33 @@ cudaError_t dwconv3x3_launch(const void* x, const float* w, void* y, int B, int 
   CUtensorMap map;
   const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)Wg, (cuuint64_t)Hg, (cuuint64_t)B};
   const cuuint64_t strides[3] = {(cuuint64_t)C * esz, (cuuint64_t)Wg * C * esz, (cuuint64_t)Hg * Wg * C * esz};
-  const cuuint32_t box[4] = {(cuuint32_t)tc, (cuuint32_t)kHalo, (cuuint32_t)kHalo, 1};
+  const cuuint32_t box[4] = {(cuuint32_t)tc, (cuuint32_t)kHaloC, (cuuint32_t)kHaloR, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   if (fn(&map, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(x), dims,
          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  const int ntx = (Wg + kTile - 1) / kTile, nty = (Hg + kTile - 1) / kTile, nct = (C + tc - 1) / tc;
-  const int ntiles = B * nty * ntx * nct;
+  const int ntx = (Wg + kTileC - 1) / kTileC, nty = (Hg + kTileR - 1) / kTileR, nct = (C + tc - 1) / tc;
+  const int nsp = B * nty * ntx;  // spatial tiles
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = ntiles < 2 * sms ? ntiles : 2 * sms;  // two blocks per SM, each double-buffered
+  // About two blocks per SM, a whole number of blocks per channel slice.
+  int bpc = (2 * sms) / nct;
+  bpc = bpc < 1 ? 1 : (bpc > nsp ? nsp : bpc);
+  const int grid = bpc * nct;
   const size_t smem = kConvSmem;
   cudaError_t e;
   if (bf) {
     e = cudaFuncSetAttribute(dwconv3x3_k<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dwconv3x3_k<__nv_bfloat16><<<grid, kConvThreads, smem, st>>>(map, w, static_cast<__nv_bfloat16*>(y), Hg, Wg, C,
-                                                                   ntx, nty, nct, ntiles);
+                                                                   ntx, nty, nct, nsp);
   } else {
     e = cudaFuncSetAttribute(dwconv3x3_k<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dwconv3x3_k<float><<<grid, kConvThreads, smem, st>>>(map, w, static_cast<float*>(y), Hg, Wg, C, ntx, nty, nct,
-                                                         ntiles);
+                                                         nsp);
   }
   return cudaGetLastError();
 }
