@@ -64,8 +64,9 @@ constexpr int kMaxStages = 2;
 
 // mbarrier indices (8 bytes each)
 enum {
-  kBarFull = 0,                       // [S]  tiles landed (or an end-of-stream job posted)
-  kBarSuf = kBarFull + kMaxStages,    // [S][4] suffix sums of a 32-row quarter done (64 arrivals)
+  kBarFull = 0,                       // [S]  log-gate tile landed (or an end-of-stream job posted)
+  kBarOps = kBarFull + kMaxStages,    // [S]  q, k, v tiles landed
+  kBarSuf = kBarOps + kMaxStages,     // [S][4] suffix sums of a 32-row quarter done (64 arrivals)
   kBarGate = kBarSuf + 4 * kMaxStages,  // [S]  gates applied (128 arrivals)
   kBarEmpty = kBarGate + kMaxStages,  // [S]  stage free (MMA commit, or the serial path)
   kBarMail = kBarEmpty + kMaxStages,  // pass-2 job handed to the output group
@@ -327,23 +328,24 @@ __device__ __forceinline__ void chunk_box(const WsArgs& a, int cf, int& y, int& 
 // ---------------------------------------------------------------------------
 // Producer
 // ---------------------------------------------------------------------------
-__device__ void tma_job(const WsArgs& a, const TensorMaps& tm, uint32_t st, uint32_t bar, int cf, bool with_q, int b,
-                        int h) {
-  const uint32_t bytes = (uint32_t)(with_q ? 2 : 1) * (uint32_t)a.Kp * 256u + (uint32_t)a.Np * 256u +
-                         (uint32_t)MC * (uint32_t)(a.dk + 4) * 4u;
-  mbar_expect_tx(bar, bytes);
+// The log-gate tile is issued first, on its own barrier, so that the suffix sums can
+// start while the operand tiles are still arriving.
+__device__ void tma_job(const WsArgs& a, const TensorMaps& tm, uint32_t st, uint32_t bar_la, uint32_t bar_ops, int cf,
+                        bool with_q, int b, int h) {
   int y, x;
   chunk_box(a, cf, y, x);
   // Pass 2 is the last use of every tile: mark its lines first to go, so that the
   // pass-1 tiles waiting for their second read stay in L2.
   const uint64_t pol = with_q ? l2_policy_evict_first() : l2_policy_evict_normal();
+  mbar_expect_tx(bar_la, (uint32_t)MC * (uint32_t)(a.dk + 4) * 4u);
+  tma_load_5d(st + a.oLA, &tm.la, 0, h, y, x, b, bar_la, pol);
+  mbar_expect_tx(bar_ops, (uint32_t)(with_q ? 2 : 1) * (uint32_t)a.Kp * 256u + (uint32_t)a.Np * 256u);
   for (int cb = 0; cb < (a.Kp >> 4); ++cb) {
-    tma_load_5d(st + a.oK + (uint32_t)cb * ATOM32, &tm.k, cb * 16, h, y, x, b, bar, pol);
-    if (with_q) tma_load_5d(st + a.oQ + (uint32_t)cb * ATOM32, &tm.q, cb * 16, h, y, x, b, bar, pol);
+    tma_load_5d(st + a.oK + (uint32_t)cb * ATOM32, &tm.k, cb * 16, h, y, x, b, bar_ops, pol);
+    if (with_q) tma_load_5d(st + a.oQ + (uint32_t)cb * ATOM32, &tm.q, cb * 16, h, y, x, b, bar_ops, pol);
   }
   for (int cb = 0; cb < (a.Np >> 4); ++cb)
-    tma_load_5d(st + a.oV + (uint32_t)cb * ATOM32, &tm.v, cb * 16, h, y, x, b, bar, pol);
-  tma_load_5d(st + a.oLA, &tm.la, 0, h, y, x, b, bar, pol);
+    tma_load_5d(st + a.oV + (uint32_t)cb * ATOM32, &tm.v, cb * 16, h, y, x, b, bar_ops, pol);
 }
 
 // ---------------------------------------------------------------------------
@@ -611,6 +613,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
   if (tid == 0) {
     for (int s = 0; s < a.nstage; ++s) {
       mbar_init(BAR(kBarFull + s), 1);
+      mbar_init(BAR(kBarOps + s), 1);
       for (int qd = 0; qd < 4; ++qd) mbar_init(BAR(kBarSuf + 4 * s + qd), 64);
       mbar_init(BAR(kBarGate + s), 128);
       mbar_init(BAR(kBarEmpty + s), 1);
@@ -661,11 +664,12 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         sJob[4 * s + 3] = buf;
         if (kind == kJobEnd) {
           mbar_arrive(BAR(kBarFull + s));
+          mbar_arrive(BAR(kBarOps + s));
         } else {
           const Item it = decode_item(a, item);
           const int c = kind == kJobP1 ? it.c0 + it.n - 1 - j : it.c0 + j;  // pass 1 walks backwards
-          tma_job(a, tm, sbase + (uint32_t)s * a.stage_bytes, BAR(kBarFull + s), fwd_chunk(a, c), kind == kJobP2,
-                  it.b, it.h);
+          tma_job(a, tm, sbase + (uint32_t)s * a.stage_bytes, BAR(kBarFull + s), BAR(kBarOps + s), fwd_chunk(a, c),
+                  kind == kJobP2, it.b, it.h);
         }
         sMisc[3] = ++jc;
         return true;
@@ -913,6 +917,10 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         }
         kind = sJob[4 * s];
         if (kind == kJobEnd) break;
+        if (m == 0 && !wait_bar(BAR(kBarOps + s), (uint32_t)(use & 1), abort_flag)) {  // q, k, v landed
+          ok_wait = false;
+          break;
+        }
         const bool pass1 = kind == kJobP1;
         const int r = 32 * quarter + lane;
         const float* urow = reinterpret_cast<const float*>(st + a.oLA) + r * (a.dk + 4);
@@ -1159,10 +1167,14 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
   // ---------------------------------------------------------------- teardown
   __syncthreads();
   if (*abort_flag && tid == 0) {
-    // Let loads still in flight land before the shared memory is released.
-    for (int jj = sMisc[4]; jj < sMisc[3]; ++jj) {
-      const long long t0 = clock64();
-      while (!mbar_try_wait(BAR(kBarFull + jj % S), (uint32_t)((jj / S) & 1)) && clock64() - t0 < kWaitCycles) {
+    // Let loads still in flight land before the shared memory is released: only the
+    // last S posted jobs can still have any (earlier stages were reposted).
+    for (int jj = max(sMisc[3] - S, 0); jj < sMisc[3]; ++jj) {
+      for (int bb = 0; bb < 2; ++bb) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(BAR((bb ? kBarOps : kBarFull) + jj % S), (uint32_t)((jj / S) & 1)) &&
+               clock64() - t0 < kWaitCycles) {
+        }
       }
     }
   }
