@@ -17,18 +17,18 @@
 // Chunks whose gates decay by more than e^80 inside the chunk are evaluated token by
 // token from the running state instead (exact).
 //
-// Roles (16 warps, 512 threads), connected by mbarriers:
+// Roles (16 warps, 512 threads; warps 2-3 idle), connected by mbarriers:
 //   warp 0      producer: takes tickets and posts jobs (pass 1 of the next item, then
 //               pass 2 of the current one); TMA loads of each chunk's q, k, v
 //               (32-byte-swizzled 16-channel boxes, the UMMA operand layout) and
 //               log-gates into a ring of stages;
 //   warp 1      MMA issuer (tcgen05, one thread) and TMEM owner;
-//   warps 2-3   suffix sums of the log-gates, one thread per pair of key channels,
-//               released to the gate warps 32 rows at a time;
-//   warps 4-7   gates applied in place (K^, Q~): lane = row of the released quarter,
-//               warp = set of 8-channel blocks;
-//   warps 8-11  output group, one thread per TMEM lane: score masking to bf16 P,
-//               G = Diag(gamma) S, output epilogue, serial path;
+//   warps 4-7   gate group, warp = quarter of the chunk's rows: suffix sums of the
+//               log-gates over the quarter (lane = pair of key channels), then the
+//               gates applied in place (K^, Q~; lane = row), then the score masking
+//               to bf16 P (lane = TMEM lane);
+//   warps 8-11  output group, one thread per TMEM lane: G = Diag(gamma) S, output
+//               epilogue, serial path;
 //   warps 12-15 look-back group, one thread per TMEM lane.
 // TMEM (512 columns): scores [0,128) -- overwritten by the bf16 P matrix (two keys per
 // column, the A operand of P V) --, O (two buffers when dv <= 96), and two buffers
@@ -55,7 +55,7 @@ namespace {
 
 constexpr int MC = kChunkTC;
 constexpr int NT = 512;
-constexpr int kWarpProd = 0, kWarpMma = 1, kWarpSuf = 2, kWarpGate = 4, kWarpEpi = 8, kWarpLb = 12;
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpGate = 4, kWarpEpi = 8, kWarpLb = 12;
 constexpr uint32_t ATOM32 = MC * 32u;    // one 16-channel block of a 32B-swizzled 128-row tile
 constexpr float kMaxGateRange = 80.0f;
 constexpr uint32_t kColS = 0;
@@ -66,8 +66,7 @@ constexpr int kMaxStages = 2;
 enum {
   kBarFull = 0,                       // [S]  log-gate tile landed (or an end-of-stream job posted)
   kBarOps = kBarFull + kMaxStages,    // [S]  q, k, v tiles landed
-  kBarSuf = kBarOps + kMaxStages,     // [S][4] suffix sums of a 32-row quarter done (64 arrivals)
-  kBarGate = kBarSuf + 4 * kMaxStages,  // [S]  gates applied (128 arrivals)
+  kBarGate = kBarOps + kMaxStages,    // [S]  gates applied (128 arrivals)
   kBarEmpty = kBarGate + kMaxStages,  // [S]  stage free (MMA commit, or the serial path)
   kBarMail = kBarEmpty + kMaxStages,  // pass-2 job handed to the output group
   kBarScFull,                         // score MMA done
@@ -101,7 +100,7 @@ struct WsArgs {
   int Kp, Np, nstage, nO, nbuf;
   uint32_t colO0, colO1, colSeg0, colSeg1, colSeg2;
   int mode, rpc, ppr;  // chunk geometry: 0 raster, 1 whole columns (rpc per chunk), 2 column pieces (ppr per column)
-  uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oMisc, oJob, oMail, oItem, oBar, oTm;
+  uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oTot, oOff, oMisc, oJob, oMail, oItem, oBar, oTm;
   ScanGeom g;
   __device__ __forceinline__ uint32_t col_seg(int buf) const {
     return buf == 0 ? colSeg0 : (buf == 1 ? colSeg1 : colSeg2);
@@ -597,7 +596,9 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
   volatile int* sWide = reinterpret_cast<volatile int*>(smem + a.oWide);  // [S] chunk evaluated serially
   float* sGam = reinterpret_cast<float*>(smem + a.oGam);    // [3][128] exp(segment gate sum)
   float* red = reinterpret_cast<float*>(smem + a.oRed);     // serial-path reduction [4][16]
-  // [0] first item [1] abort [2] look-back flag [3] jobs posted [4] jobs taken [5] end item index
+  float* sTot = reinterpret_cast<float*>(smem + a.oTot);    // [4][128] log-gate sums of the row quarters
+  float* sOff = reinterpret_cast<float*>(smem + a.oOff);    // [4][128] log-gate sums after each quarter
+  // [0] first item [1] abort [2] look-back flag [3] jobs posted [5] end item index
   volatile int* sMisc = reinterpret_cast<volatile int*>(smem + a.oMisc);
   volatile int* sJob = reinterpret_cast<volatile int*>(smem + a.oJob);    // [S][4] kind, item, j, buf
   volatile int* sMail = reinterpret_cast<volatile int*>(smem + a.oMail);  // [4]    stage, wide, item, j
@@ -614,7 +615,6 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     for (int s = 0; s < a.nstage; ++s) {
       mbar_init(BAR(kBarFull + s), 1);
       mbar_init(BAR(kBarOps + s), 1);
-      for (int qd = 0; qd < 4; ++qd) mbar_init(BAR(kBarSuf + 4 * s + qd), 64);
       mbar_init(BAR(kBarGate + s), 128);
       mbar_init(BAR(kBarEmpty + s), 1);
     }
@@ -637,7 +637,6 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     sMisc[0] = atomicAdd(a.ticket, 1);
     sMisc[1] = 0;
     sMisc[3] = 0;
-    sMisc[4] = 0;
     sMisc[5] = 0x7fffffff;
   }
   for (int x = tid; x < kMaxStages * 128; x += NT) sBL[x] = 0.f;  // rows >= dk: gamma = 1
@@ -827,114 +826,145 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       }
     }
   } else if (warp < kWarpGate) {
-    // ------------------------------------------------------------ suffix sums
-    // In place over the log-gate tile: u_r = base + sum of the log-gates scanned after
-    // row r (base = the later chunks of the segment in pass 1, 0 in pass 2).  Rows are
-    // walked from the last scanned one; each finished quarter of 32 rows is released
-    // to the gate warp that owns it.
-    const int c = 2 * (tid - 32 * kWarpSuf);  // key channels c, c + 1
-    float2 off = make_float2(0.f, 0.f);
-    int ks = 0;  // items through pass 1
+    // warps 2-3 have no role
+  } else if (warp < kWarpEpi) {
+    // ------------------------------------------------------------ gates
+    // Gate warp gq owns rows 32gq..32gq+31 of every chunk (its TMEM subpartition).
+    // (A) lane = pair of key channels: exclusive suffix sums of the log-gates over the
+    //     warp's 32 rows in scan order, in place; the quarter totals go to sTot.
+    // (B) after the group barrier: u = local suffix + the totals of the later quarters
+    //     (+ the later chunks of the segment in pass 1); lane = row: K^ = k exp(u) and,
+    //     in pass 2, Q~ = q exp(-u), in place.  A chunk whose |u| exceeds the fp32-safe
+    //     range anywhere is evaluated serially instead (flagged here; the serial path
+    //     reads the raw q and k from global memory).
+    const int gq = warp - kWarpGate;
+    const int pw = a.dk + 4;             // log-gate row pitch in floats
+    const int np = (a.dk + 1) >> 1;      // key-channel pairs
+    const bool act0 = lane < np, act1 = lane + 32 < np;
+    float2 cy0 = make_float2(0.f, 0.f), cy1 = cy0;  // pass 1: later chunks of the segment
+    int ks = 0;   // items through pass 1
+    int kbg = 0;  // non-serial pass-2 jobs masked so far
     for (int jc = 0;; ++jc) {
       const int s = jc % S, use = jc / S;
-      if (!group_and(1, 64, wait_bar(BAR(kBarFull + s), (uint32_t)(use & 1), abort_flag))) break;
-      if (c == 0) sMisc[4] = jc + 1;
-      const int kind = sJob[4 * s], j = sJob[4 * s + 2], buf = sJob[4 * s + 3];
+      if (!group_and(4, 128, wait_bar(BAR(kBarFull + s), (uint32_t)(use & 1), abort_flag))) break;
+      const int kind = sJob[4 * s];
       if (kind == kJobEnd) {
-        for (int qd = 0; qd < 4; ++qd) mbar_arrive(BAR(kBarSuf + 4 * s + qd));
+        mbar_arrive(BAR(kBarGate + s));
         break;
       }
+      const int j = sJob[4 * s + 2], buf = sJob[4 * s + 3];
       const bool pass1 = kind == kJobP1;
       const bool last1 = pass1 && j == decode_item(a, sJob[4 * s + 1]).n - 1;
       // sGam[buf] is rewritten once the look-back of item ks - nbuf has read it.
       if (last1 && ks >= a.nbuf &&
-          !group_and(1, 64, wait_bar(BAR(kBarSinReady + buf), (uint32_t)(((ks / a.nbuf) - 1) & 1), abort_flag)))
+          !group_and(4, 128, wait_bar(BAR(kBarSinReady + buf), (uint32_t)(((ks / a.nbuf) - 1) & 1), abort_flag)))
         break;
-      if (pass1 && j == 0) off = make_float2(0.f, 0.f);
-      const bool act = c < a.dk;
-      const int pw = (a.dk + 4) >> 1;  // row pitch in float2
-      float2* ptr = reinterpret_cast<float2*>(smem + (uint32_t)s * a.stage_bytes + a.oLA) +
-                    (a.g.reverse ? 0 : (MC - 1)) * pw + (c >> 1);  // last scanned row first
-      const int step = a.g.reverse ? pw : -pw;
-      const float2 base = pass1 ? off : make_float2(0.f, 0.f);
-      float2 acc = base;
-#pragma unroll 1
-      for (int m = 0; m < 4; ++m) {
-        if (act) {
-#pragma unroll 1
-          for (int h16 = 0; h16 < 2; ++h16) {
-            // Sixteen rows are loaded before their stores so that the loads overlap.
-            float2 x[16];
-#pragma unroll
-            for (int q = 0; q < 16; ++q) x[q] = ptr[q * step];
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              ptr[q * step] = acc;
-              acc.x += x[q].x;
-              acc.y += x[q].y;
-            }
-            ptr += 16 * step;
-          }
-        }
-        if (m == 3 && act) {  // chunk totals before the last quarter is released
-          sBL[s * 128 + c] = acc.x - base.x;
-          sBL[s * 128 + c + 1] = acc.y - base.y;
-          if (pass1) {
-            off = acc;
-            if (last1) {
-              // exp(segment gate sum) of growth gates must stay finite
-              if (!(off.x <= kMaxGateRange) || !(off.y <= kMaxGateRange)) report_status(GLA_ERR_RANGE);
-              sGam[buf * 128 + c] = __expf(off.x);
-              sGam[buf * 128 + c + 1] = __expf(off.y);
-            }
-          }
-        }
-        mbar_arrive(BAR(kBarSuf + 4 * s + (a.g.reverse ? m : 3 - m)));
-      }
-      if (last1) ++ks;
-    }
-  } else if (warp < kWarpEpi) {
-    // ------------------------------------------------------------ gates
-    // K^ = k exp(u) (and Q~ = q exp(-u) in pass 2) in place.  Lane l of gate warp w
-    // gates row 32q + l of each quarter q, in the order the suffix pass releases them,
-    // on the 8-channel blocks w, w + 4, w + 8, ...  A chunk whose |u| exceeds the
-    // fp32-safe range anywhere is evaluated serially instead (flagged here; the serial
-    // path reads the raw q and k from global memory).
-    const int gw = warp - kWarpGate;
-    int kbg = 0;  // non-serial pass-2 jobs masked so far
-    for (int jc = 0;; ++jc) {
-      const int s = jc % S, use = jc / S;
-      int kind = kJobEnd;
-      bool ok_wait = true;
-      float umax = 0.f;  // pass 1: largest u; pass 2: largest |u|
+      if (pass1 && j == 0) cy0 = cy1 = make_float2(0.f, 0.f);
       uint8_t* st = smem + (uint32_t)s * a.stage_bytes;
+      float* lag = reinterpret_cast<float*>(st + a.oLA);
+      // (A) rows of the quarter in decreasing scan position
+      {
+        const int dr = a.g.reverse ? (pw >> 1) : -(pw >> 1);  // in float2
+        float2* p0 = reinterpret_cast<float2*>(lag + (a.g.reverse ? 32 * gq : 32 * gq + 31) * pw) + lane;
+        float2* p1 = p0 + 32;
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
 #pragma unroll 1
-      for (int m = 0; m < 4; ++m) {
-        const int quarter = a.g.reverse ? m : 3 - m;
-        if (!wait_bar(BAR(kBarSuf + 4 * s + quarter), (uint32_t)(use & 1), abort_flag)) {
-          ok_wait = false;
-          break;
+        for (int h8 = 0; h8 < 4; ++h8) {
+          float2 x0[8], x1[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            x0[q] = act0 ? p0[q * dr] : make_float2(0.f, 0.f);
+            x1[q] = act1 ? p1[q * dr] : make_float2(0.f, 0.f);
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (act0) p0[q * dr] = acc0;
+            if (act1) p1[q * dr] = acc1;
+            acc0.x += x0[q].x;
+            acc0.y += x0[q].y;
+            acc1.x += x1[q].x;
+            acc1.y += x1[q].y;
+          }
+          p0 += 8 * dr;
+          p1 += 8 * dr;
         }
-        kind = sJob[4 * s];
-        if (kind == kJobEnd) break;
-        if (m == 0 && !wait_bar(BAR(kBarOps + s), (uint32_t)(use & 1), abort_flag)) {  // q, k, v landed
-          ok_wait = false;
-          break;
+        float2* tot = reinterpret_cast<float2*>(sTot + gq * 128);
+        tot[lane] = acc0;
+        tot[lane + 32] = acc1;
+      }
+      named_sync(4, 128);
+      // Offsets of this quarter and the chunk totals, for pairs lane and lane + 32.
+      {
+        const float2* tot = reinterpret_cast<const float2*>(sTot);
+        float2 o0 = pass1 ? cy0 : make_float2(0.f, 0.f), o1 = pass1 ? cy1 : make_float2(0.f, 0.f);
+        float2 c0 = make_float2(0.f, 0.f), c1 = c0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 t0 = tot[q * 64 + lane], t1 = tot[q * 64 + lane + 32];
+          c0.x += t0.x;
+          c0.y += t0.y;
+          c1.x += t1.x;
+          c1.y += t1.y;
+          if (a.g.reverse ? q < gq : q > gq) {
+            o0.x += t0.x;
+            o0.y += t0.y;
+            o1.x += t1.x;
+            o1.y += t1.y;
+          }
         }
-        const bool pass1 = kind == kJobP1;
-        const int r = 32 * quarter + lane;
-        const float* urow = reinterpret_cast<const float*>(st + a.oLA) + r * (a.dk + 4);
+        float2* off = reinterpret_cast<float2*>(sOff + gq * 128);
+        off[lane] = o0;
+        off[lane + 32] = o1;
+        if (gq == 0) {
+          float2* bl = reinterpret_cast<float2*>(sBL + s * 128);  // chunk gate sums; channels >= dk stay 0
+          if (act0) bl[lane] = c0;
+          if (act1) bl[lane + 32] = c1;
+        }
+        if (pass1) {
+          cy0.x += c0.x;
+          cy0.y += c0.y;
+          cy1.x += c1.x;
+          cy1.y += c1.y;
+          if (last1 && gq == 0) {
+            // exp(segment gate sum) of growth gates must stay finite
+            bool bad = false;
+            if (act0) {
+              bad |= !(cy0.x <= kMaxGateRange) || !(cy0.y <= kMaxGateRange);
+              sGam[buf * 128 + 2 * lane] = __expf(cy0.x);
+              sGam[buf * 128 + 2 * lane + 1] = __expf(cy0.y);
+            }
+            if (act1) {
+              bad |= !(cy1.x <= kMaxGateRange) || !(cy1.y <= kMaxGateRange);
+              sGam[buf * 128 + 2 * lane + 64] = __expf(cy1.x);
+              sGam[buf * 128 + 2 * lane + 65] = __expf(cy1.y);
+            }
+            if (bad) report_status(GLA_ERR_RANGE);
+          }
+        }
+      }
+      __syncwarp();
+      if (last1) ++ks;
+      // (B) lane = row; q, k, v landed
+      if (!group_and(4, 128, wait_bar(BAR(kBarOps + s), (uint32_t)(use & 1), abort_flag))) break;
+      float umax = 0.f;  // pass 1: largest u; pass 2: largest |u|
+      {
+        const int r = 32 * gq + lane;
+        const float* urow = lag + r * pw;
+        const float* offq = sOff + gq * 128;
         // exp(u) is rounded to bf16 pairs and applied with packed bf16 multiplies,
         // exp(-u) as its reciprocal.
 #pragma unroll 1
-        for (int cc = 8 * gw; cc < a.dk; cc += 32) {
+        for (int cc = 0; cc < a.dk; cc += 8) {
           const uint32_t o = sw32_off((uint32_t)r, (uint32_t)cc);
           const float4 u0 = *reinterpret_cast<const float4*>(urow + cc);
           const float4 u1 = *reinterpret_cast<const float4*>(urow + cc + 4);
+          const float4 f0 = *reinterpret_cast<const float4*>(offq + cc);
+          const float4 f1 = *reinterpret_cast<const float4*>(offq + cc + 4);
           uint4 kw = *reinterpret_cast<const uint4*>(st + a.oK + o);
           uint4 qw = make_uint4(0u, 0u, 0u, 0u);
           if (!pass1) qw = *reinterpret_cast<const uint4*>(st + a.oQ + o);
-          const float ev[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+          const float ev[8] = {u0.x + f0.x, u0.y + f0.y, u0.z + f0.z, u0.w + f0.w,
+                               u1.x + f1.x, u1.y + f1.y, u1.z + f1.z, u1.w + f1.w};
           uint32_t* uk = reinterpret_cast<uint32_t*>(&kw);
           uint32_t* uq = reinterpret_cast<uint32_t*>(&qw);
 #pragma unroll
@@ -949,68 +979,60 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
           if (!pass1) *reinterpret_cast<uint4*>(st + a.oQ + o) = qw;
         }
       }
-      if (!ok_wait) break;
-      if (kind == kJobEnd) {
-        mbar_arrive(BAR(kBarGate + s));
-        break;
-      }
       fence_proxy_async_smem();
-      const bool pass1 = kind == kJobP1;
       // NaN compares false: a NaN or infinite u also counts as out of range.
       bool bad = !(umax <= kMaxGateRange);
-      if (!pass1 && gw == 0)
+      if (!pass1 && gq == 0)
         for (int cc = lane; cc < a.dk; cc += 32) bad |= !(sBL[s * 128 + cc] <= kMaxGateRange);  // exp(chunk sum)
       if (pass1) {
         if (bad) report_status(GLA_ERR_RANGE);  // exp(u) of growth gates overflows
-      } else {
-        const bool wide = group_or(4, 128, bad);
-        if (gw == 0 && lane == 0) sWide[s] = wide;
         mbar_arrive(BAR(kBarGate + s));
-        if (!wide) {
-          // scores -> mask (keys scanned no later than the row) -> bf16 P in TMEM.
-          // Warp w owns TMEM lanes (rows) 32w..32w+31.
-          if (!group_and(4, 128, wait_bar(BAR(kBarScFull), (uint32_t)(kbg & 1), abort_flag))) break;
-          ++kbg;
-          tc_fence_after();
-          const int i = 32 * gw + lane;
-          const uint32_t lane_base = (uint32_t)(32 * gw) << 16;
-          {
-            const int rlo = 32 * (warp & 3), rhi = rlo + 31;
-#pragma unroll 1
-            for (int cb = 0; cb < MC; cb += 32) {
-              const bool none = a.g.reverse ? (cb + 31 < rlo) : (cb > rhi);
-              const bool all = a.g.reverse ? (cb >= rhi) : (cb + 31 <= rlo);
-              uint32_t sc[2][16];
-              if (!none) tmem_ld_cols<2>(tbase + kColS + lane_base + (uint32_t)cb, 32, sc);
-              uint32_t pk[16];
-              if (none) {
-#pragma unroll
-                for (int q = 0; q < 16; ++q) pk[q] = 0u;
-              } else if (all) {
-#pragma unroll
-                for (int q = 0; q < 32; q += 2) pk[q >> 1] = pack_u2(sc[q >> 4][q & 15], sc[q >> 4][(q & 15) + 1]);
-              } else {
-#pragma unroll
-                for (int q = 0; q < 32; q += 2) {
-                  const int s0 = cb + q, s1 = cb + q + 1;
-                  const bool k0 = a.g.reverse ? (s0 >= i) : (s0 <= i);
-                  const bool k1 = a.g.reverse ? (s1 >= i) : (s1 <= i);
-                  const float v0 = __uint_as_float(sc[q >> 4][q & 15]);
-                  const float v1 = __uint_as_float(sc[q >> 4][(q & 15) + 1]);
-                  pk[q >> 1] = pack_bf16x2(k0 ? v0 : 0.f, k1 ? v1 : 0.f);
-                }
-              }
-              // bf16 pairs of keys overwrite score columns this thread has already read.
-              tmem_st16u(tbase + kColS + lane_base + (uint32_t)(cb >> 1), pk);
-            }
-          }
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(BAR(kBarPReady));
-        }
         continue;
       }
+      const bool wide = group_or(4, 128, bad);
+      if (gq == 0 && lane == 0) sWide[s] = wide;
       mbar_arrive(BAR(kBarGate + s));
+      if (wide) continue;
+      // scores -> mask (keys scanned no later than the row) -> bf16 P in TMEM.
+      // Warp gq owns TMEM lanes (rows) 32gq..32gq+31.
+      if (!group_and(4, 128, wait_bar(BAR(kBarScFull), (uint32_t)(kbg & 1), abort_flag))) break;
+      ++kbg;
+      tc_fence_after();
+      const int i = 32 * gq + lane;
+      const uint32_t lane_base = (uint32_t)(32 * gq) << 16;
+      {
+        const int rlo = 32 * gq, rhi = rlo + 31;
+#pragma unroll 1
+        for (int cb = 0; cb < MC; cb += 32) {
+          const bool none = a.g.reverse ? (cb + 31 < rlo) : (cb > rhi);
+          const bool all = a.g.reverse ? (cb >= rhi) : (cb + 31 <= rlo);
+          uint32_t sc[2][16];
+          if (!none) tmem_ld_cols<2>(tbase + kColS + lane_base + (uint32_t)cb, 32, sc);
+          uint32_t pk[16];
+          if (none) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) pk[q] = 0u;
+          } else if (all) {
+#pragma unroll
+            for (int q = 0; q < 32; q += 2) pk[q >> 1] = pack_u2(sc[q >> 4][q & 15], sc[q >> 4][(q & 15) + 1]);
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; q += 2) {
+              const int s0 = cb + q, s1 = cb + q + 1;
+              const bool k0 = a.g.reverse ? (s0 >= i) : (s0 <= i);
+              const bool k1 = a.g.reverse ? (s1 >= i) : (s1 <= i);
+              const float v0 = __uint_as_float(sc[q >> 4][q & 15]);
+              const float v1 = __uint_as_float(sc[q >> 4][(q & 15) + 1]);
+              pk[q >> 1] = pack_bf16x2(k0 ? v0 : 0.f, k1 ? v1 : 0.f);
+            }
+          }
+          // bf16 pairs of keys overwrite score columns this thread has already read.
+          tmem_st16u(tbase + kColS + lane_base + (uint32_t)(cb >> 1), pk);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(BAR(kBarPReady));
     }
   } else if (warp < kWarpLb) {
     // ------------------------------------------------------------ output group (pass 2)
@@ -1185,7 +1207,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
 
 struct WsLayout {
   int NC, NS, G, Kp, Np, nstage, mode, rpc, ppr;
-  uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oMisc, oJob, oMail, oItem, oBar, oTm;
+  uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oTot, oOff, oMisc, oJob, oMail, oItem, oBar, oTm;
   int nO, nbuf;
   uint32_t colO0, colO1, colSeg0, colSeg1, colSeg2;
   size_t smem;
@@ -1228,7 +1250,7 @@ WsLayout ws_layout(const GlaShape& s) {
   // channel blocks from oK; the stage is at least that large.
   L.stage_bytes = al1024(L.oLA + la > 8 * ATOM32 ? L.oLA + la : 8 * ATOM32);
   const uint32_t gtile = al1024((uint32_t)L.Kp * (uint32_t)L.Np * 2u);
-  const uint32_t fixed = gtile + kMaxStages * 512 + 256 + 1536 + 256 + 64 + 16 * kMaxStages + 16 + 32 +
+  const uint32_t fixed = gtile + kMaxStages * 512 + 256 + 1536 + 256 + 4096 + 64 + 16 * kMaxStages + 16 + 32 +
                          8 * kNumBars + 16;
   L.nstage = (1024 + 2 * (size_t)L.stage_bytes + fixed <= kMaxSmem) ? 2 : 1;
   L.oG = (uint32_t)L.nstage * L.stage_bytes;
@@ -1236,7 +1258,9 @@ WsLayout ws_layout(const GlaShape& s) {
   L.oWide = L.oBL + kMaxStages * 512;
   L.oGam = L.oWide + 256;
   L.oRed = L.oGam + 1536;
-  L.oMisc = L.oRed + 256;
+  L.oTot = L.oRed + 256;
+  L.oOff = L.oTot + 2048;
+  L.oMisc = L.oOff + 2048;
   L.oJob = L.oMisc + 64;
   L.oMail = L.oJob + 16 * kMaxStages;
   L.oItem = L.oMail + 16;
@@ -1342,6 +1366,8 @@ cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const fl
   a.oWide = L.oWide;
   a.oGam = L.oGam;
   a.oRed = L.oRed;
+  a.oTot = L.oTot;
+  a.oOff = L.oOff;
   a.oMisc = L.oMisc;
   a.oJob = L.oJob;
   a.oMail = L.oMail;
