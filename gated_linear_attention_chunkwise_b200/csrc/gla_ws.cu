@@ -17,16 +17,16 @@
 // Chunks whose gates decay by more than e^80 inside the chunk are evaluated token by
 // token from the running state instead (exact).
 //
-// Roles (16 warps, 512 threads; warps 2-3 idle), connected by mbarriers:
+// Roles (16 warps, 512 threads), connected by mbarriers:
 //   warp 0      producer: takes tickets and posts jobs (pass 1 of the next item, then
 //               pass 2 of the current one); TMA loads of each chunk's q, k, v
 //               (32-byte-swizzled 16-channel boxes, the UMMA operand layout) and
 //               log-gates into a ring of stages;
 //   warp 1      MMA issuer (tcgen05, one thread) and TMEM owner;
-//   warps 4-7   gate group, warp = quarter of the chunk's rows: suffix sums of the
-//               log-gates over the quarter (lane = pair of key channels), then the
-//               gates applied in place (K^, Q~; lane = row), then the score masking
-//               to bf16 P (lane = TMEM lane);
+//   warps 2-3   suffix sums of the log-gates, two row quarters per warp in parallel
+//               (lane = pair of key channels), and each quarter's offset;
+//   warps 4-7   gate group, warp = quarter of the chunk's rows: the gates applied in
+//               place (K^, Q~; lane = row), then the score masking to bf16 P;
 //   warps 8-11  output group, one thread per TMEM lane: G = Diag(gamma) S, output
 //               epilogue, serial path;
 //   warps 12-15 look-back group, one thread per TMEM lane.
@@ -55,7 +55,7 @@ namespace {
 
 constexpr int MC = kChunkTC;
 constexpr int NT = 512;
-constexpr int kWarpProd = 0, kWarpMma = 1, kWarpGate = 4, kWarpEpi = 8, kWarpLb = 12;
+constexpr int kWarpProd = 0, kWarpMma = 1, kWarpSuf = 2, kWarpGate = 4, kWarpEpi = 8, kWarpLb = 12;
 constexpr uint32_t ATOM32 = MC * 32u;    // one 16-channel block of a 32B-swizzled 128-row tile
 constexpr float kMaxGateRange = 80.0f;
 constexpr uint32_t kColS = 0;
@@ -66,7 +66,8 @@ constexpr int kMaxStages = 2;
 enum {
   kBarFull = 0,                       // [S]  log-gate tile landed (or an end-of-stream job posted)
   kBarOps = kBarFull + kMaxStages,    // [S]  q, k, v tiles landed
-  kBarGate = kBarOps + kMaxStages,    // [S]  gates applied (128 arrivals)
+  kBarSufDone = kBarOps + kMaxStages, // [S]  suffix sums and quarter offsets done (64 arrivals)
+  kBarGate = kBarSufDone + kMaxStages,  // [S]  gates applied (128 arrivals)
   kBarEmpty = kBarGate + kMaxStages,  // [S]  stage free (MMA commit, or the serial path)
   kBarMail = kBarEmpty + kMaxStages,  // pass-2 job handed to the output group
   kBarScFull,                         // score MMA done
@@ -597,7 +598,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
   float* sGam = reinterpret_cast<float*>(smem + a.oGam);    // [3][128] exp(segment gate sum)
   float* red = reinterpret_cast<float*>(smem + a.oRed);     // serial-path reduction [4][16]
   float* sTot = reinterpret_cast<float*>(smem + a.oTot);    // [4][128] log-gate sums of the row quarters
-  float* sOff = reinterpret_cast<float*>(smem + a.oOff);    // [4][128] log-gate sums after each quarter
+  float* sOff = reinterpret_cast<float*>(smem + a.oOff);    // [S][4][128] log-gate sums after each quarter
   // [0] first item [1] abort [2] look-back flag [3] jobs posted [5] end item index
   volatile int* sMisc = reinterpret_cast<volatile int*>(smem + a.oMisc);
   volatile int* sJob = reinterpret_cast<volatile int*>(smem + a.oJob);    // [S][4] kind, item, j, buf
@@ -615,6 +616,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     for (int s = 0; s < a.nstage; ++s) {
       mbar_init(BAR(kBarFull + s), 1);
       mbar_init(BAR(kBarOps + s), 1);
+      mbar_init(BAR(kBarSufDone + s), 64);
       mbar_init(BAR(kBarGate + s), 128);
       mbar_init(BAR(kBarEmpty + s), 1);
     }
@@ -826,30 +828,25 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       }
     }
   } else if (warp < kWarpGate) {
-    // warps 2-3 have no role
-  } else if (warp < kWarpEpi) {
-    // ------------------------------------------------------------ gates
-    // Gate warp gq owns rows 32gq..32gq+31 of every chunk (its TMEM subpartition).
-    // (A) lane = pair of key channels: exclusive suffix sums of the log-gates over the
-    //     warp's 32 rows in scan order, in place; the quarter totals go to sTot.
-    // (B) after the group barrier: u = local suffix + the totals of the later quarters
-    //     (+ the later chunks of the segment in pass 1); lane = row: K^ = k exp(u) and,
-    //     in pass 2, Q~ = q exp(-u), in place.  A chunk whose |u| exceeds the fp32-safe
-    //     range anywhere is evaluated serially instead (flagged here; the serial path
-    //     reads the raw q and k from global memory).
-    const int gq = warp - kWarpGate;
-    const int pw = a.dk + 4;             // log-gate row pitch in floats
-    const int np = (a.dk + 1) >> 1;      // key-channel pairs
+    // ------------------------------------------------------------ suffix sums
+    // Warp sw walks row quarters 2sw and 2sw+1 of every chunk; lane = pair of key
+    // channels (lanes 0..3 also take pairs 32..35 and beyond).  Per quarter: exclusive
+    // suffix sums of the log-gates over its 32 rows in scan order, in place; the
+    // quarter totals go to sTot.  After the pair barrier each warp turns them into the
+    // offsets of its quarters (totals of the later quarters, + the later chunks of the
+    // segment in pass 1), so that the gate warps add one offset per channel.
+    const int sw = warp - kWarpSuf;
+    const int pw = a.dk + 4;         // log-gate row pitch in floats
+    const int np = (a.dk + 1) >> 1;  // key-channel pairs
     const bool act0 = lane < np, act1 = lane + 32 < np;
     float2 cy0 = make_float2(0.f, 0.f), cy1 = cy0;  // pass 1: later chunks of the segment
-    int ks = 0;   // items through pass 1
-    int kbg = 0;  // non-serial pass-2 jobs masked so far
+    int ks = 0;                                     // items through pass 1
     for (int jc = 0;; ++jc) {
       const int s = jc % S, use = jc / S;
-      if (!group_and(4, 128, wait_bar(BAR(kBarFull + s), (uint32_t)(use & 1), abort_flag))) break;
+      if (!group_and(1, 64, wait_bar(BAR(kBarFull + s), (uint32_t)(use & 1), abort_flag))) break;
       const int kind = sJob[4 * s];
       if (kind == kJobEnd) {
-        mbar_arrive(BAR(kBarGate + s));
+        mbar_arrive(BAR(kBarSufDone + s));
         break;
       }
       const int j = sJob[4 * s + 2], buf = sJob[4 * s + 3];
@@ -857,65 +854,91 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       const bool last1 = pass1 && j == decode_item(a, sJob[4 * s + 1]).n - 1;
       // sGam[buf] is rewritten once the look-back of item ks - nbuf has read it.
       if (last1 && ks >= a.nbuf &&
-          !group_and(4, 128, wait_bar(BAR(kBarSinReady + buf), (uint32_t)(((ks / a.nbuf) - 1) & 1), abort_flag)))
+          !group_and(1, 64, wait_bar(BAR(kBarSinReady + buf), (uint32_t)(((ks / a.nbuf) - 1) & 1), abort_flag)))
         break;
       if (pass1 && j == 0) cy0 = cy1 = make_float2(0.f, 0.f);
-      uint8_t* st = smem + (uint32_t)s * a.stage_bytes;
-      float* lag = reinterpret_cast<float*>(st + a.oLA);
-      // (A) rows of the quarter in decreasing scan position
+      float* lag = reinterpret_cast<float*>(smem + (uint32_t)s * a.stage_bytes + a.oLA);
       {
+        // The two quarters' walks are interleaved (independent chains).
         const int dr = a.g.reverse ? (pw >> 1) : -(pw >> 1);  // in float2
-        float2* p0 = reinterpret_cast<float2*>(lag + (a.g.reverse ? 32 * gq : 32 * gq + 31) * pw) + lane;
-        float2* p1 = p0 + 32;
-        float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
+        float2* pa = reinterpret_cast<float2*>(lag + (a.g.reverse ? 64 * sw : 64 * sw + 31) * pw) + lane;
+        float2* pb = pa + 16 * pw;  // the other quarter: 32 rows on
+        float2 a0 = make_float2(0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
 #pragma unroll 1
         for (int h8 = 0; h8 < 4; ++h8) {
-          float2 x0[8], x1[8];
+          float2 xa[8], xb[8], ya[8], yb[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            x0[q] = act0 ? p0[q * dr] : make_float2(0.f, 0.f);
-            x1[q] = act1 ? p1[q * dr] : make_float2(0.f, 0.f);
+            xa[q] = act0 ? pa[q * dr] : make_float2(0.f, 0.f);
+            xb[q] = act0 ? pb[q * dr] : make_float2(0.f, 0.f);
+            ya[q] = act1 ? pa[q * dr + 32] : make_float2(0.f, 0.f);
+            yb[q] = act1 ? pb[q * dr + 32] : make_float2(0.f, 0.f);
           }
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            if (act0) p0[q * dr] = acc0;
-            if (act1) p1[q * dr] = acc1;
-            acc0.x += x0[q].x;
-            acc0.y += x0[q].y;
-            acc1.x += x1[q].x;
-            acc1.y += x1[q].y;
+            if (act0) {
+              pa[q * dr] = a0;
+              pb[q * dr] = b0;
+            }
+            if (act1) {
+              pa[q * dr + 32] = a1;
+              pb[q * dr + 32] = b1;
+            }
+            a0.x += xa[q].x;
+            a0.y += xa[q].y;
+            b0.x += xb[q].x;
+            b0.y += xb[q].y;
+            a1.x += ya[q].x;
+            a1.y += ya[q].y;
+            b1.x += yb[q].x;
+            b1.y += yb[q].y;
           }
-          p0 += 8 * dr;
-          p1 += 8 * dr;
+          pa += 8 * dr;
+          pb += 8 * dr;
         }
-        float2* tot = reinterpret_cast<float2*>(sTot + gq * 128);
-        tot[lane] = acc0;
-        tot[lane + 32] = acc1;
+        float2* ta = reinterpret_cast<float2*>(sTot + (2 * sw) * 128);
+        float2* tb = reinterpret_cast<float2*>(sTot + (2 * sw + 1) * 128);
+        ta[lane] = a0;
+        ta[lane + 32] = a1;
+        tb[lane] = b0;
+        tb[lane + 32] = b1;
       }
-      named_sync(4, 128);
-      // Offsets of this quarter and the chunk totals, for pairs lane and lane + 32.
+      named_sync(1, 64);
+      // Offsets of this warp's quarters and the chunk totals, for pairs lane and lane + 32.
       {
         const float2* tot = reinterpret_cast<const float2*>(sTot);
-        float2 o0 = pass1 ? cy0 : make_float2(0.f, 0.f), o1 = pass1 ? cy1 : make_float2(0.f, 0.f);
-        float2 c0 = make_float2(0.f, 0.f), c1 = c0;
+        float2 t0[4], t1[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float2 t0 = tot[q * 64 + lane], t1 = tot[q * 64 + lane + 32];
-          c0.x += t0.x;
-          c0.y += t0.y;
-          c1.x += t1.x;
-          c1.y += t1.y;
-          if (a.g.reverse ? q < gq : q > gq) {
-            o0.x += t0.x;
-            o0.y += t0.y;
-            o1.x += t1.x;
-            o1.y += t1.y;
-          }
+          t0[q] = tot[q * 64 + lane];
+          t1[q] = tot[q * 64 + lane + 32];
         }
-        float2* off = reinterpret_cast<float2*>(sOff + gq * 128);
-        off[lane] = o0;
-        off[lane + 32] = o1;
-        if (gq == 0) {
+        const float2 z = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int e2 = 0; e2 < 2; ++e2) {
+          const int qq = 2 * sw + e2;
+          float2 o0 = pass1 ? cy0 : z, o1 = pass1 ? cy1 : z;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (a.g.reverse ? q < qq : q > qq) {
+              o0.x += t0[q].x;
+              o0.y += t0[q].y;
+              o1.x += t1[q].x;
+              o1.y += t1[q].y;
+            }
+          float2* off = reinterpret_cast<float2*>(sOff + (s * 4 + qq) * 128);
+          off[lane] = o0;
+          off[lane + 32] = o1;
+        }
+        float2 c0 = z, c1 = z;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          c0.x += t0[q].x;
+          c0.y += t0[q].y;
+          c1.x += t1[q].x;
+          c1.y += t1[q].y;
+        }
+        if (sw == 0) {
           float2* bl = reinterpret_cast<float2*>(sBL + s * 128);  // chunk gate sums; channels >= dk stay 0
           if (act0) bl[lane] = c0;
           if (act1) bl[lane + 32] = c1;
@@ -925,7 +948,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
           cy0.y += c0.y;
           cy1.x += c1.x;
           cy1.y += c1.y;
-          if (last1 && gq == 0) {
+          if (last1 && sw == 0) {
             // exp(segment gate sum) of growth gates must stay finite
             bool bad = false;
             if (act0) {
@@ -940,17 +963,41 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
             }
             if (bad) report_status(GLA_ERR_RANGE);
           }
+          if (last1) ++ks;
         }
       }
-      __syncwarp();
-      if (last1) ++ks;
-      // (B) lane = row; q, k, v landed
+      // (sTot is rewritten for the next chunk only after the group barrier at its start,
+      // so both warps have read it by then.)
+      mbar_arrive(BAR(kBarSufDone + s));
+    }
+  } else if (warp < kWarpEpi) {
+    // ------------------------------------------------------------ gates
+    // Gate warp gq owns rows 32gq..32gq+31 of every chunk (its TMEM subpartition):
+    // u = the in-place local suffix sum + the offset of its quarter; K^ = k exp(u) and,
+    // in pass 2, Q~ = q exp(-u), in place (lane = row); then the score masking.  A
+    // chunk whose |u| exceeds the fp32-safe range anywhere is evaluated serially instead
+    // (flagged here; the serial path reads the raw q and k from global memory).
+    const int gq = warp - kWarpGate;
+    const int pw = a.dk + 4;  // log-gate row pitch in floats
+    int kbg = 0;              // non-serial pass-2 jobs masked so far
+    for (int jc = 0;; ++jc) {
+      const int s = jc % S, use = jc / S;
+      if (!group_and(4, 128, wait_bar(BAR(kBarSufDone + s), (uint32_t)(use & 1), abort_flag))) break;
+      const int kind = sJob[4 * s];
+      if (kind == kJobEnd) {
+        mbar_arrive(BAR(kBarGate + s));
+        break;
+      }
+      const bool pass1 = kind == kJobP1;
+      uint8_t* st = smem + (uint32_t)s * a.stage_bytes;
+      const float* lag = reinterpret_cast<const float*>(st + a.oLA);
+      // lane = row; q, k, v landed
       if (!group_and(4, 128, wait_bar(BAR(kBarOps + s), (uint32_t)(use & 1), abort_flag))) break;
       float umax = 0.f;  // pass 1: largest u; pass 2: largest |u|
       {
         const int r = 32 * gq + lane;
         const float* urow = lag + r * pw;
-        const float* offq = sOff + gq * 128;
+        const float* offq = sOff + (s * 4 + gq) * 128;
         // exp(u) is rounded to bf16 pairs and applied with packed bf16 multiplies,
         // exp(-u) as its reciprocal.
 #pragma unroll 1
@@ -1250,7 +1297,7 @@ WsLayout ws_layout(const GlaShape& s) {
   // channel blocks from oK; the stage is at least that large.
   L.stage_bytes = al1024(L.oLA + la > 8 * ATOM32 ? L.oLA + la : 8 * ATOM32);
   const uint32_t gtile = al1024((uint32_t)L.Kp * (uint32_t)L.Np * 2u);
-  const uint32_t fixed = gtile + kMaxStages * 512 + 256 + 1536 + 256 + 4096 + 64 + 16 * kMaxStages + 16 + 32 +
+  const uint32_t fixed = gtile + kMaxStages * 512 + 256 + 1536 + 256 + 2048 * (1 + kMaxStages) + 64 + 16 * kMaxStages + 16 + 32 +
                          8 * kNumBars + 16;
   L.nstage = (1024 + 2 * (size_t)L.stage_bytes + fixed <= kMaxSmem) ? 2 : 1;
   L.oG = (uint32_t)L.nstage * L.stage_bytes;
@@ -1260,7 +1307,7 @@ WsLayout ws_layout(const GlaShape& s) {
   L.oRed = L.oGam + 1536;
   L.oTot = L.oRed + 256;
   L.oOff = L.oTot + 2048;
-  L.oMisc = L.oOff + 2048;
+  L.oMisc = L.oOff + 2048 * kMaxStages;
   L.oJob = L.oMisc + 64;
   L.oMail = L.oJob + 16 * kMaxStages;
   L.oItem = L.oMail + 16;
