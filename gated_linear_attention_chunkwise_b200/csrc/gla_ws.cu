@@ -724,23 +724,33 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       bool tail = false;           // Q~ G and K^T V of the last non-serial job still to issue
       int t_s = 0, t_buf = 0, t_kb = 0;
       bool ok = true;
+      // Operand descriptors of stage 0 (stage s: + s * dstage); a K step adds a constant
+      // to the start-address field.  Loops are unrolled to their maximum trip count so
+      // that each MMA costs little more than its issue.
+      const uint64_t dQ = desc_sw32(sbase + a.oQ, 16u, 256u);      // K-major, step ATOM32
+      const uint64_t dK = desc_sw32(sbase + a.oK, 16u, 256u);      // K-major, step ATOM32
+      const uint64_t dKt = desc_sw32(sbase + a.oK, ATOM32, 256u);  // MN-major (K^ transposed), step 512 B
+      const uint64_t dV = desc_sw32(sbase + a.oV, ATOM32, 256u);   // MN-major, step 512 B
+      const uint64_t dG = desc_sw32(sbase + a.oG, (uint32_t)a.Kp * 32u, 256u);
+      const uint64_t dstage = (uint64_t)(a.stage_bytes >> 4);
+      constexpr uint64_t kStepK = ATOM32 >> 4, kStepMN = 512u >> 4;
+      const int nk = a.Kp >> 4;
+      const uint32_t id_s = idesc_bf16_f32(MC, MC, false, false);
+      const uint32_t id_pv = idesc_bf16_f32(MC, a.Np, false, true);
+      const uint32_t id_kv = idesc_bf16_f32(MC, a.Np, true, true);
       auto issue_tail = [&]() -> bool {
         if (!tail) return true;
         tail = false;
         if (!wait_bar(BAR(kBarGReady), (uint32_t)(t_kb & 1), abort_flag)) return false;
         tc_fence_after();
         const int ob = t_kb % a.nO;
-        const uint32_t st = sbase + (uint32_t)t_s * a.stage_bytes;
-        const uint32_t id_pv = idesc_bf16_f32(MC, a.Np, false, true);
-#pragma unroll 1
-        for (int kk = 0; kk < (a.Kp >> 4); ++kk)
-          umma_ss(tbase + a.col_o(ob), desc_sw32(st + a.oQ + (uint32_t)kk * ATOM32, 16u, 256u),
-                  desc_sw32(sbase + a.oG + (uint32_t)kk * 512u, (uint32_t)a.Kp * 32u, 256u), id_pv, 1u);
-        const uint32_t id_s = idesc_bf16_f32(MC, a.Np, true, true);
-#pragma unroll 1
-        for (int kk = 0; kk < MC / 16; ++kk)
-          umma_ss(tbase + a.col_seg(t_buf), desc_sw32(st + a.oK + (uint32_t)kk * 512u, ATOM32, 256u),
-                  desc_sw32(st + a.oV + (uint32_t)kk * 512u, ATOM32, 256u), id_s, 1u);
+        const uint64_t so = (uint64_t)t_s * dstage;
+        const uint32_t tO = tbase + a.col_o(ob), tS = tbase + a.col_seg(t_buf);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          if (kk < nk) umma_ss(tO, dQ + so + kk * kStepK, dG + kk * kStepMN, id_pv, 1u);
+#pragma unroll
+        for (int kk = 0; kk < MC / 16; ++kk) umma_ss(tS, dKt + so + kk * kStepMN, dV + so + kk * kStepMN, id_kv, 1u);
         umma_commit(BAR(kBarBatch + ob));
         umma_commit(BAR(kBarEmpty + t_s));
         return true;
@@ -759,7 +769,6 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
           mbar_arrive(BAR(kBarSegDone + km % a.nbuf));
           break;
         }
-        const uint32_t st = sbase + (uint32_t)s * a.stage_bytes;
         const int n = decode_item(a, item).n;
         if (kind == kJobP1) {
           // The buffer is free once pass 2 of item km - 2 is done with it.
@@ -767,11 +776,11 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
               !wait_bar(BAR(kBarSegFree + buf), (uint32_t)(((km / a.nbuf) - 1) & 1), abort_flag))
             break;
           tc_fence_after();
-          const uint32_t id = idesc_bf16_f32(MC, a.Np, true, true);
-#pragma unroll 1
-          for (int kk = 0; kk < MC / 16; ++kk)
-            umma_ss(tbase + a.col_seg(buf), desc_sw32(st + a.oK + (uint32_t)kk * 512u, ATOM32, 256u),
-                    desc_sw32(st + a.oV + (uint32_t)kk * 512u, ATOM32, 256u), id, (j > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t so = (uint64_t)s * dstage;
+          const uint32_t tS = tbase + a.col_seg(buf);
+          umma_ss(tS, dKt + so, dV + so, id_kv, j > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 1; kk < MC / 16; ++kk) umma_ss(tS, dKt + so + kk * kStepMN, dV + so + kk * kStepMN, id_kv, 1u);
           umma_commit(BAR(kBarEmpty + s));
           if (j == n - 1) {
             umma_commit(BAR(kBarSegDone + buf));
@@ -793,25 +802,23 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
           if (!issue_tail()) break;
           continue;
         }
-        {
-          const uint32_t id = idesc_bf16_f32(MC, MC, false, false);
-#pragma unroll 1
-          for (int kk = 0; kk < (a.Kp >> 4); ++kk)
-            umma_ss(tbase + kColS, desc_sw32(st + a.oQ + (uint32_t)kk * ATOM32, 16u, 256u),
-                    desc_sw32(st + a.oK + (uint32_t)kk * ATOM32, 16u, 256u), id, kk > 0 ? 1u : 0u);
-          umma_commit(BAR(kBarScFull));
-        }
+        const uint64_t so = (uint64_t)s * dstage;
+        umma_ss(tbase + kColS, dQ + so, dK + so, id_s, 0u);
+#pragma unroll
+        for (int kk = 1; kk < 8; ++kk)
+          if (kk < nk) umma_ss(tbase + kColS, dQ + so + kk * kStepK, dK + so + kk * kStepK, id_s, 1u);
+        umma_commit(BAR(kBarScFull));
         if (!issue_tail()) break;
         if (!wait_bar(BAR(kBarPReady), (uint32_t)(kb & 1), abort_flag)) break;
         const int ob = kb % a.nO;
         if (kb >= a.nO && !wait_bar(BAR(kBarOFree + ob), (uint32_t)(((kb / a.nO) - 1) & 1), abort_flag)) break;
         tc_fence_after();
         {
-          const uint32_t id_pv = idesc_bf16_f32(MC, a.Np, false, true);
-#pragma unroll 1
-          for (int kk = 0; kk < MC / 16; ++kk)  // P is bf16 in the score columns
-            umma_ts(tbase + a.col_o(ob), tbase + kColS + (uint32_t)(kk * 8),
-                    desc_sw32(st + a.oV + (uint32_t)kk * 512u, ATOM32, 256u), id_pv, kk > 0 ? 1u : 0u);
+          const uint32_t tO = tbase + a.col_o(ob);
+          umma_ts(tO, tbase + kColS, dV + so, id_pv, 0u);  // P is bf16 in the score columns
+#pragma unroll
+          for (int kk = 1; kk < MC / 16; ++kk)
+            umma_ts(tO, tbase + kColS + (uint32_t)(kk * 8), dV + so + kk * kStepMN, id_pv, 1u);
         }
         tail = true;
         t_s = s;
