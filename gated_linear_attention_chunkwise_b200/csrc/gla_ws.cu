@@ -58,6 +58,8 @@ constexpr int NT = 512;
 constexpr int kWarpProd = 0, kWarpMma = 1, kWarpSuf = 2, kWarpGate = 4, kWarpEpi = 8, kWarpLb = 12;
 constexpr uint32_t ATOM32 = MC * 32u;    // one 16-channel block of a 32B-swizzled 128-row tile
 constexpr float kMaxGateRange = 80.0f;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kMaxGateRange2 = kMaxGateRange * kLog2e;  // the same bound on log2-scaled sums
 constexpr uint32_t kColS = 0;
 constexpr uint32_t kLayoutSW32 = 6;
 constexpr int kMaxStages = 2;
@@ -248,6 +250,13 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// 2^x (hardware approximation); the gate sums are kept in log2 units.
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Lane-wise product of two packed bf16 pairs, rounded to bf16.
 __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t x, uint32_t y) {
   __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&x), *reinterpret_cast<__nv_bfloat162*>(&y));
@@ -839,7 +848,8 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     // Warp sw walks row quarters 2sw and 2sw+1 of every chunk; lane = pair of key
     // channels (lanes 0..3 also take pairs 32..35 and beyond).  Per quarter: exclusive
     // suffix sums of the log-gates over its 32 rows in scan order, in place; the
-    // quarter totals go to sTot.  After the pair barrier each warp turns them into the
+    // quarter totals go to sTot.  All gate sums from here on are in log2 units (times
+    // log2 e).  After the pair barrier each warp turns them into the
     // offsets of its quarters (totals of the later quarters, + the later chunks of the
     // segment in pass 1), so that the gate warps add one offset per channel.
     const int sw = warp - kWarpSuf;
@@ -891,14 +901,14 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
               pa[q * dr + 32] = a1;
               pb[q * dr + 32] = b1;
             }
-            a0.x += xa[q].x;
-            a0.y += xa[q].y;
-            b0.x += xb[q].x;
-            b0.y += xb[q].y;
-            a1.x += ya[q].x;
-            a1.y += ya[q].y;
-            b1.x += yb[q].x;
-            b1.y += yb[q].y;
+            a0.x = fmaf(xa[q].x, kLog2e, a0.x);
+            a0.y = fmaf(xa[q].y, kLog2e, a0.y);
+            b0.x = fmaf(xb[q].x, kLog2e, b0.x);
+            b0.y = fmaf(xb[q].y, kLog2e, b0.y);
+            a1.x = fmaf(ya[q].x, kLog2e, a1.x);
+            a1.y = fmaf(ya[q].y, kLog2e, a1.y);
+            b1.x = fmaf(yb[q].x, kLog2e, b1.x);
+            b1.y = fmaf(yb[q].y, kLog2e, b1.y);
           }
           pa += 8 * dr;
           pb += 8 * dr;
@@ -959,14 +969,14 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
             // exp(segment gate sum) of growth gates must stay finite
             bool bad = false;
             if (act0) {
-              bad |= !(cy0.x <= kMaxGateRange) || !(cy0.y <= kMaxGateRange);
-              sGam[buf * 128 + 2 * lane] = __expf(cy0.x);
-              sGam[buf * 128 + 2 * lane + 1] = __expf(cy0.y);
+              bad |= !(cy0.x <= kMaxGateRange2) || !(cy0.y <= kMaxGateRange2);
+              sGam[buf * 128 + 2 * lane] = exp2_approx(cy0.x);
+              sGam[buf * 128 + 2 * lane + 1] = exp2_approx(cy0.y);
             }
             if (act1) {
-              bad |= !(cy1.x <= kMaxGateRange) || !(cy1.y <= kMaxGateRange);
-              sGam[buf * 128 + 2 * lane + 64] = __expf(cy1.x);
-              sGam[buf * 128 + 2 * lane + 65] = __expf(cy1.y);
+              bad |= !(cy1.x <= kMaxGateRange2) || !(cy1.y <= kMaxGateRange2);
+              sGam[buf * 128 + 2 * lane + 64] = exp2_approx(cy1.x);
+              sGam[buf * 128 + 2 * lane + 65] = exp2_approx(cy1.y);
             }
             if (bad) report_status(GLA_ERR_RANGE);
           }
@@ -1005,8 +1015,8 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         const int r = 32 * gq + lane;
         const float* urow = lag + r * pw;
         const float* offq = sOff + (s * 4 + gq) * 128;
-        // exp(u) is rounded to bf16 pairs and applied with packed bf16 multiplies,
-        // exp(-u) as its reciprocal.
+        // exp(u) = 2^(u log2 e) is rounded to bf16 pairs and applied with packed bf16
+        // multiplies, exp(-u) as its reciprocal.
 #pragma unroll 1
         for (int cc = 0; cc < a.dk; cc += 8) {
           const uint32_t o = sw32_off((uint32_t)r, (uint32_t)cc);
@@ -1025,7 +1035,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
           for (int jj = 0; jj < 4; ++jj) {
             const float a0 = ev[2 * jj], a1 = ev[2 * jj + 1];
             umax = fmaxf(umax, pass1 ? fmaxf(a0, a1) : fmaxf(fabsf(a0), fabsf(a1)));
-            const float p0 = __expf(a0), p1 = __expf(a1);
+            const float p0 = exp2_approx(a0), p1 = exp2_approx(a1);
             uk[jj] = mul_bf16x2(uk[jj], pack_bf16x2(p0, p1));
             if (!pass1) uq[jj] = mul_bf16x2(uq[jj], pack_bf16x2(__fdividef(1.f, p0), __fdividef(1.f, p1)));
           }
@@ -1035,9 +1045,9 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       }
       fence_proxy_async_smem();
       // NaN compares false: a NaN or infinite u also counts as out of range.
-      bool bad = !(umax <= kMaxGateRange);
+      bool bad = !(umax <= kMaxGateRange2);
       if (!pass1 && gq == 0)
-        for (int cc = lane; cc < a.dk; cc += 32) bad |= !(sBL[s * 128 + cc] <= kMaxGateRange);  // exp(chunk sum)
+        for (int cc = lane; cc < a.dk; cc += 32) bad |= !(sBL[s * 128 + cc] <= kMaxGateRange2);  // exp(chunk sum)
       if (pass1) {
         if (bad) report_status(GLA_ERR_RANGE);  // exp(u) of growth gates overflows
         mbar_arrive(BAR(kBarGate + s));
@@ -1167,7 +1177,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         if (!last && !wide) {
           // G = Diag(gamma) S (state -> state, bf16 copy into the G tile)
           {
-            const float gm = __expf(sBL[s * 128 + i]);
+            const float gm = exp2_approx(sBL[s * 128 + i]);  // sums in log2 units
 #pragma unroll 1
             for (int c0 = 0; c0 < a.Np; c0 += 32) {
               uint32_t t[2][16];
