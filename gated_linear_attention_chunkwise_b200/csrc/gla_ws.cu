@@ -1278,7 +1278,7 @@ struct WsLayout {
   size_t flag_bytes, agg_bytes, aggg_bytes;
 };
 
-constexpr int kSegChunks = 4;
+constexpr int kSegChunks = 3;
 constexpr size_t kMaxSmem = 227 * 1024;
 
 uint32_t al1024(uint32_t x) { return (x + 1023u) & ~1023u; }
