@@ -725,13 +725,10 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    // Pass-2 order: S(j) ... P V(j), then S(j+1) when chunk j+1 is already gated, then
-    // Q~ G(j) and K^T V(j), so that the masking of chunk j+1 overlaps the state MMAs of
-    // chunk j.
+    // Pass-2 order per chunk: S, then Q~ G and K^T V (while the gate warps mask S into
+    // P), then P V; the stage is released when P V completes.
     if (lane == 0) {
       int kb = 0, jb = 0, km = 0;  // non-serial pass-2 jobs, pass-2 jobs, items through pass 1
-      bool tail = false;           // Q~ G and K^T V of the last non-serial job still to issue
-      int t_s = 0, t_buf = 0, t_kb = 0;
       bool ok = true;
       // Operand descriptors of stage 0 (stage s: + s * dstage); a K step adds a constant
       // to the start-address field.  Loops are unrolled to their maximum trip count so
@@ -747,51 +744,29 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       const uint32_t id_s = idesc_bf16_f32(MC, MC, false, false);
       const uint32_t id_pv = idesc_bf16_f32(MC, a.Np, false, true);
       const uint32_t id_kv = idesc_bf16_f32(MC, a.Np, true, true);
-      auto issue_tail = [&]() -> bool {
-        if (!tail) return true;
-        tail = false;
-        if (!wait_bar(BAR(kBarGReady), (uint32_t)(t_kb & 1), abort_flag)) return false;
-        tc_fence_after();
-        const int ob = t_kb % a.nO;
-        const uint64_t so = (uint64_t)t_s * dstage;
-        const uint32_t tO = tbase + a.col_o(ob), tS = tbase + a.col_seg(t_buf);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          if (kk < nk) umma_ss(tO, dQ + so + kk * kStepK, dG + kk * kStepMN, id_pv, 1u);
-#pragma unroll
-        for (int kk = 0; kk < MC / 16; ++kk) umma_ss(tS, dKt + so + kk * kStepMN, dV + so + kk * kStepMN, id_kv, 1u);
-        umma_commit(BAR(kBarBatch + ob));
-        umma_commit(BAR(kBarEmpty + t_s));
-        return true;
-      };
       for (int jc = 0; ok; ++jc) {
         const int s = jc % S, use = jc / S;
-        // The deferred MMAs go first unless this job is already gated: its stage may be
-        // waiting for them.
-        if (tail && !mbar_try_wait(BAR(kBarGate + s), (uint32_t)(use & 1)) && !issue_tail()) break;
         if (!wait_bar(BAR(kBarGate + s), (uint32_t)(use & 1), abort_flag)) break;
         tc_fence_after();
         const int kind = sJob[4 * s], item = sJob[4 * s + 1], j = sJob[4 * s + 2], buf = sJob[4 * s + 3];
-        if (kind != kJobP2 && !issue_tail()) break;
         if (kind == kJobEnd) {
           sMisc[5] = km;  // the look-back and output groups stop at item km
           mbar_arrive(BAR(kBarSegDone + km % a.nbuf));
           break;
         }
-        const int n = decode_item(a, item).n;
+        const uint64_t so = (uint64_t)s * dstage;
+        const uint32_t tS = tbase + a.col_seg(buf);
         if (kind == kJobP1) {
           // The buffer is free once pass 2 of item km - 2 is done with it.
           if (j == 0 && km >= a.nbuf &&
               !wait_bar(BAR(kBarSegFree + buf), (uint32_t)(((km / a.nbuf) - 1) & 1), abort_flag))
             break;
           tc_fence_after();
-          const uint64_t so = (uint64_t)s * dstage;
-          const uint32_t tS = tbase + a.col_seg(buf);
           umma_ss(tS, dKt + so, dV + so, id_kv, j > 0 ? 1u : 0u);
 #pragma unroll
           for (int kk = 1; kk < MC / 16; ++kk) umma_ss(tS, dKt + so + kk * kStepMN, dV + so + kk * kStepMN, id_kv, 1u);
           umma_commit(BAR(kBarEmpty + s));
-          if (j == n - 1) {
+          if (j == decode_item(a, item).n - 1) {
             umma_commit(BAR(kBarSegDone + buf));
             ++km;
           }
@@ -807,35 +782,34 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         sMail[3] = j;
         mbar_arrive(BAR(kBarMail));
         ++jb;
-        if (wide) {  // evaluated serially by the output group, which frees the stage
-          if (!issue_tail()) break;
-          continue;
-        }
-        const uint64_t so = (uint64_t)s * dstage;
+        if (wide) continue;  // evaluated serially by the output group, which frees the stage
+        // S = Q~ K^T (masked into P by the gate warps meanwhile)
         umma_ss(tbase + kColS, dQ + so, dK + so, id_s, 0u);
 #pragma unroll
         for (int kk = 1; kk < 8; ++kk)
           if (kk < nk) umma_ss(tbase + kColS, dQ + so + kk * kStepK, dK + so + kk * kStepK, id_s, 1u);
         umma_commit(BAR(kBarScFull));
-        if (!issue_tail()) break;
-        if (!wait_bar(BAR(kBarPReady), (uint32_t)(kb & 1), abort_flag)) break;
+        // O = Q~ G and S += K^T V once the output group has scaled the state into G,
+        // then O += P V: the stage is free when these complete.
         const int ob = kb % a.nO;
+        if (!wait_bar(BAR(kBarGReady), (uint32_t)(kb & 1), abort_flag)) break;
         if (kb >= a.nO && !wait_bar(BAR(kBarOFree + ob), (uint32_t)(((kb / a.nO) - 1) & 1), abort_flag)) break;
         tc_fence_after();
-        {
-          const uint32_t tO = tbase + a.col_o(ob);
-          umma_ts(tO, tbase + kColS, dV + so, id_pv, 0u);  // P is bf16 in the score columns
+        const uint32_t tO = tbase + a.col_o(ob);
+        umma_ss(tO, dQ + so, dG, id_pv, 0u);
 #pragma unroll
-          for (int kk = 1; kk < MC / 16; ++kk)
-            umma_ts(tO, tbase + kColS + (uint32_t)(kk * 8), dV + so + kk * kStepMN, id_pv, 1u);
-        }
-        tail = true;
-        t_s = s;
-        t_buf = buf;
-        t_kb = kb;
+        for (int kk = 1; kk < 8; ++kk)
+          if (kk < nk) umma_ss(tO, dQ + so + kk * kStepK, dG + kk * kStepMN, id_pv, 1u);
+#pragma unroll
+        for (int kk = 0; kk < MC / 16; ++kk) umma_ss(tS, dKt + so + kk * kStepMN, dV + so + kk * kStepMN, id_kv, 1u);
+        if (!wait_bar(BAR(kBarPReady), (uint32_t)(kb & 1), abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < MC / 16; ++kk)  // P is bf16 in the score columns
+          umma_ts(tO, tbase + kColS + (uint32_t)(kk * 8), dV + so + kk * kStepMN, id_pv, 1u);
+        umma_commit(BAR(kBarBatch + ob));
+        umma_commit(BAR(kBarEmpty + s));
         ++kb;
-        // With one stage, or at the end of an item, the next job cannot come first.
-        if ((S == 1 || j == n - 1) && !issue_tail()) break;
       }
       // Every MMA of this CTA completes before TMEM is released (bounded).
       umma_commit(BAR(kBarDrain));
