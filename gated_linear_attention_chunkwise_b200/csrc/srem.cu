@@ -174,8 +174,11 @@ __global__ void __launch_bounds__(kConvThreads) dwconv3x3_k(const __grid_constan
         for (int di = 0; di < 3; ++di)
 #pragma unroll
           for (int dj = 0; dj < 3; ++dj) {
-            acc[oc].x = fmaf(wt[di * 3 + dj].x, win[di][oc + dj].x, acc[oc].x);
-            if (kCh == 2) acc[oc].y = fmaf(wt[di * 3 + dj].y, win[di][oc + dj].y, acc[oc].y);
+            if (kCh == 2) {  // both channels in one packed fp32 FMA (each rounded as fmaf)
+              acc[oc] = __ffma2_rn(wt[di * 3 + dj], win[di][oc + dj], acc[oc]);
+            } else {
+              acc[oc].x = fmaf(wt[di * 3 + dj].x, win[di][oc + dj].x, acc[oc].x);
+            }
           }
       }
       if (r < rows) {
