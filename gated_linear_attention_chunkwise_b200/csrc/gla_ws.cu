@@ -101,6 +101,7 @@ struct WsArgs {
   int* ticket;
   int H, BH, dk, dv, NC, NS, G, items;
   int Kp, Np, nstage, nO, nbuf;
+  int nak, nav;  // full 16-channel atoms of q/k and v loaded by one box each (raster scans; else 0)
   uint32_t colO0, colO1, colSeg0, colSeg1, colSeg2;
   int mode, rpc, ppr;  // chunk geometry: 0 raster, 1 whole columns (rpc per chunk), 2 column pieces (ppr per column)
   uint32_t stage_bytes, oK, oV, oQ, oLA, oG, oBL, oWide, oGam, oRed, oTot, oOff, oMisc, oJob, oMail, oItem, oBar, oTm;
@@ -130,6 +131,9 @@ __device__ __forceinline__ Item decode_item(const WsArgs& a, int item) {
 
 struct TensorMaps {
   CUtensorMap q, k, v, la;  // operand tiles (16-channel boxes, 32-byte swizzle) and log-gate tiles
+  // Raster scans: all full 16-channel atoms of an operand tile in one box (the
+  // channel atoms are a box dimension); the rest, if any, come from q, k, v.
+  CUtensorMap qa, ka, va;
 };
 
 // ---------------------------------------------------------------------------
@@ -349,11 +353,16 @@ __device__ void tma_job(const WsArgs& a, const TensorMaps& tm, uint32_t st, uint
   mbar_expect_tx(bar_la, (uint32_t)MC * (uint32_t)(a.dk + 4) * 4u);
   tma_load_5d(st + a.oLA, &tm.la, 0, h, y, x, b, bar_la, pol);
   mbar_expect_tx(bar_ops, (uint32_t)(with_q ? 2 : 1) * (uint32_t)a.Kp * 256u + (uint32_t)a.Np * 256u);
-  for (int cb = 0; cb < (a.Kp >> 4); ++cb) {
+  if (a.nak) {  // (channel, row, atom, head, batch)
+    tma_load_5d(st + a.oK, &tm.ka, 0, y, 0, h, b, bar_ops, pol);
+    if (with_q) tma_load_5d(st + a.oQ, &tm.qa, 0, y, 0, h, b, bar_ops, pol);
+  }
+  for (int cb = a.nak; cb < (a.Kp >> 4); ++cb) {
     tma_load_5d(st + a.oK + (uint32_t)cb * ATOM32, &tm.k, cb * 16, h, y, x, b, bar_ops, pol);
     if (with_q) tma_load_5d(st + a.oQ + (uint32_t)cb * ATOM32, &tm.q, cb * 16, h, y, x, b, bar_ops, pol);
   }
-  for (int cb = 0; cb < (a.Np >> 4); ++cb)
+  if (a.nav) tma_load_5d(st + a.oV, &tm.va, 0, y, 0, h, b, bar_ops, pol);
+  for (int cb = a.nav; cb < (a.Np >> 4); ++cb)
     tma_load_5d(st + a.oV + (uint32_t)cb * ATOM32, &tm.v, cb * 16, h, y, x, b, bar_ops, pol);
 }
 
@@ -1360,6 +1369,23 @@ bool encode_map(CUtensorMap* m, const void* base, bool f32, int d, int box0, CUt
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Raster 5-D map over a [B][T][H][d] bf16 tensor viewed as (16 channels, token,
+// 16-channel atom, head, batch): a box of (16, 128, natoms, 1, 1) lands as natoms
+// consecutive 32-byte-swizzled atoms of 128 rows.  natoms * 16 <= d keeps every
+// element of the box inside the head's channels.
+bool encode_atoms_map(CUtensorMap* m, const void* base, int d, int natoms, const GlaShape& s) {
+  EncodeTiledFn fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t T = (cuuint64_t)s.T(), H = (cuuint64_t)s.H;
+  const cuuint64_t dims[5] = {16, T, (cuuint64_t)natoms, H, (cuuint64_t)s.B};
+  const cuuint64_t strides[4] = {H * d * 2, 32, (cuuint64_t)d * 2, T * H * d * 2};
+  const cuuint32_t box[5] = {16, (cuuint32_t)MC, (cuuint32_t)natoms, 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 size_t gla_ws_workspace_bytes(const GlaShape& s) {
@@ -1436,6 +1462,14 @@ cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const fl
         encode_map(&tm.v, v, false, s.dv, 16, CU_TENSOR_MAP_SWIZZLE_32B, s, column, box_rows, box_runs) &&
         encode_map(&tm.la, la, true, s.dk, s.dk + 4, CU_TENSOR_MAP_SWIZZLE_NONE, s, column, box_rows, box_runs)))
     return cudaErrorInvalidValue;
+  a.nak = a.nav = 0;
+  if (L.mode == 0) {
+    a.nak = s.dk / 16;
+    a.nav = s.dv / 16;
+    if ((a.nak && !(encode_atoms_map(&tm.qa, q, s.dk, a.nak, s) && encode_atoms_map(&tm.ka, k, s.dk, a.nak, s))) ||
+        (a.nav && !encode_atoms_map(&tm.va, v, s.dv, a.nav, s)))
+      return cudaErrorInvalidValue;
+  }
   cudaError_t e = cudaMemsetAsync(ws, 0, L.flag_bytes, st);  // flags and the ticket counter
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(gla_ws_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
