@@ -22,7 +22,8 @@
 //               pass 2 of the current one); TMA loads of each chunk's q, k, v
 //               (32-byte-swizzled 16-channel boxes, the UMMA operand layout) and
 //               log-gates into a ring of stages;
-//   warp 1      MMA issuer (tcgen05, one thread) and TMEM owner;
+//   warp 1      MMA issuer (tcgen05, one thread) and TMEM owner; per pass-2 chunk
+//               S = Q~ K^T, then Q~ G and K^T V, then P V;
 //   warps 2-3   suffix sums of the log-gates, two row quarters per warp in parallel
 //               (lane = pair of key channels), and each quarter's offset;
 //   warps 4-7   gate group, warp = quarter of the chunk's rows: the gates applied in
@@ -37,10 +38,12 @@
 //
 // Chunks follow the direction's base order (raster rows, or grid columns for T->B /
 // B->T) and are always cut in forward order; reversed scans visit them backwards and
-// walk each chunk's rows backwards.  Each chunk is one TMA box per tensor: 128
+// walk each chunk's rows backwards.  A chunk is: 128
 // consecutive raster positions; 128/Hgrid whole columns when Hgrid divides 128;
 // otherwise one column cut into pieces of at most 128 rows.  Rows past the grid are
-// zero-filled by the TMA and contribute nothing.
+// zero-filled by the TMA and contribute nothing.  The operand tiles arrive as 16-channel
+// 32-byte-swizzled atoms; raster scans load all full atoms of a tile with one box.
+// All gate sums are kept in log2 units (times log2 e), so a gate is one ex2.
 #include <math.h>
 #include <string.h>
 
