@@ -361,12 +361,34 @@ def run_gpu(args):
                                        "srem_reorient": statistics.mean(reor_ms) * 1e3},
             "gla_only": {"tokens_heads_per_s": w.token_heads / gla_avg_s,
                          "tflops": GLA_FLOP_PER_TOKEN_HEAD * w.token_heads / gla_avg_s / 1e12},
+            "per_kernel": per_kernel(w, gla_ms, conv_ms, reor_ms, hbm),
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def per_kernel(w, gla_ms, conv_ms, reor_ms, hbm):
+    """Achieved algorithmic GB/s (and TFLOP/s for the GLA) of each op of a layer and of
+    the layer as a whole, from the event-timed means, with the fraction of the HBM peak."""
+    grid_bytes = 2 * w.B * w.T * w.C * 2  # bf16 in + out, dwconv and reorient alike
+    rows = {"gla_fwd": (statistics.mean(gla_ms), GLA_BYTES_PER_TOKEN_HEAD * w.token_heads,
+                        GLA_FLOP_PER_TOKEN_HEAD * w.token_heads),
+            "dwconv3x3": (statistics.mean(conv_ms), grid_bytes, 18 * w.B * w.T * w.C),
+            "srem_reorient": (statistics.mean(reor_ms), grid_bytes, 0)}
+    out = {}
+    tot_ms = tot_b = 0.0
+    for name, (ms, nbytes, flops) in rows.items():
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[name] = {"us": ms * 1e3, "bytes": nbytes, "GB_per_s": gbs, "frac_of_hbm": gbs / hbm,
+                     "TFLOP_per_s": flops / (ms / 1e3) / 1e12}
+        tot_ms += ms
+        tot_b += nbytes
+    out["layer"] = {"us": tot_ms * 1e3, "bytes": tot_b, "GB_per_s": tot_b / (tot_ms / 1e3) / 1e9,
+                    "frac_of_hbm": tot_b / (tot_ms / 1e3) / 1e9 / hbm}
+    return out
 
 
 def main():
