@@ -83,10 +83,41 @@ int validate_grid(const void* x, const void* y, int B, int Hg, int Wg, int C, in
   return GLA_OK;
 }
 
+// Per-device memory pool for the GLA scratch: stream-ordered like the default pool, but
+// it keeps its memory across stream synchronisations (the default pool returns it at
+// every synchronisation, so the next call would map it again on the host).
+// dig_gla_release() trims it.
+cudaMemPool_t g_pool[64];
+
+cudaMemPool_t workspace_pool(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props;
+    memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t p = nullptr;
+    if (cudaMemPoolCreate(&p, &props) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    uint64_t keep = UINT64_MAX;
+    cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+    g_pool[dev] = p;
+  }
+  return g_pool[dev];
+}
+
 int run_with_workspace(size_t bytes, cudaStream_t st, cudaError_t (*fn)(void*, void*), void* ctx) {
   void* ws = nullptr;
   if (bytes) {
-    if (cudaMallocAsync(&ws, bytes, st) != cudaSuccess) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GLA_ERR_CUDA;
+    cudaMemPool_t pool = workspace_pool(dev);
+    const cudaError_t e = pool ? cudaMallocFromPoolAsync(&ws, bytes, pool, st) : cudaMallocAsync(&ws, bytes, st);
+    if (e != cudaSuccess) {
       cudaGetLastError();
       return GLA_ERR_NOMEM;
     }
@@ -213,6 +244,8 @@ const char* dig_gla_status_string(int status) {
 void dig_gla_release(void) {
   std::lock_guard<std::mutex> lk(dig::g_mu);
   memset(dig::g_arch_ok, 0, sizeof(dig::g_arch_ok));
+  for (cudaMemPool_t p : dig::g_pool)
+    if (p) cudaMemPoolTrimTo(p, 0);  // memory of allocations still in flight stays
 }
 
 }  // extern "C"

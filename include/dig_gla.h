@@ -78,7 +78,8 @@ enum { GLA_BF16 = 0, GLA_F32 = 1 };
  * the chunk are evaluated token by token (exact, slower).  Growth gates
  * (log_alpha > 0) whose product exceeds e^80 inside a chunk cannot be represented
  * in fp32: GLA_ERR_RANGE is recorded in the device status.
- * Workspace: stream-ordered (cudaMallocAsync), freed on the same stream.
+ * Workspace: stream-ordered, from a per-device pool of the library (cudaMallocFromPoolAsync;
+ * the pool keeps its memory across synchronisations), freed on the same stream.
  * `out` must not overlap any input.
  */
 int gla_fwd(const void* q, const void* k, const void* v, const float* log_alpha, int B, int H, int Hgrid,
@@ -160,7 +161,13 @@ int dig_gla_device_status(cudaStream_t stream);
 /* Human-readable name of a gla_status_t value (static storage). */
 const char* dig_gla_status_string(int status);
 
-/* Releases cached host-side state (nothing is cached on the device). */
+/*
+ * dig_gla_release -- forgets cached host-side state and returns the library's
+ * unused GLA scratch memory to the device.  The scratch comes from a per-device
+ * stream-ordered memory pool that keeps its memory across stream synchronisations
+ * (so repeated calls do not map it again); scratch of calls still in flight stays
+ * allocated until they complete.
+ */
 void dig_gla_release(void);
 
 #ifdef __cplusplus
