@@ -328,6 +328,7 @@ def run_gpu(args):
 
     peaks, peak_kind = measured_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    extra = other_configs(dig, dev, stream, hbm) if (rank == 0 and not args.no_other_configs) else None
     gla_avg_s = statistics.mean(gla_ms) / 1e3
     gla_bytes = GLA_BYTES_PER_TOKEN_HEAD * w.token_heads
     achieved = gla_bytes / gla_avg_s / 1e9
@@ -362,12 +363,48 @@ def run_gpu(args):
             "gla_only": {"tokens_heads_per_s": w.token_heads / gla_avg_s,
                          "tflops": GLA_FLOP_PER_TOKEN_HEAD * w.token_heads / gla_avg_s / 1e12},
             "per_kernel": per_kernel(w, gla_ms, conv_ms, reor_ms, hbm),
+            "other_configs_gla_fwd": extra,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def other_configs(dig, dev, stream, hbm, reps=10):
+    """GLA forward alone on the other bf16 configurations (median of `reps` calls per
+    scan direction, event-timed, inputs resident in HBM; c2 and c3 fit in L2, so their
+    numbers are L2-warm), with the fraction of the HBM roofline on their algorithmic
+    bytes.  Supplementary to the headline line."""
+    res = {}
+    for name in ("c2", "c3", "c5"):
+        cw = workloads.WORKLOADS[name]
+        q, k, v, la = [t.to(dev) for t in workloads.gla_inputs(cw, seed=7)]
+        out = torch.empty((cw.B, cw.T, cw.H, cw.dv), dtype=torch.bfloat16, device=dev)
+        nbytes = (2 * (2 * cw.dk + cw.dv) + 4 * cw.dk + 2 * cw.dv) * cw.token_heads
+        per_dir = []
+        for d in range(4):
+            for _ in range(3):
+                dig.gla_fwd(q, k, v, la, cw.Hgrid, cw.Wgrid, d, out=out)
+            ts = []
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                dig.gla_fwd(q, k, v, la, cw.Hgrid, cw.Wgrid, d, out=out)
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                ts.append(e0.elapsed_time(e1) * 1e3)
+            per_dir.append(statistics.median(ts))
+        us = statistics.mean(per_dir)
+        res[name] = {"workload": cw.name, "us_per_dir": per_dir, "bytes": nbytes,
+                     "tokens_heads_per_s": cw.token_heads / (us / 1e6),
+                     "frac_of_hbm": nbytes / (us / 1e6) / 1e9 / hbm}
+        del q, k, v, la, out
+    status = dig.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after the other configurations: {dig.status_string(status)}")
+    return res
 
 
 def per_kernel(w, gla_ms, conv_ms, reor_ms, hbm):
@@ -400,6 +437,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the supplementary GLA timings on the c2, c3 and c5 shapes")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
