@@ -1086,8 +1086,10 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     }
   } else if (warp < kWarpLb) {
     // ------------------------------------------------------------ output group (pass 2)
-    // Per non-serial chunk j: mask S(j) into P(j); epilogue of chunk j-1 (its MMAs also
-    // finished the state update); G = Diag(gamma_j) S; then the MMAs of chunk j run.
+    // Per chunk j (its scores are masked by the gate warps): once the MMAs of chunk j-1
+    // have completed (O(j-1) written, state updated), G = Diag(gamma_j) S for chunk j's
+    // Q~ G and K^T V; then the epilogue of chunk j-1 while chunk j's MMAs run.  A
+    // chunk flagged serial is evaluated here token by token instead.
     const int i = 32 * (warp & 3) + lane;  // TMEM lane = row / key channel
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     const int e = tid - 32 * kWarpEpi;
@@ -1189,6 +1191,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
             }
             tmem_st_wait();
           }
+          fence_proxy_async_smem();  // the G tile is read by the tensor core
           tc_fence_before();
           mbar_arrive(BAR(kBarGReady));
         }
