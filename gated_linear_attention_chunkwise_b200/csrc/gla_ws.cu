@@ -484,10 +484,12 @@ __device__ __forceinline__ float fold_state(const WsArgs& a, const float* src, i
 // return.  Steps: publish the aggregate and exp(segment gate sum) (flag 1); fold
 // earlier segments of the same head, nearest first, into the incoming state until an
 // inclusive state is found (decoupled look-back); publish this segment's inclusive
-// state Diag(gamma_seg) S_in + aggregate (flag 2).  Predecessor flags are read 32 at a
-// time by one warp; sLb is a small shared scratch.
+// state Diag(gamma_seg) S_in + aggregate (flag 2), handing S_in to pass 2 (sin_item,
+// bar_sin) just before that flag's fence.  Predecessor flags are read 32 at a time by
+// one warp; sLb is a small shared scratch.
 __device__ __forceinline__ void lookback(const WsArgs& a, int seg, int bh, int64_t seg_id, uint32_t tSeg, int i, int e,
-                                         float gs, volatile int* sLb) {
+                                         float gs, volatile int* sLb, uint32_t bar_sin, volatile int* sin_item,
+                                         int item) {
   const int DQ = a.dv >> 2;
   const int lane = e & 31;
   if (i < a.dk) a.agg_g[seg_id * a.dk + i] = gs;
@@ -514,7 +516,9 @@ __device__ __forceinline__ void lookback(const WsArgs& a, int seg, int bh, int64
   }
   tmem_st_wait();
   named_sync(3, 128);
-  if (e == 0) {
+  // The flag is released by a thread of the last warp: the first warp scans the
+  // predecessors' flags meanwhile, without waiting for this fence.
+  if (e == 127) {
     __threadfence();
     st_release(a.flags + seg_id, 1);
   }
@@ -592,6 +596,9 @@ __device__ __forceinline__ void lookback(const WsArgs& a, int seg, int bh, int64
   tc_fence_before();
   named_sync(3, 128);
   if (e == 0) {
+    // TMEM is no longer read here: pass 2 may take the incoming state now.
+    *sin_item = item;
+    mbar_arrive(bar_sin);
     __threadfence();
     st_release(a.flags + seg_id, 2);
   }
@@ -1231,11 +1238,8 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       tc_fence_after();
       const int item = sItem[buf];
       const Item it = decode_item(a, item);
-      lookback(a, it.seg, it.bh, it.seg_id, tbase + a.col_seg(buf) + lane_base, i, e, sGam[buf * 128 + i], sMisc + 2);
-      if (e == 0) {
-        sItem[3 + buf] = item;
-        mbar_arrive(BAR(kBarSinReady + buf));
-      }
+      lookback(a, it.seg, it.bh, it.seg_id, tbase + a.col_seg(buf) + lane_base, i, e, sGam[buf * 128 + i], sMisc + 2,
+               BAR(kBarSinReady + buf), sItem + 3 + buf, item);
     }
   }
 
