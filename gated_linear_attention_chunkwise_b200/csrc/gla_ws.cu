@@ -34,7 +34,9 @@
 // TMEM (512 columns): scores [0,128) -- overwritten by the bf16 P matrix (two keys per
 // column, the A operand of P V) --, O (two buffers when dv <= 96), and two buffers
 // that each hold an item's segment aggregate, then its incoming state, then its
-// running state.  A stage is free once the MMAs that read it complete.
+// running state.  A stage is released in two parts: its log-gate, q and k tiles once
+// the K^T V MMAs complete (the next job's loads into them start while P V still runs),
+// its v tile once P V completes.
 //
 // Chunks follow the direction's base order (raster rows, or grid columns for T->B /
 // B->T) and are always cut in forward order; reversed scans visit them backwards and
@@ -70,11 +72,13 @@ constexpr int kMaxStages = 2;
 // mbarrier indices (8 bytes each)
 enum {
   kBarFull = 0,                       // [S]  log-gate tile landed (or an end-of-stream job posted)
-  kBarOps = kBarFull + kMaxStages,    // [S]  q, k, v tiles landed
-  kBarSufDone = kBarOps + kMaxStages, // [S]  suffix sums and quarter offsets done (64 arrivals)
+  kBarOps = kBarFull + kMaxStages,    // [S]  q, k tiles landed
+  kBarOpsV = kBarOps + kMaxStages,    // [S]  v tile landed
+  kBarSufDone = kBarOpsV + kMaxStages, // [S]  suffix sums and quarter offsets done (64 arrivals)
   kBarGate = kBarSufDone + kMaxStages,  // [S]  gates applied (128 arrivals)
-  kBarEmpty = kBarGate + kMaxStages,  // [S]  stage free (MMA commit, or the serial path)
-  kBarMail = kBarEmpty + kMaxStages,  // pass-2 job handed to the output group
+  kBarEmpty = kBarGate + kMaxStages,  // [S]  log-gate, q, k tiles free (MMA commit, or the serial path)
+  kBarEmptyV = kBarEmpty + kMaxStages, // [S] v tile free
+  kBarMail = kBarEmptyV + kMaxStages, // pass-2 job handed to the output group
   kBarScFull,                         // score MMA done
   kBarScEmpty,                        // pass-2 job taken by the output group (128 arrivals)
   kBarPReady,                         // P written by the gate warps (128 arrivals)
@@ -355,7 +359,7 @@ __device__ void tma_job(const WsArgs& a, const TensorMaps& tm, uint32_t st, uint
   const uint64_t pol = with_q ? l2_policy_evict_first() : l2_policy_evict_normal();
   mbar_expect_tx(bar_la, (uint32_t)MC * (uint32_t)(a.dk + 4) * 4u);
   tma_load_5d(st + a.oLA, &tm.la, 0, h, y, x, b, bar_la, pol);
-  mbar_expect_tx(bar_ops, (uint32_t)(with_q ? 2 : 1) * (uint32_t)a.Kp * 256u + (uint32_t)a.Np * 256u);
+  mbar_expect_tx(bar_ops, (uint32_t)(with_q ? 2 : 1) * (uint32_t)a.Kp * 256u);
   if (a.nak) {  // (channel, row, atom, head, batch)
     tma_load_5d(st + a.oK, &tm.ka, 0, y, 0, h, b, bar_ops, pol);
     if (with_q) tma_load_5d(st + a.oQ, &tm.qa, 0, y, 0, h, b, bar_ops, pol);
@@ -364,9 +368,17 @@ __device__ void tma_job(const WsArgs& a, const TensorMaps& tm, uint32_t st, uint
     tma_load_5d(st + a.oK + (uint32_t)cb * ATOM32, &tm.k, cb * 16, h, y, x, b, bar_ops, pol);
     if (with_q) tma_load_5d(st + a.oQ + (uint32_t)cb * ATOM32, &tm.q, cb * 16, h, y, x, b, bar_ops, pol);
   }
-  if (a.nav) tma_load_5d(st + a.oV, &tm.va, 0, y, 0, h, b, bar_ops, pol);
+}
+// The chunk's v tile (its own barrier: the v part of a stage is released last).
+__device__ void tma_job_v(const WsArgs& a, const TensorMaps& tm, uint32_t st, uint32_t bar_v, int cf, bool pass2,
+                          int b, int h) {
+  int y, x;
+  chunk_box(a, cf, y, x);
+  const uint64_t pol = pass2 ? l2_policy_evict_first() : l2_policy_evict_normal();
+  mbar_expect_tx(bar_v, (uint32_t)a.Np * 256u);
+  if (a.nav) tma_load_5d(st + a.oV, &tm.va, 0, y, 0, h, b, bar_v, pol);
   for (int cb = a.nav; cb < (a.Np >> 4); ++cb)
-    tma_load_5d(st + a.oV + (uint32_t)cb * ATOM32, &tm.v, cb * 16, h, y, x, b, bar_ops, pol);
+    tma_load_5d(st + a.oV + (uint32_t)cb * ATOM32, &tm.v, cb * 16, h, y, x, b, bar_v, pol);
 }
 
 // ---------------------------------------------------------------------------
@@ -627,7 +639,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
   float* red = reinterpret_cast<float*>(smem + a.oRed);     // serial-path reduction [4][16]
   float* sTot = reinterpret_cast<float*>(smem + a.oTot);    // [4][128] log-gate sums of the row quarters
   float* sOff = reinterpret_cast<float*>(smem + a.oOff);    // [S][4][128] log-gate sums after each quarter
-  // [0] first item [1] abort [2] look-back flag [3] jobs posted [5] end item index
+  // [0] first item [1] abort [3] jobs posted [5] end item index [6..7] look-back scan result
   volatile int* sMisc = reinterpret_cast<volatile int*>(smem + a.oMisc);
   volatile int* sJob = reinterpret_cast<volatile int*>(smem + a.oJob);    // [S][4] kind, item, j, buf
   volatile int* sMail = reinterpret_cast<volatile int*>(smem + a.oMail);  // [4]    stage, wide, item, j
@@ -644,6 +656,8 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     for (int s = 0; s < a.nstage; ++s) {
       mbar_init(BAR(kBarFull + s), 1);
       mbar_init(BAR(kBarOps + s), 1);
+      mbar_init(BAR(kBarOpsV + s), 1);
+      mbar_init(BAR(kBarEmptyV + s), 1);
       mbar_init(BAR(kBarSufDone + s), 64);
       mbar_init(BAR(kBarGate + s), 128);
       mbar_init(BAR(kBarEmpty + s), 1);
@@ -667,6 +681,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     sMisc[0] = atomicAdd(a.ticket, 1);
     sMisc[1] = 0;
     sMisc[3] = 0;
+    sMisc[4] = 0;
     sMisc[5] = 0x7fffffff;
   }
   for (int x = tid; x < kMaxStages * 128; x += NT) sBL[x] = 0.f;  // rows >= dk: gamma = 1
@@ -683,6 +698,11 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
   } else if (warp == kWarpProd) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // Warm the TMA descriptor cache with every tensor map this kernel loads through.
+      const CUtensorMap* maps[7] = {&tm.la, &tm.k, &tm.q, &tm.v, &tm.ka, &tm.qa, &tm.va};
+#pragma unroll
+      for (int m = 0; m < 7; ++m)
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(maps[m])) : "memory");
       int jc = 0;
       auto post = [&](int kind, int item, int j, int buf) -> bool {
         const int s = jc % S, use = jc / S;
@@ -694,13 +714,19 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         if (kind == kJobEnd) {
           mbar_arrive(BAR(kBarFull + s));
           mbar_arrive(BAR(kBarOps + s));
+          mbar_arrive(BAR(kBarOpsV + s));
+          sMisc[3] = jc + 1;
         } else {
           const Item it = decode_item(a, item);
           const int c = kind == kJobP1 ? it.c0 + it.n - 1 - j : it.c0 + j;  // pass 1 walks backwards
           tma_job(a, tm, sbase + (uint32_t)s * a.stage_bytes, BAR(kBarFull + s), BAR(kBarOps + s), fwd_chunk(a, c),
                   kind == kJobP2, it.b, it.h);
+          sMisc[3] = jc + 1;  // log-gate, q, k loads of this job issued
+          if (use > 0 && !wait_bar(BAR(kBarEmptyV + s), (uint32_t)((use - 1) & 1), abort_flag)) return false;
+          tma_job_v(a, tm, sbase + (uint32_t)s * a.stage_bytes, BAR(kBarOpsV + s), fwd_chunk(a, c), kind == kJobP2,
+                    it.b, it.h);
         }
-        sMisc[3] = ++jc;
+        sMisc[4] = ++jc;  // v load issued too
         return true;
       };
       auto post_p1 = [&](int item, int k) -> bool {
@@ -745,7 +771,8 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     // Pass-2 order per chunk: S, then Q~ G and K^T V (while the gate warps mask S into
-    // P), then P V; the stage is released when P V completes.
+    // P), then P V; the stage's q/k/log-gate part is released after K^T V, its v part
+    // after P V.
     if (lane == 0) {
       int kb = 0, jb = 0, km = 0;  // non-serial pass-2 jobs, pass-2 jobs, items through pass 1
       bool ok = true;
@@ -780,11 +807,13 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
           if (j == 0 && km >= a.nbuf &&
               !wait_bar(BAR(kBarSegFree + buf), (uint32_t)(((km / a.nbuf) - 1) & 1), abort_flag))
             break;
+          if (!wait_bar(BAR(kBarOpsV + s), (uint32_t)(use & 1), abort_flag)) break;
           tc_fence_after();
           umma_ss(tS, dKt + so, dV + so, id_kv, j > 0 ? 1u : 0u);
 #pragma unroll
           for (int kk = 1; kk < MC / 16; ++kk) umma_ss(tS, dKt + so + kk * kStepMN, dV + so + kk * kStepMN, id_kv, 1u);
           umma_commit(BAR(kBarEmpty + s));
+          umma_commit(BAR(kBarEmptyV + s));
           if (j == decode_item(a, item).n - 1) {
             umma_commit(BAR(kBarSegDone + buf));
             ++km;
@@ -796,7 +825,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         tc_fence_after();
         const int wide = sWide[s];
         sMail[0] = s;
-        sMail[1] = wide;
+        sMail[1] = wide | ((use & 1) << 1);  // + the stage use's parity (v barrier)
         sMail[2] = item;
         sMail[3] = j;
         mbar_arrive(BAR(kBarMail));
@@ -820,14 +849,17 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         for (int kk = 1; kk < 8; ++kk)
           if (kk < nk) umma_ss(tO, dQ + so + kk * kStepK, dG + kk * kStepMN, id_pv, 1u);
 #pragma unroll
+        if (!wait_bar(BAR(kBarOpsV + s), (uint32_t)(use & 1), abort_flag)) break;
+        tc_fence_after();
         for (int kk = 0; kk < MC / 16; ++kk) umma_ss(tS, dKt + so + kk * kStepMN, dV + so + kk * kStepMN, id_kv, 1u);
+        umma_commit(BAR(kBarEmpty + s));  // q, k and the log-gate tile are no longer read
         if (!wait_bar(BAR(kBarPReady), (uint32_t)(kb & 1), abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < MC / 16; ++kk)  // P is bf16 in the score columns
           umma_ts(tO, tbase + kColS + (uint32_t)(kk * 8), dV + so + kk * kStepMN, id_pv, 1u);
         umma_commit(BAR(kBarBatch + ob));
-        umma_commit(BAR(kBarEmpty + s));
+        umma_commit(BAR(kBarEmptyV + s));
         ++kb;
       }
       // Every MMA of this CTA completes before TMEM is released (bounded).
@@ -1152,13 +1184,15 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         const bool last = j == it.n;
         bool wide = false;
         int s = 0, cf = 0;
+        uint32_t vpar = 0;
         if (!last) {
           if (!group_and(2, 128, wait_bar(BAR(kBarMail), (uint32_t)(jb & 1), abort_flag))) {
             ok = false;
             break;
           }
           s = sMail[0];
-          wide = sMail[1] != 0;
+          wide = (sMail[1] & 1) != 0;
+          vpar = (uint32_t)((sMail[1] >> 1) & 1);
           ++jb;
           cf = fwd_chunk(a, it.c0 + j);
           mbar_arrive(BAR(kBarScEmpty));  // the job is taken (the gate warps mask its scores)
@@ -1207,10 +1241,17 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         pending = false;
         if (last) break;
         if (wide) {
+          if (!group_and(2, 128, wait_bar(BAR(kBarOpsV + s), vpar, abort_flag))) {
+            ok = false;
+            break;
+          }
           chunk_serial(a, st, red, tbase + a.col_seg(buf), lane_base, i, cf, it.b, it.h);
           tc_fence_before();
           named_sync(2, 128);
-          if (e == 0) mbar_arrive(BAR(kBarEmpty + s));
+          if (e == 0) {
+            mbar_arrive(BAR(kBarEmpty + s));
+            mbar_arrive(BAR(kBarEmptyV + s));
+          }
           continue;
         }
         pending = true;
@@ -1238,7 +1279,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       tc_fence_after();
       const int item = sItem[buf];
       const Item it = decode_item(a, item);
-      lookback(a, it.seg, it.bh, it.seg_id, tbase + a.col_seg(buf) + lane_base, i, e, sGam[buf * 128 + i], sMisc + 2,
+      lookback(a, it.seg, it.bh, it.seg_id, tbase + a.col_seg(buf) + lane_base, i, e, sGam[buf * 128 + i], sMisc + 6,
                BAR(kBarSinReady + buf), sItem + 3 + buf, item);
     }
   }
@@ -1248,11 +1289,12 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
   if (*abort_flag && tid == 0) {
     // Let loads still in flight land before the shared memory is released: only the
     // last S posted jobs can still have any (earlier stages were reposted).
-    for (int jj = max(sMisc[3] - S, 0); jj < sMisc[3]; ++jj) {
-      for (int bb = 0; bb < 2; ++bb) {
+    for (int bb = 0; bb < 3; ++bb) {
+      const int posted = bb == 2 ? sMisc[4] : sMisc[3];
+      const int bar = bb == 0 ? kBarFull : (bb == 1 ? kBarOps : kBarOpsV);
+      for (int jj = max(posted - S, 0); jj < posted; ++jj) {
         const long long t0 = clock64();
-        while (!mbar_try_wait(BAR((bb ? kBarOps : kBarFull) + jj % S), (uint32_t)((jj / S) & 1)) &&
-               clock64() - t0 < kWaitCycles) {
+        while (!mbar_try_wait(BAR(bar + jj % S), (uint32_t)((jj / S) & 1)) && clock64() - t0 < kWaitCycles) {
         }
       }
     }
