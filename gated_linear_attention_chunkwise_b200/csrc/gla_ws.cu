@@ -286,9 +286,9 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(bar), "l"(policy)
       : "memory");
 }
-__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
@@ -354,9 +354,9 @@ __device__ void tma_job(const WsArgs& a, const TensorMaps& tm, uint32_t st, uint
                         bool with_q, int b, int h) {
   int y, x;
   chunk_box(a, cf, y, x);
-  // Pass 2 is the last use of every tile: mark its lines first to go, so that the
-  // pass-1 tiles waiting for their second read stay in L2.
-  const uint64_t pol = with_q ? l2_policy_evict_first() : l2_policy_evict_normal();
+  // Pass 1 marks its tiles' lines evict-last: pass 2 reads them again about one item
+  // later.  Pass 2 is the last use of every tile and marks its lines first to go.
+  const uint64_t pol = with_q ? l2_policy_evict_first() : l2_policy_evict_last();
   mbar_expect_tx(bar_la, (uint32_t)MC * (uint32_t)(a.dk + 4) * 4u);
   tma_load_5d(st + a.oLA, &tm.la, 0, h, y, x, b, bar_la, pol);
   mbar_expect_tx(bar_ops, (uint32_t)(with_q ? 2 : 1) * (uint32_t)a.Kp * 256u);
@@ -374,7 +374,7 @@ __device__ void tma_job_v(const WsArgs& a, const TensorMaps& tm, uint32_t st, ui
                           int b, int h) {
   int y, x;
   chunk_box(a, cf, y, x);
-  const uint64_t pol = pass2 ? l2_policy_evict_first() : l2_policy_evict_normal();
+  const uint64_t pol = pass2 ? l2_policy_evict_first() : l2_policy_evict_last();
   mbar_expect_tx(bar_v, (uint32_t)a.Np * 256u);
   if (a.nav) tma_load_5d(st + a.oV, &tm.va, 0, y, 0, h, b, bar_v, pol);
   for (int cb = a.nav; cb < (a.Np >> 4); ++cb)
