@@ -5,7 +5,7 @@ caller's current CUDA stream and forwards raw device pointers to the C ABI of
 `libdig_gla.so` (declared in include/dig_gla.h).  All computation happens in
 the library's sm_100a kernels; there is no CPU or PyTorch fallback, and
 importing this package fails if the library has not been built
-(`python -m gated_linear_attention_chunkwise_b200.build`).
+(`python gated_linear_attention_chunkwise_b200/build.py`).
 
 Names follow the C ABI: gla_fwd, gla_fwd_f32, srem_reorient, dwconv3x3,
 device_status (dig_gla_device_status), status_string (dig_gla_status_string).
@@ -22,7 +22,7 @@ __all__ = ["gla_fwd", "gla_fwd_f32", "srem_reorient", "dwconv3x3", "device_statu
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdig_gla.so")
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m gated_linear_attention_chunkwise_b200.build`"
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python gated_linear_attention_chunkwise_b200/build.py`"
                       " (nvcc, sm_100a). There is no fallback implementation.")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -36,6 +36,8 @@ _lib.dig_gla_status_string.argtypes = [_i]
 _lib.dig_gla_status_string.restype = ctypes.c_char_p
 _lib.dig_gla_release.argtypes = []
 _lib.dig_gla_release.restype = None
+_lib.dig_gla_test_skip_items.argtypes = [_i]
+_lib.dig_gla_test_skip_items.restype = None
 for _fn in (_lib.gla_fwd, _lib.gla_fwd_f32, _lib.srem_reorient, _lib.dwconv3x3, _lib.dig_gla_device_status):
     _fn.restype = ctypes.c_int
 
@@ -162,6 +164,13 @@ def dwconv3x3(x, w, out=None, stream=None):
                             _stream_handle(x.device, stream))
     _check("dwconv3x3", rc)
     return out
+
+
+def skip_items_for_test(n: int) -> None:
+    """Test hook: the next gla_fwd call leaves out its first n work items, so the
+    look-back waits that need them run out (device status GLA_ERR_TIMEOUT afterwards,
+    output unspecified).  n <= 0 clears it."""
+    _lib.dig_gla_test_skip_items(int(n))
 
 
 def device_status(stream=None, device=None) -> int:

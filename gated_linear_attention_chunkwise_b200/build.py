@@ -1,6 +1,8 @@
 """Builds the in-tree CUDA library libdig_gla.so for sm_100a with nvcc.
 
-    python -m gated_linear_attention_chunkwise_b200.build [--force] [--verbose]
+    python gated_linear_attention_chunkwise_b200/build.py [--force] [--verbose]
+
+(run by path: importing the package loads the library, which may not exist yet).
 
 The library is placed next to this file so that it travels with the source tree.
 """

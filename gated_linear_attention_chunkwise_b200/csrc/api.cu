@@ -8,6 +8,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "dev_common.cuh"
@@ -154,6 +155,9 @@ cudaError_t read_and_clear_device_status(int* status, cudaStream_t st) {
   return cudaSuccess;
 }
 
+std::atomic<int> g_test_skip{0};
+int take_test_skip_items() { return g_test_skip.exchange(0); }
+
 }  // namespace dig
 
 using dig::GlaShape;
@@ -240,6 +244,8 @@ const char* dig_gla_status_string(int status) {
     default: return "GLA_ERR_UNKNOWN";
   }
 }
+
+void dig_gla_test_skip_items(int n) { dig::g_test_skip.store(n > 0 ? n : 0); }
 
 void dig_gla_release(void) {
   std::lock_guard<std::mutex> lk(dig::g_mu);

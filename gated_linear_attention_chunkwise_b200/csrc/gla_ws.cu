@@ -107,6 +107,7 @@ struct WsArgs {
   int* flags;     // [BH][NS]               0 nothing, 1 aggregate, 2 inclusive
   int* ticket;
   int H, BH, dk, dv, NC, NS, G, items;
+  int skip;  // items left out (test hook; 0 normally)
   int Kp, Np, nstage, nO, nbuf;
   int nak, nav;  // full 16-channel atoms of q/k and v loaded by one box each (raster scans; else 0)
   uint32_t colO0, colO1, colSeg0, colSeg1, colSeg2;
@@ -678,7 +679,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
     }
     mbar_init(BAR(kBarDrain), 1);
     fence_mbar_init();
-    sMisc[0] = atomicAdd(a.ticket, 1);
+    sMisc[0] = atomicAdd(a.ticket, 1) + a.skip;
     sMisc[1] = 0;
     sMisc[3] = 0;
     sMisc[4] = 0;
@@ -751,7 +752,7 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
       int have = 0;  // items claimed (their pass 1 posted)
       bool ok = true, more = true;
       auto claim = [&]() {
-        const int t = have == 0 ? sMisc[0] : atomicAdd(a.ticket, 1);
+        const int t = have == 0 ? sMisc[0] : atomicAdd(a.ticket, 1) + a.skip;
         if (t >= a.items) {
           more = false;
           return;
@@ -1497,6 +1498,7 @@ cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const fl
   a.colSeg2 = L.colSeg2;
   a.nbuf = L.nbuf;
   a.items = (int)(BH * L.NS);
+  a.skip = take_test_skip_items();
   a.oTm = L.oTm;
   a.g = make_geom(s.Hg, s.Wg, s.dir);
 

@@ -42,6 +42,9 @@ cudaError_t srem_reorient_launch(const void* x, void* y, int dir, int inverse, i
 cudaError_t dwconv3x3_launch(const void* x, const float* w, void* y, int B, int Hg, int Wg, int C, int dtype,
                              cudaStream_t st);
 
+// ---- test hook: work items the next bf16 GLA call leaves out (0 normally) ----
+int take_test_skip_items();
+
 // ---- status word ----
 cudaError_t read_and_clear_device_status(int* status, cudaStream_t st);
 

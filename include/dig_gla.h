@@ -170,6 +170,18 @@ const char* dig_gla_status_string(int status);
  */
 void dig_gla_release(void);
 
+/*
+ * dig_gla_test_skip_items -- test hook for gla_fwd's bounded waits (bf16 path only).
+ * The next gla_fwd call of this process starts its work-item counter at n instead of
+ * 0, so its first n items (segments of 3 chunks, taken segment-major over B*H) are
+ * never processed and never publish their look-back flags; the waits of later
+ * segments on those flags run out after about a second of GPU time.  That call
+ * returns GLA_OK, dig_gla_device_status then reports GLA_ERR_TIMEOUT, and its output
+ * is unspecified; the CUDA context stays usable and later calls are unaffected.
+ * n <= 0 clears a pending request.
+ */
+void dig_gla_test_skip_items(int n);
+
 #ifdef __cplusplus
 }
 #endif

@@ -22,8 +22,8 @@ def declared_functions():
 
 @pytest.fixture(scope="module")
 def lib():
-    from gated_linear_attention_chunkwise_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._cuda_builder().build()  # by path: the package loads the library on import
     import gated_linear_attention_chunkwise_b200 as pkg
     return pkg.lib()
 

@@ -230,6 +230,28 @@ def test_gla_on_side_stream(dig):
     check_bf16(out.float().cpu().numpy(), oracle.gla_fwd(q, k, v, la, 16, 16, 2), "side stream")
 
 
+def test_gla_lookback_wait_runs_out_and_reports_timeout(dig):
+    """A look-back flag that nothing sets: the wait gives up, the status word says so,
+    and the context stays usable.  32x32 grid = 8 chunks = 3 segments, one head; the
+    test hook leaves out segment 0, whose flags the other two segments wait for."""
+    import time
+    w = workloads.custom(1, 1, 32, 32, 64, 64, "bf16")
+    q, k, v, la = workloads.gla_inputs(w, seed=4)
+    qd, kd, vd, ld = to_dev(q, k, v, la)
+    assert dig.device_status() == 0
+    dig.skip_items_for_test(1)
+    t0 = time.monotonic()
+    dig.gla_fwd(qd, kd, vd, ld, 32, 32, 0)
+    status = dig.device_status()
+    waited = time.monotonic() - t0
+    print(f"bounded look-back wait: status {dig.status_string(status)} after {waited:.2f} s")
+    assert status == -5  # GLA_ERR_TIMEOUT
+    assert waited < 60.0
+    # The hook applies to one call only, and the next call is exact again.
+    got = gpu_gla(dig, q, k, v, la, 32, 32, 0)
+    check_bf16(got, oracle.gla_fwd(q, k, v, la, 32, 32, 0), "after a timed-out call")
+
+
 # --------------------------------------------------------------------------- GLA fp32
 def test_gla_f32_config_c1(dig):
     w = workloads.WORKLOADS["c1"]
