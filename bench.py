@@ -361,7 +361,9 @@ def run_gpu(args):
                                        "dwconv3x3": statistics.mean(conv_ms) * 1e3,
                                        "srem_reorient": statistics.mean(reor_ms) * 1e3},
             "gla_only": {"tokens_heads_per_s": w.token_heads / gla_avg_s,
-                         "tflops": GLA_FLOP_PER_TOKEN_HEAD * w.token_heads / gla_avg_s / 1e12},
+                         "tflops": GLA_FLOP_PER_TOKEN_HEAD * w.token_heads / gla_avg_s / 1e12,
+                         "median_us": statistics.median(gla_ms) * 1e3,
+                         "median_us_by_dir": [statistics.median(gla_ms[l::LAYERS]) * 1e3 for l in range(LAYERS)]},
             "per_kernel": per_kernel(w, gla_ms, conv_ms, reor_ms, hbm),
             "other_configs_gla_fwd": extra,
         }
