@@ -217,6 +217,17 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------------------- GPU arm
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks of the process group (x itself on a single rank):
+    every multi-rank time is the slowest rank's."""
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_gpu(args):
     import torch.distributed as dist
 
@@ -289,10 +300,7 @@ def run_gpu(args):
     if status != 0:
         raise RuntimeError(f"device status after timing: {dig.status_string(status)}")
 
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(elapsed_ms, world, dev)
     th_per_step = w.token_heads * LAYERS
     value = th_per_step * args.steps * world / (max_ms / 1e3)
 
@@ -343,10 +351,7 @@ def run_gpu(args):
         stream.wait_event(out_free[l])  # every result is on the host
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = th_per_step * e2e_steps * world / (float(te.item()) / 1e3)
+    e2e_value = th_per_step * e2e_steps * world / (max_over_ranks(e0.elapsed_time(e1), world, dev) / 1e3)
 
     peaks, peak_kind = measured_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
