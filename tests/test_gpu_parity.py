@@ -126,6 +126,7 @@ SMALL_CASES = [
     (1, 1, 20, 13, 128, 128),   # largest dims
     (1, 2, 16, 24, 16, 48),
     (1, 1, 1, 1, 64, 64),       # T = 1
+    (1, 2, 130, 3, 64, 64),     # columns longer than a chunk: two pieces per column
 ]
 
 
