@@ -25,6 +25,8 @@ namespace {
 std::mutex g_mu;
 int g_arch_ok[64];  // per device: 0 unknown, 1 sm_100, -1 other
 
+}  // namespace
+
 int check_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GLA_ERR_CUDA;
@@ -40,12 +42,16 @@ int check_device() {
   return g_arch_ok[dev] == 1 ? GLA_OK : GLA_ERR_UNSUPPORTED;
 }
 
+namespace {
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
   return a0 < b0 + nb && b0 < a0 + na;
 }
+
+}  // namespace
 
 int validate_gla(const void* q, const void* k, const void* v, const void* la, const void* out, int B, int H,
                  int Hg, int Wg, int dk, int dv, int dir, size_t elt) {
@@ -66,6 +72,8 @@ int validate_gla(const void* q, const void* k, const void* v, const void* la, co
     return GLA_ERR_INVALID_ARG;
   return GLA_OK;
 }
+
+namespace {
 
 int validate_grid(const void* x, const void* y, int B, int Hg, int Wg, int C, int dtype, size_t* row_bytes) {
   if (!x || !y) return GLA_ERR_INVALID_ARG;
@@ -248,10 +256,18 @@ const char* dig_gla_status_string(int status) {
 void dig_gla_test_skip_items(int n) { dig::g_test_skip.store(n > 0 ? n : 0); }
 
 void dig_gla_release(void) {
-  std::lock_guard<std::mutex> lk(dig::g_mu);
-  memset(dig::g_arch_ok, 0, sizeof(dig::g_arch_ok));
-  for (cudaMemPool_t p : dig::g_pool)
-    if (p) cudaMemPoolTrimTo(p, 0);  // memory of allocations still in flight stays
+  {
+    std::lock_guard<std::mutex> lk(dig::g_mu);
+    memset(dig::g_arch_ok, 0, sizeof(dig::g_arch_ok));
+    for (cudaMemPool_t& p : dig::g_pool) {
+      // Allocations still in flight keep their memory until they are freed; the
+      // pool itself goes once they are.  The next call creates a new one.
+      if (p) cudaMemPoolDestroy(p);
+      p = nullptr;
+    }
+  }
+  cudaGetLastError();
+  dig::noalloc_forget();
 }
 
 }  // extern "C"

@@ -1,6 +1,6 @@
 // gla_simt.cu -- chunk-wise GLA forward with fp32 q/k/v/out on CUDA cores.
 //
-// Same decomposition as the tensor-core path (gla_tc.cu), with chunks of 64 scan
+// Chunk-wise decomposition in three kernels, with chunks of 64 scan
 // positions and every product in fp32 FMA, so the result carries no bf16/tf32
 // operand rounding:
 //   pass 1  S_loc = K^T V with K^_s = k_s exp(u_s),  gamma = exp(g)

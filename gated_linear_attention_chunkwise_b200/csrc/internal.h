@@ -45,6 +45,15 @@ cudaError_t dwconv3x3_launch(const void* x, const float* w, void* y, int B, int 
 // ---- test hook: work items the next bf16 GLA call leaves out (0 normally) ----
 int take_test_skip_items();
 
+// ---- host checks shared by the entry points (api.cu) ----
+// GLA_OK when the current device is an sm_100 part (cached per device).
+int check_device();
+// Argument validation of a GLA call with q/k/v/out elements of `elt` bytes.
+int validate_gla(const void* q, const void* k, const void* v, const void* la, const void* out, int B, int H, int Hg,
+                 int Wg, int dk, int dv, int dir, size_t elt);
+// Forgets the cached device address of the no-allocation scratch array (gla_noalloc.cu).
+void noalloc_forget();
+
 // ---- status word ----
 cudaError_t read_and_clear_device_status(int* status, cudaStream_t st);
 

@@ -106,13 +106,16 @@ int gla_fwd_f32(const float* q, const float* k, const float* v, const float* log
  * array of DIG_GLA_NOALLOC_SCRATCH_BYTES (8 MiB) of device memory inside the
  * library, which every GPU that loads the library holds until the process exits.
  *
- *   - Capacity: the call needs 2*ceil(T/64)*B*H*dk*dv*4 + ceil(T/64)*B*H*(dk+1)*4
- *     bytes of scratch (each term rounded up to 256); a larger problem returns
- *     GLA_ERR_UNSUPPORTED and launches nothing.  (c1: B=2, H=6, T=256, d=64 needs
- *     about 1.6 MB.)
+ *   - Capacity: with n = B*H*ceil(T/64) and rup(x) = x rounded up to a multiple
+ *     of 256, the call needs
+ *         2*rup(n*dk*dv*4) + rup(n*dk*4) + rup(n*4)
+ *     bytes of scratch, at most DIG_GLA_NOALLOC_SCRATCH_BYTES; a larger problem
+ *     returns GLA_ERR_UNSUPPORTED and launches nothing.  (B=2, H=6, T=256, d=64
+ *     needs about 1.6 MB; B=H=1, dk=dv=128 fits up to T=4032.)
  *   - First call per device: it looks up the array's device address with
  *     cudaGetSymbolAddress (with that device current) and caches it.  Make this
- *     first call before any stream capture.
+ *     first call before any stream capture.  Call dig_gla_release() before a
+ *     cudaDeviceReset: a new context places the array at a new address.
  *   - Sharing: every call uses the same array, which keeps the last call's
  *     contents; nothing in it needs to start at zero.  Calls that overlap on the
  *     GPU (concurrent streams, or host threads launching at the same time) race on
@@ -162,11 +165,13 @@ int dig_gla_device_status(cudaStream_t stream);
 const char* dig_gla_status_string(int status);
 
 /*
- * dig_gla_release -- forgets cached host-side state and returns the library's
- * unused GLA scratch memory to the device.  The scratch comes from a per-device
- * stream-ordered memory pool that keeps its memory across stream synchronisations
- * (so repeated calls do not map it again); scratch of calls still in flight stays
- * allocated until they complete.
+ * dig_gla_release -- forgets cached host-side state (device checks, the device
+ * addresses of gla_fwd_f32_noalloc's scratch array) and destroys the library's
+ * per-device memory pools, returning their memory to the device.  The GLA scratch
+ * comes from such a pool, which keeps its memory across stream synchronisations so
+ * that repeated calls do not map it again; scratch of calls still in flight stays
+ * allocated until they complete.  Call it before cudaDeviceReset (the cached pools
+ * and addresses belong to the context being destroyed); later calls set up anew.
  */
 void dig_gla_release(void);
 
