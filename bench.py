@@ -13,7 +13,14 @@ needed between iterations.
 The metric is token-heads per second (B*T*H per layer) over the whole step;
 `roofline` reports the GLA forward (the dominant op) against measured HBM
 bandwidth; `cpu_baseline` times the fp64 CPU oracle on a bounded sample of the
-same workload.  Under torchrun (N > 1) every rank runs its own replica of the
+same workload (all host threads, and one thread beside it).  `value` is the step
+throughput; `gla_only` gives the GLA forward alone, the op the metric names.
+
+Beside the headline (rank 0, unless --no-extras): a long window of c4 GLA launches
+(at least one second of device time, its own clock samples, median per direction),
+and the 28-layer DiG-XL/2 stack at 2048 resolution (gla_fwd -> dwconv3x3 ->
+srem_reorient per layer, fresh inputs per layer, dir = layer % 4), timed with and
+without the reorientation.  Under torchrun (N > 1) every rank runs its own replica of the
 workload (no data exchange: heads and batches are independent), and rank 0
 prints the aggregate.
 """
@@ -174,6 +181,24 @@ def oracle_sample(seconds_target: float = 12.0):
     desc = (f"fp64 C oracle on heads 0..{nh - 1} of {w.B * w.H} (whole 12544-token scans) x 4 directions, "
             f"plus dwconv3x3 + reorient on the sampled heads' channels")
     return nh * w.T * LAYERS, secs, threads, desc
+
+
+def oracle_sample_one_core():
+    """The oracle on one host thread: one head of the c4 workload through the four
+    directions (whole 12544-token scans) plus dwconv3x3 and the reorientation on that
+    head's 72 channels.  Returns (token_heads, seconds, description)."""
+    import oracle
+    w = WORKLOAD
+    q, k, v, la = (t.double().numpy() for t in workloads.gla_inputs(w, seed=0))
+    conv_w = workloads.conv_weight(w.C, seed=0).double().numpy()
+    t0 = time.perf_counter()
+    for layer in range(LAYERS):
+        out = oracle.gla_fwd(q, k, v, la, w.Hgrid, w.Wgrid, layer, nthreads=1, heads=(0, 1))
+        grid = out[:1, :, :1, :].reshape(1, w.Hgrid, w.Wgrid, w.dv)
+        oracle.dwconv3x3(grid, conv_w[: w.dv], nthreads=1)
+        oracle.reorient(grid.reshape(1, w.T, w.dv), (layer + 1) % 4, 0, w.Hgrid, w.Wgrid)
+    secs = time.perf_counter() - t0
+    return w.T * LAYERS, secs, "fp64 C oracle, 1 thread: head 0 of 32 x 4 directions, conv + reorient on its channels"
 
 
 def run_reference(args):
@@ -357,6 +382,10 @@ def run_gpu(args):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     extra = other_configs(dig, dev, stream, hbm) if (rank == 0 and not args.no_other_configs) else None
     gla_avg_s = statistics.mean(gla_ms) / 1e3
+    window = stack = None
+    if rank == 0 and not args.no_extras:
+        window = long_window(dig, dev, stream, dev_in, outs, hbm, gla_us_hint=gla_avg_s * 1e6)
+        stack = stack_c5(dig, dev, stream, hbm)
     gla_bytes = GLA_BYTES_PER_TOKEN_HEAD * w.token_heads
     achieved = gla_bytes / gla_avg_s / 1e9
     traffic = recorded_traffic()
@@ -368,8 +397,12 @@ def run_gpu(args):
             th, secs, threads, desc = oracle_sample(args.cpu_seconds)
             cpu = {"value": th / secs, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
                    "seconds": secs}
+            th1, secs1, desc1 = oracle_sample_one_core()
+            cpu["one_core"] = {"value": th1 / secs1, "unit": UNIT, "cores": 1, "sample": desc1, "seconds": secs1}
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": METRIC, "value": value, "unit": UNIT,
+            "value_is": ("step throughput: token-heads per second through 4 x (gla_fwd + dwconv3x3 + "
+                         "srem_reorient) on c4; the GLA forward alone is gla_only.tokens_heads_per_s"), "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_dict({"parallelism": f"replicas x{world}" if world > 1 else "single GPU"}),
@@ -393,6 +426,8 @@ def run_gpu(args):
                          "median_us_by_dir": [statistics.median(gla_ms[l::LAYERS]) * 1e3 for l in range(LAYERS)]},
             "per_kernel": per_kernel(w, gla_ms, conv_ms, reor_ms, hbm),
             "other_configs_gla_fwd": extra,
+            "gla_long_window_c4": window,
+            "stack_c5_28_layers": stack,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -436,6 +471,104 @@ def other_configs(dig, dev, stream, hbm, reps=10):
     return res
 
 
+def stack_c5(dig, dev, stream, hbm, reps=5):
+    """The 28-layer DiG-XL/2 stack at 2048 resolution (128x128 grid, B=1, H=16, d=72):
+    layer l runs gla_fwd(dir = l % 4) -> dwconv3x3 -> srem_reorient(dir = (l+1) % 4)
+    on its own seeded inputs (drawn on the device, 189 MB per layer, 5.3 GB in all)
+    and writes its own output buffers.  Timed with CUDA events around the whole stack,
+    median of `reps` stacks, with and without the reorientation (whose result feeds
+    nothing, since every layer's q/k/v are fresh)."""
+    w = workloads.WORKLOADS["c5"]
+    L = w.layers
+    ins = [workloads.gla_inputs_device(w, seed=l, device=dev) for l in range(L)]
+    cws = [workloads.conv_weight_device(w.C, seed=l, device=dev) for l in range(L)]
+    outs = [torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device=dev) for _ in range(L)]
+    convs = [torch.empty((w.B, w.Hgrid, w.Wgrid, w.C), dtype=torch.bfloat16, device=dev) for _ in range(L)]
+    reor = [torch.empty((w.B, w.T, w.C), dtype=torch.bfloat16, device=dev) for _ in range(L)]
+
+    def run(with_reorient, ev=None):
+        for l in range(L):
+            q, k, v, la = ins[l]
+            if ev is not None:
+                ev[l][0].record(stream)
+            dig.gla_fwd(q, k, v, la, w.Hgrid, w.Wgrid, l % 4, out=outs[l])
+            if ev is not None:
+                ev[l][1].record(stream)
+            dig.dwconv3x3(outs[l].view(w.B, w.Hgrid, w.Wgrid, w.C), cws[l], out=convs[l])
+            if ev is not None:
+                ev[l][2].record(stream)
+            if with_reorient:
+                dig.srem_reorient(convs[l].view(w.B, w.T, w.C), (l + 1) % 4, 0, w.Hgrid, w.Wgrid, out=reor[l])
+            if ev is not None:
+                ev[l][3].record(stream)
+
+    res = {"workload": w.name, "layers": L, "dirs": "layer % 4", "inputs": "fresh per layer, seed = layer",
+           "reps": reps}
+    for with_reorient in (True, False):
+        run(with_reorient)
+        totals, gla, conv, reo = [], [], [], []
+        for _ in range(reps):
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(L)]
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record(stream)
+            run(with_reorient, ev)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            totals.append(e0.elapsed_time(e1) * 1e3)
+            gla += [e[0].elapsed_time(e[1]) * 1e3 for e in ev]
+            conv += [e[1].elapsed_time(e[2]) * 1e3 for e in ev]
+            if with_reorient:
+                reo += [e[2].elapsed_time(e[3]) * 1e3 for e in ev]
+        us = statistics.median(totals)
+        key = "with_reorient" if with_reorient else "without_reorient"
+        res[key] = {"stack_us": us, "tokens_heads_per_s": w.token_heads * L / (us / 1e6),
+                    "gla_fwd_us_per_layer": statistics.mean(gla), "dwconv3x3_us_per_layer": statistics.mean(conv)}
+        if with_reorient:
+            res[key]["srem_reorient_us_per_layer"] = statistics.mean(reo)
+    gla_bytes = (2 * (2 * w.dk + w.dv) + 4 * w.dk + 2 * w.dv) * w.token_heads
+    res["gla_fwd_frac_of_hbm"] = gla_bytes / (res["with_reorient"]["gla_fwd_us_per_layer"] / 1e6) / 1e9 / hbm
+    status = dig.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after the c5 stack: {dig.status_string(status)}")
+    del ins, outs, convs, reor
+    return res
+
+
+def long_window(dig, dev, stream, dev_in, outs, hbm, seconds=1.0, gla_us_hint=220.0):
+    """c4 GLA forward alone, back to back over the four directions for at least
+    `seconds` of device time (each launch on its own layer's inputs, 347 MB > L2), with
+    its own clock samples: median per direction and the mean."""
+    w = WORKLOAD
+    rounds = int(seconds * 1e6 / (4 * gla_us_hint)) + 1
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(4)]
+          for _ in range(rounds)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index or 0) as clk:
+        e0.record(stream)
+        for r in range(rounds):
+            for l in range(4):
+                q, k, v, la = dev_in[l]
+                ev[r][l][0].record(stream)
+                dig.gla_fwd(q, k, v, la, w.Hgrid, w.Wgrid, l, out=outs[l])
+                ev[r][l][1].record(stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    per_dir = [[ev[r][l][0].elapsed_time(ev[r][l][1]) * 1e3 for r in range(rounds)] for l in range(4)]
+    allv = [x for d in per_dir for x in d]
+    mean_us = statistics.mean(allv)
+    status = dig.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after the long window: {dig.status_string(status)}")
+    return {"launches": 4 * rounds, "window_s": e0.elapsed_time(e1) / 1e3,
+            "median_us_by_dir": [statistics.median(d) for d in per_dir], "mean_us": mean_us,
+            "p90_us": sorted(allv)[int(0.9 * len(allv))],
+            "tokens_heads_per_s": w.token_heads / (mean_us / 1e6),
+            "frac_of_hbm": GLA_BYTES_PER_TOKEN_HEAD * w.token_heads / (mean_us / 1e6) / 1e9 / hbm,
+            "clocks": clk.summary()}
+
+
 def per_kernel(w, gla_ms, conv_ms, reor_ms, hbm):
     """Achieved algorithmic GB/s (and TFLOP/s for the GLA) of each op of a layer and of
     the layer as a whole, from the event-timed means, with the fraction of the HBM peak."""
@@ -468,6 +601,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-configs", action="store_true",
                     help="skip the supplementary GLA timings on the c2, c3 and c5 shapes")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the long c4 GLA window and the 28-layer c5 stack")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

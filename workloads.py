@@ -113,3 +113,31 @@ def grid_tensor(B: int, Hgrid: int, Wgrid: int, C: int, dtype=torch.bfloat16, se
     gen.manual_seed(int(seed) + 2_000_003)
     x = torch.randn((B, Hgrid, Wgrid, C), generator=gen, dtype=torch.float32)
     return x.to(dtype).contiguous()
+
+
+def gla_inputs_device(w: Workload, seed: int, device, qkv_scale: float | None = None):
+    """The same recipe as gla_inputs, drawn on `device` from a device generator seeded
+    by `seed` (a different random stream from the CPU one, so the values differ from
+    gla_inputs'): for timing many fresh layers without a host round trip, never for
+    parity checks."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    scale = (1.0 / math.sqrt(w.dk)) if qkv_scale is None else qkv_scale
+    shp_k = (w.B, w.T, w.H, w.dk)
+    shp_v = (w.B, w.T, w.H, w.dv)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q = (torch.randn(shp_k, generator=gen, dtype=torch.float32, device=device) * scale).to(dt)
+    k = (torch.randn(shp_k, generator=gen, dtype=torch.float32, device=device) * scale).to(dt)
+    v = (torch.randn(shp_v, generator=gen, dtype=torch.float32, device=device) * scale).to(dt)
+    g = torch.randn(shp_k, generator=gen, dtype=torch.float32, device=device) + w.g_mean
+    log_alpha = torch.nn.functional.logsigmoid(g) / 16.0
+    return q.contiguous(), k.contiguous(), v.contiguous(), log_alpha.contiguous()
+
+
+def conv_weight_device(C: int, seed: int, device, noise: float = 0.01):
+    """conv_weight's recipe drawn on `device` (timing only)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed) + 1_000_003)
+    w = torch.randn((C, 3, 3), generator=gen, dtype=torch.float32, device=device) * noise
+    w[:, 1, 1] += 1.0
+    return w.contiguous()
