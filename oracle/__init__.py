@@ -15,6 +15,9 @@ Functions and the passages they follow (see the C file for the full statement):
   gla_fwd          the GLA recurrence S_t = Diag(alpha_t) S_{t-1} + k_t^T v_t,
                    o_t = q_t S_t over the scan order, zero initial state, update
                    before read (diffusers draft "gated_linear_attention").
+  gla_bwd          the exact gradient of that recurrence (dq, dk, dv, dlog_alpha
+                   for a given d out), as reverse-mode differentiation of its steps
+                   in reverse scan order (DiG notes, training like DiT).
   dwconv3x3        DiG notes, SREM / DiG Block step (4): 3x3 depthwise conv on
                    the 2D token grid, zero padding.
   reorient         DiG notes, SREM: the O(T) transpose + flip as a row gather.
@@ -59,6 +62,10 @@ def _load():
         lib.oracle_gla_fwd.argtypes = [dp, dp, dp, dp] + [c_int] * 7 + [dp, c_int]
         lib.oracle_gla_fwd_heads.argtypes = [dp, dp, dp, dp] + [c_int] * 7 + [dp, c_int, c_i64, c_i64]
         lib.oracle_gla_fwd_planted.argtypes = [dp, dp, dp, dp] + [c_int] * 7 + [dp, c_int]
+        lib.oracle_gla_bwd.argtypes = [dp] * 5 + [c_int] * 7 + [dp] * 4 + [c_int, c_i64, c_i64]
+        lib.oracle_gla_bwd_planted.argtypes = [dp] * 5 + [c_int] * 7 + [dp] * 4 + [c_int]
+        lib.oracle_gla_bwd.restype = c_int
+        lib.oracle_gla_bwd_planted.restype = c_int
         lib.oracle_dwconv3x3.argtypes = [dp, dp, c_int, c_int, c_int, c_int, dp, c_int]
         lib.oracle_reorient.argtypes = [ctypes.c_void_p, c_int, c_int, c_int, c_int, c_int, c_i64,
                                         ctypes.c_void_p]
@@ -125,6 +132,32 @@ def gla_fwd(q, k, v, log_alpha, Hgrid: int, Wgrid: int, direction: int, nthreads
     else:
         rc = _check(lib.oracle_gla_fwd(*args, nthreads), "gla_fwd")
     return (out, rc) if return_threads else out
+
+
+def gla_bwd(q, k, v, log_alpha, dout, Hgrid: int, Wgrid: int, direction: int, nthreads: int = 0,
+            heads: tuple | None = None, planted: int = 0):
+    """fp64 GLA backward: the gradients (dq, dk, dv, dlog_alpha) of sum(dout * out),
+    out = gla_fwd(q, k, v, log_alpha, ...).  Shapes as gla_fwd; dout is [B,T,H,dv].
+
+    heads=(begin, end) restricts the work to flattened heads b*H+h in [begin, end)
+    (other gradients stay zero); each worker holds one head's T forward states.
+    planted != 0 runs a deliberately wrong variant.
+    """
+    q, k, v, la, do = _f64(q), _f64(k), _f64(v), _f64(log_alpha), _f64(dout)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    assert T == Hgrid * Wgrid and k.shape == q.shape and la.shape == q.shape and v.shape[:3] == q.shape[:3]
+    assert do.shape == v.shape
+    gq, gk, gv, gl = (np.zeros(a.shape, dtype=np.float64) for a in (q, k, v, la))
+    lib = _load()
+    args = (_dp(q), _dp(k), _dp(v), _dp(la), _dp(do), B, H, Hgrid, Wgrid, dk, dv, direction,
+            _dp(gq), _dp(gk), _dp(gv), _dp(gl))
+    if planted:
+        _check(lib.oracle_gla_bwd_planted(*args, planted), "gla_bwd_planted")
+    else:
+        lo, hi = (0, -1) if heads is None else (int(heads[0]), int(heads[1]))
+        _check(lib.oracle_gla_bwd(*args, nthreads, lo, hi), "gla_bwd")
+    return gq, gk, gv, gl
 
 
 def dwconv3x3(x, w, nthreads: int = 0) -> np.ndarray:

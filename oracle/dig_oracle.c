@@ -40,9 +40,25 @@
  * Threads: independent (batch, head) pairs or conv image rows are spread over
  * POSIX threads; this changes no arithmetic, only which core runs it.
  *
+ *  - GLA backward (DiG notes, "损失函数 / 训练策略": the model is trained like DiT,
+ *    so gradients flow back through every GLA layer; "硬件友好的效率设计": the
+ *    chunk-wise form is the training path).  The pages give no formula for it: it
+ *    is the exact gradient of the recurrence above, written as reverse-mode
+ *    differentiation of its steps, one step at a time in reverse scan order.  With
+ *    dO the gradient of the loss with respect to out, and G the gradient with
+ *    respect to the state S_p after step p (G = 0 past the last step):
+ *        G    += q_p^T dO_p                        (o_p = q_p S_p reads S_p)
+ *        dq_p  = dO_p S_p^T
+ *        dk_p  = G v_p^T,   dv_p = k_p G           (S_p contains k_p^T v_p)
+ *        dlog_alpha_p[i] = alpha_p[i] * sum_j G[i][j] S_{p-1}[i][j]
+ *        G     = Diag(alpha_p) G                   (S_p = Diag(alpha_p) S_{p-1} + ...)
+ *    The forward states S_p of the head are kept (T * dk * dv values) so that the
+ *    reverse sweep reads them exactly.
+ *
  * Planted mistakes: oracle_gla_fwd_planted() runs the same recurrence with one
- * deliberate error selected by `planted` (1..7).  Tests use it to show that the
- * oracle's pins catch each kind of mistake; the method itself is planted == 0.
+ * deliberate error selected by `planted` (1..7), and oracle_gla_bwd_planted()
+ * the backward sweep with one of 1..6.  Tests use them to show that the oracle's
+ * pins catch each kind of mistake; the method itself is planted == 0.
  */
 #include <math.h>
 #include <pthread.h>
@@ -308,6 +324,181 @@ int oracle_gla_fwd_planted(const double *q, const double *k, const double *v, co
 {
     if (planted < 0 || planted > 7) return ORACLE_BAD_ARG;
     return gla_common(q, k, v, log_alpha, B, H, Hgrid, Wgrid, dk, dv, dir, out, 1, planted, 0, -1);
+}
+
+/* ------------------------------------------------------------------------- */
+/* GLA backward: reverse sweep of the recurrence (fp64).                      */
+/* ------------------------------------------------------------------------- */
+typedef struct {
+    const double *q, *k, *v, *la, *dout;
+    double *dq, *dk, *dv, *dla;
+    const int64_t *order;
+    int64_t T;
+    int64_t bh_base;
+    int H, dk_, dv_;
+    int planted; /* 0 = the method; 1..6 = a planted mistake (tests only) */
+    int status;
+} gla_bwd_ctx;
+
+static void gla_bwd_head(void *vctx, int64_t i_local)
+{
+    gla_bwd_ctx *c = (gla_bwd_ctx *)vctx;
+    const int64_t bh = c->bh_base + i_local;
+    const int64_t b = bh / c->H, h = bh % c->H;
+    const int dk = c->dk_, dv = c->dv_;
+    const int64_t T = c->T, H = c->H;
+    const size_t sz = (size_t)dk * dv;
+    /* states[p] = S after step p; states[-1] (the zero initial state) is `zero` */
+    double *states = (double *)malloc(sizeof(double) * sz * (size_t)T);
+    double *zero = (double *)calloc(sz, sizeof(double));
+    double *G = (double *)calloc(sz, sizeof(double));
+    if (!states || !zero || !G) {
+        free(states);
+        free(zero);
+        free(G);
+        c->status = ORACLE_NOMEM;
+        return;
+    }
+
+    /* forward sweep: the states the reverse sweep reads */
+    for (int64_t p = 0; p < T; ++p) {
+        const int64_t t = c->order[p];
+        const double *kt = c->k + tok_off(b, t, h, T, H, dk);
+        const double *vt = c->v + tok_off(b, t, h, T, H, dv);
+        const double *lt = c->la + tok_off(b, t, h, T, H, dk);
+        const double *Sp = p ? states + (size_t)(p - 1) * sz : zero;
+        double *Sn = states + (size_t)p * sz;
+        for (int i = 0; i < dk; ++i) {
+            const double alpha = exp(lt[i]);
+            for (int j = 0; j < dv; ++j) Sn[(int64_t)i * dv + j] = alpha * Sp[(int64_t)i * dv + j] + kt[i] * vt[j];
+        }
+    }
+
+    /* reverse sweep */
+    for (int64_t p = T - 1; p >= 0; --p) {
+        const int64_t t = c->order[p];
+        const double *qt = c->q + tok_off(b, t, h, T, H, dk);
+        const double *kt = c->k + tok_off(b, t, h, T, H, dk);
+        const double *vt = c->v + tok_off(b, t, h, T, H, dv);
+        const double *lt = c->la + tok_off(b, t, h, T, H, dk);
+        const double *go = c->dout + tok_off(b, t, h, T, H, dv);
+        double *gq = c->dq + tok_off(b, t, h, T, H, dk);
+        double *gk = c->dk + tok_off(b, t, h, T, H, dk);
+        double *gv = c->dv + tok_off(b, t, h, T, H, dv);
+        double *gl = c->dla + tok_off(b, t, h, T, H, dk);
+        const double *Sp = states + (size_t)p * sz;                     /* S_p     */
+        const double *Sm = p ? states + (size_t)(p - 1) * sz : zero;     /* S_{p-1} */
+
+        /* o_p = q_p S_p: S_p receives q_p^T dO_p (planted 1: it is forgotten) */
+        if (c->planted != 1)
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j) G[(int64_t)i * dv + j] += qt[i] * go[j];
+        /* dq_p = dO_p S_p^T (planted 2: the state before the update is read) */
+        const double *Sq = (c->planted == 2) ? Sm : Sp;
+        for (int i = 0; i < dk; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dv; ++j) acc += go[j] * Sq[(int64_t)i * dv + j];
+            gq[i] = acc;
+        }
+        /* dk_p = G v_p^T, dv_p = k_p G (planted 3: q_p read in place of k_p) */
+        for (int i = 0; i < dk; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dv; ++j) acc += G[(int64_t)i * dv + j] * vt[j];
+            gk[i] = acc;
+        }
+        const double *kv = (c->planted == 3) ? qt : kt;
+        for (int j = 0; j < dv; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < dk; ++i) acc += kv[i] * G[(int64_t)i * dv + j];
+            gv[j] = acc;
+        }
+        /* dlog_alpha_p[i] = alpha_p[i] sum_j G[i][j] S_{p-1}[i][j]
+           (planted 4: S_p in place of S_{p-1}; planted 5: the factor alpha dropped) */
+        const double *Sa = (c->planted == 4) ? Sp : Sm;
+        for (int i = 0; i < dk; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dv; ++j) acc += G[(int64_t)i * dv + j] * Sa[(int64_t)i * dv + j];
+            gl[i] = (c->planted == 5) ? acc : exp(lt[i]) * acc;
+        }
+        /* gradient to S_{p-1}: G = Diag(alpha_p) G (planted 6: decay skipped) */
+        if (c->planted != 6)
+            for (int i = 0; i < dk; ++i) {
+                const double alpha = exp(lt[i]);
+                for (int j = 0; j < dv; ++j) G[(int64_t)i * dv + j] *= alpha;
+            }
+    }
+    free(states);
+    free(zero);
+    free(G);
+}
+
+static int gla_bwd_common(const double *q, const double *k, const double *v, const double *log_alpha,
+                          const double *dout, int B, int H, int Hgrid, int Wgrid, int dk, int dv, int dir,
+                          double *dq, double *dk_out, double *dv_out, double *dla, int nthreads, int planted,
+                          int64_t bh_begin, int64_t bh_end)
+{
+    if (!q || !k || !v || !log_alpha || !dout || !dq || !dk_out || !dv_out || !dla) return ORACLE_BAD_ARG;
+    if (B <= 0 || H <= 0 || Hgrid <= 0 || Wgrid <= 0 || dk <= 0 || dv <= 0) return ORACLE_BAD_ARG;
+    if (dir < 0 || dir > 3) return ORACLE_BAD_ARG;
+    const int64_t T = (int64_t)Hgrid * Wgrid;
+    const int64_t BH = (int64_t)B * H;
+    if (bh_begin < 0) bh_begin = 0;
+    if (bh_end < 0 || bh_end > BH) bh_end = BH;
+    if (bh_begin > bh_end) return ORACLE_BAD_ARG;
+    int64_t *order = (int64_t *)malloc(sizeof(int64_t) * T);
+    if (!order) return ORACLE_NOMEM;
+    int rc = oracle_scan_order(dir, Hgrid, Wgrid, order);
+    if (rc != ORACLE_OK) {
+        free(order);
+        return rc;
+    }
+    gla_bwd_ctx c;
+    c.q = q;
+    c.k = k;
+    c.v = v;
+    c.la = log_alpha;
+    c.dout = dout;
+    c.dq = dq;
+    c.dk = dk_out;
+    c.dv = dv_out;
+    c.dla = dla;
+    c.order = order;
+    c.T = T;
+    c.bh_base = bh_begin;
+    c.H = H;
+    c.dk_ = dk;
+    c.dv_ = dv;
+    c.planted = planted;
+    c.status = ORACLE_OK;
+    int used = run_pool(gla_bwd_head, &c, bh_end - bh_begin, nthreads);
+    free(order);
+    if (c.status != ORACLE_OK) return c.status;
+    return used;
+}
+
+/*
+ * GLA backward over flattened heads bh = b*H + h in [bh_begin, bh_end) (bh_end < 0:
+ * all).  Inputs as oracle_gla_fwd plus dout [B][T][H][dv]; outputs dq, dk,
+ * dlog_alpha [B][T][H][dk] and dv [B][T][H][dv] (heads outside the range are not
+ * written).  Each worker holds one head's T forward states.  Returns the number
+ * of threads used or a negative error code.
+ */
+int oracle_gla_bwd(const double *q, const double *k, const double *v, const double *log_alpha,
+                   const double *dout, int B, int H, int Hgrid, int Wgrid, int dk, int dv, int dir, double *dq,
+                   double *dk_out, double *dv_out, double *dla, int nthreads, int64_t bh_begin, int64_t bh_end)
+{
+    return gla_bwd_common(q, k, v, log_alpha, dout, B, H, Hgrid, Wgrid, dk, dv, dir, dq, dk_out, dv_out, dla,
+                          nthreads, 0, bh_begin, bh_end);
+}
+
+/* The backward sweep with one deliberate mistake (tests of the pins only). */
+int oracle_gla_bwd_planted(const double *q, const double *k, const double *v, const double *log_alpha,
+                           const double *dout, int B, int H, int Hgrid, int Wgrid, int dk, int dv, int dir,
+                           double *dq, double *dk_out, double *dv_out, double *dla, int planted)
+{
+    if (planted < 0 || planted > 6) return ORACLE_BAD_ARG;
+    return gla_bwd_common(q, k, v, log_alpha, dout, B, H, Hgrid, Wgrid, dk, dv, dir, dq, dk_out, dv_out, dla, 1,
+                          planted, 0, -1);
 }
 
 /* ------------------------------------------------------------------------- */
