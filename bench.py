@@ -20,7 +20,7 @@ Beside the headline (rank 0, unless --no-extras): a long window of c4 GLA launch
 (at least one second of device time, its own clock samples, median per direction),
 and the 28-layer DiG-XL/2 stack at 2048 resolution (gla_fwd -> dwconv3x3 ->
 srem_reorient per layer, fresh inputs per layer, dir = layer % 4), timed with and
-without the reorientation.  Under torchrun (N > 1) every rank runs its own replica of the
+without the reorientation; and the GLA backward (gla_bwd) on c4 and c2.  Under torchrun (N > 1) every rank runs its own replica of the
 workload (no data exchange: heads and batches are independent), and rank 0
 prints the aggregate.
 """
@@ -382,10 +382,11 @@ def run_gpu(args):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     extra = other_configs(dig, dev, stream, hbm) if (rank == 0 and not args.no_other_configs) else None
     gla_avg_s = statistics.mean(gla_ms) / 1e3
-    window = stack = None
+    window = stack = bwd = None
     if rank == 0 and not args.no_extras:
         window = long_window(dig, dev, stream, dev_in, outs, hbm, gla_us_hint=gla_avg_s * 1e6)
         stack = stack_c5(dig, dev, stream, hbm)
+        bwd = bwd_configs(dig, dev, stream, hbm)
     gla_bytes = GLA_BYTES_PER_TOKEN_HEAD * w.token_heads
     achieved = gla_bytes / gla_avg_s / 1e9
     traffic = recorded_traffic()
@@ -428,6 +429,7 @@ def run_gpu(args):
             "other_configs_gla_fwd": extra,
             "gla_long_window_c4": window,
             "stack_c5_28_layers": stack,
+            "gla_bwd": bwd,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -567,6 +569,42 @@ def long_window(dig, dev, stream, dev_in, outs, hbm, seconds=1.0, gla_us_hint=22
             "tokens_heads_per_s": w.token_heads / (mean_us / 1e6),
             "frac_of_hbm": GLA_BYTES_PER_TOKEN_HEAD * w.token_heads / (mean_us / 1e6) / 1e9 / hbm,
             "clocks": clk.summary()}
+
+
+def bwd_configs(dig, dev, stream, hbm, reps=5):
+    """The GLA backward (gla_bwd, bf16) on c4 and c2: median of `reps` calls per
+    direction, event-timed, inputs resident in HBM, against the HBM roofline of its
+    algorithmic bytes: q, k, v, dout, log_alpha read once, dq, dk, dv, dlog_alpha
+    written once."""
+    res = {}
+    for name in ("c4", "c2"):
+        cw = workloads.WORKLOADS[name]
+        q, k, v, la = [t.to(dev) for t in workloads.gla_inputs(cw, seed=11)]
+        do = workloads.gla_dout(cw, seed=11).to(dev)
+        per_th = 2 * (2 * cw.dk + 2 * cw.dv) + 4 * cw.dk + 2 * (2 * cw.dk + cw.dv) + 4 * cw.dk
+        nbytes = per_th * cw.token_heads
+        per_dir = []
+        for d in range(4):
+            dig.gla_bwd(q, k, v, la, do, cw.Hgrid, cw.Wgrid, d)
+            ts = []
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                dig.gla_bwd(q, k, v, la, do, cw.Hgrid, cw.Wgrid, d)
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                ts.append(e0.elapsed_time(e1) * 1e3)
+            per_dir.append(statistics.median(ts))
+        us = statistics.mean(per_dir)
+        res[name] = {"workload": cw.name, "kernel": "gla_bwd (3 launches: local terms, chunk scans, gradients)",
+                     "us_per_dir": per_dir, "bytes": nbytes, "bytes_per_token_head": per_th,
+                     "tokens_heads_per_s": cw.token_heads / (us / 1e6),
+                     "frac_of_hbm": nbytes / (us / 1e6) / 1e9 / hbm}
+        del q, k, v, la, do
+    status = dig.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after the backward: {dig.status_string(status)}")
+    return res
 
 
 def per_kernel(w, gla_ms, conv_ms, reor_ms, hbm):

@@ -73,6 +73,30 @@ int validate_gla(const void* q, const void* k, const void* v, const void* la, co
   return GLA_OK;
 }
 
+// The backward's extra tensors: dout is read like v; dq, dk, dv, dlog_alpha are
+// written and may overlap nothing (validate_gla has checked q, k, v, log_alpha and dq).
+int validate_gla_bwd(const void* q, const void* k, const void* v, const void* la, const void* dout, const void* dq,
+                     const void* dk_out, const void* dv_out, const void* dla, int B, int H, int Hg, int Wg, int dk,
+                     int dv, int dir, size_t elt) {
+  int rc = validate_gla(q, k, v, la, dq, B, H, Hg, Wg, dk, dv, dir, elt);
+  if (rc != GLA_OK) return rc;
+  if (!dout || !dk_out || !dv_out || !dla) return GLA_ERR_INVALID_ARG;
+  if (!aligned16(dout) || !aligned16(dk_out) || !aligned16(dv_out) || !aligned16(dla)) return GLA_ERR_ALIGNMENT;
+  const size_t rows = (size_t)B * Hg * Wg * H;
+  const size_t nk = rows * dk * elt, nv = rows * dv * elt, nl = rows * dk * 4;
+  const void* in[5] = {q, k, v, la, dout};
+  const size_t nin[5] = {nk, nk, nv, nl, nv};
+  const void* outs[4] = {dq, dk_out, dv_out, dla};
+  const size_t nout[4] = {nk, nk, nv, nl};
+  for (int o = 0; o < 4; ++o) {
+    for (int i = 0; i < 5; ++i)
+      if (overlaps(outs[o], nout[o], in[i], nin[i])) return GLA_ERR_INVALID_ARG;
+    for (int o2 = o + 1; o2 < 4; ++o2)
+      if (overlaps(outs[o], nout[o], outs[o2], nout[o2])) return GLA_ERR_INVALID_ARG;
+  }
+  return GLA_OK;
+}
+
 namespace {
 
 int validate_grid(const void* x, const void* y, int B, int Hg, int Wg, int C, int dtype, size_t* row_bytes) {
@@ -187,9 +211,48 @@ cudaError_t run_f32(void* ws, void* ctx) {
   return dig::gla_f32_forward(static_cast<const float*>(c->q), static_cast<const float*>(c->k),
                               static_cast<const float*>(c->v), c->la, static_cast<float*>(c->out), c->s, ws, c->st);
 }
+struct BwdCall {
+  const void *q, *k, *v;
+  const float* la;
+  const void* dout;
+  void *dq, *dk, *dv;
+  float* dla;
+  GlaShape s;
+  int bf16;
+  cudaStream_t st;
+};
+cudaError_t run_bwd(void* ws, void* ctx) {
+  const BwdCall* c = static_cast<const BwdCall*>(ctx);
+  return dig::gla_bwd_launch(c->q, c->k, c->v, c->la, c->dout, c->dq, c->dk, c->dv, c->dla, c->s, c->bf16, ws,
+                             c->st);
+}
+int gla_bwd_common(const void* q, const void* k, const void* v, const float* la, const void* dout, int B, int H,
+                   int Hgrid, int Wgrid, int dk, int dv, int dir, void* dq, void* dk_out, void* dv_out, float* dla,
+                   int bf16, cudaStream_t stream) {
+  int rc = dig::validate_gla_bwd(q, k, v, la, dout, dq, dk_out, dv_out, dla, B, H, Hgrid, Wgrid, dk, dv, dir,
+                                 bf16 ? 2 : 4);
+  if (rc != GLA_OK) return rc;
+  if ((rc = dig::check_device()) != GLA_OK) return rc;
+  BwdCall c{q, k, v, la, dout, dq, dk_out, dv_out, dla, GlaShape{B, H, Hgrid, Wgrid, dk, dv, dir}, bf16, stream};
+  return dig::run_with_workspace(dig::gla_bwd_workspace_bytes(c.s), stream, run_bwd, &c);
+}
 }  // namespace
 
 extern "C" {
+
+int gla_bwd(const void* q, const void* k, const void* v, const float* log_alpha, const void* dout, int B, int H,
+            int Hgrid, int Wgrid, int dk, int dv, int dir, void* dq, void* dk_out, void* dv_out, float* dlog_alpha,
+            cudaStream_t stream) {
+  return gla_bwd_common(q, k, v, log_alpha, dout, B, H, Hgrid, Wgrid, dk, dv, dir, dq, dk_out, dv_out, dlog_alpha, 1,
+                        stream);
+}
+
+int gla_bwd_f32(const float* q, const float* k, const float* v, const float* log_alpha, const float* dout, int B,
+                int H, int Hgrid, int Wgrid, int dk, int dv, int dir, float* dq, float* dk_out, float* dv_out,
+                float* dlog_alpha, cudaStream_t stream) {
+  return gla_bwd_common(q, k, v, log_alpha, dout, B, H, Hgrid, Wgrid, dk, dv, dir, dq, dk_out, dv_out, dlog_alpha, 0,
+                        stream);
+}
 
 int gla_fwd(const void* q, const void* k, const void* v, const float* log_alpha, int B, int H, int Hgrid, int Wgrid,
             int dk, int dv, int dir, void* out, cudaStream_t stream) {

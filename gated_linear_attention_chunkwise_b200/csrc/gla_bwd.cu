@@ -1,0 +1,522 @@
+// gla_bwd.cu -- chunk-wise GLA backward on CUDA cores (fp32 arithmetic; bf16 or
+// fp32 q/k/v/dout/dq/dk/dv, fp32 log-gates and their gradient).
+//
+// The gradient of the recurrence S_t = Diag(alpha_t) S_{t-1} + k_t^T v_t,
+// o_t = q_t S_t (DiG trains like DiT, so the GLA layers are differentiated) is
+// taken chunk by chunk.  Inside a chunk of MC scan positions, with u_r the sum of
+// the log-gates scanned after row r, g the chunk total, S_in the state entering
+// the chunk and D the gradient of the loss with respect to the state leaving it:
+//   Q~ = q e^{-u},  K^ = k e^{u},  G = Diag(e^g) S_in
+//   A  = mask(dO V^T),  P = mask(Q~ K^T)             (s <= r in scan order)
+//   dQ~ = dO G^T + A K^,    dq = e^{-u} dQ~
+//   dK^ = A^T Q~ + V D^T,   dk = e^{u} dK^
+//   dV  = P^T dO + K^ D
+// Across chunks the forward state and its gradient run in opposite directions:
+//   S_in(c+1) = Diag(gamma_c) S_in(c) + K^_c^T V_c
+//   D(c-1)    = Diag(gamma_c) D(c) + Qbar_c^T dO_c,   Qbar = q e^{g-u} = q e^{b}
+// (b the inclusive prefix sum of the log-gates inside the chunk).
+// The log-gates enter only through their prefix sums b, and o depends on b through
+// q e^{b} and k e^{-b}; so dlog_alpha_r = sum over t >= r (scan order) of
+// q_t dq_t - k_t dk_t = Q~_t dQ~_t - K^_t dK^_t.  The part of that sum beyond the
+// chunk is the gradient of a scalar gate placed at the chunk's end,
+// carry_c[i] = sum_j D(c)[i][j] S_in(c+1)[i][j], so every chunk finishes on its own.
+//
+// Three kernels: per-chunk local terms (K^T V and Qbar^T dO), the two scans over
+// chunks (one thread per state element), and the per-chunk gradients.  Chunks
+// whose gates leave the fp32-safe range (|u| > 80, e.g. a full reset) take an exact
+// token-by-token reverse sweep from S_in and D instead of the factorised form.
+#include <math.h>
+
+#include "dev_common.cuh"
+#include "internal.h"
+
+namespace dig {
+
+namespace {
+
+constexpr int NT = 256;
+constexpr float kRange = 80.0f;
+
+template <typename TI>
+struct BwdArgs {
+  const TI* q;
+  const TI* k;
+  const TI* v;
+  const float* la;
+  const TI* dout;
+  TI* dq;
+  TI* dk_out;
+  TI* dv_out;
+  float* dla;
+  float* sx;     // [BH][NC][dk][dv]: K^T V of chunk c, then S_in(c+1)
+  float* dd;     // [BH][NC][dk][dv]: Qbar^T dO of chunk c, then D(c)
+  float* gamma;  // [BH][NC][dk]
+  int* flags;    // [BH][NC]: 1 = evaluate this chunk token by token
+  int H, dk, dv, NC;
+  ScanGeom g;
+};
+
+__device__ __forceinline__ void load8(const float* p, float* d) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  d[0] = a.x, d[1] = a.y, d[2] = a.z, d[3] = a.w, d[4] = b.x, d[5] = b.y, d[6] = b.z, d[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* d) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    const float2 f = __bfloat1622float2(h[x]);
+    d[2 * x] = f.x;
+    d[2 * x + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void store1(float* p, float x) { *p = x; }
+__device__ __forceinline__ void store1(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+
+// Rows f0 .. f0+MC-1 (base positions) of head h, batch b of a [B][T][H][d] tensor
+// into an fp32 tile with a pitch of d+4 floats; rows outside the sequence are zero.
+template <int MC, typename TE>
+__device__ __forceinline__ void stage(float* dst, const TE* src, int d, const ScanGeom& g, int f0, int b, int h,
+                                      int H) {
+  const int cpr = d / 8;
+  const int pitch = d + 4;
+  for (int idx = threadIdx.x; idx < MC * cpr; idx += NT) {
+    const int r = idx / cpr;
+    const int cc = idx - r * cpr;
+    const int f = f0 + r;
+    float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (f >= 0 && f < g.T) load8(src + (((int64_t)b * g.T + base_pos_to_token(g, f)) * H + h) * d + cc * 8, x);
+    float* o = dst + r * pitch + cc * 8;
+    *reinterpret_cast<float4*>(o) = make_float4(x[0], x[1], x[2], x[3]);
+    *reinterpret_cast<float4*>(o + 4) = make_float4(x[4], x[5], x[6], x[7]);
+  }
+}
+
+// Threads i < dk: the log-gate tile becomes, in place, the exclusive suffix sums u
+// along the scan order; the chunk total goes to sTot[i].  Returns bit 1 if |u| or
+// the total leave the fp32-safe range (evaluate token by token), bit 2 if growth
+// gates exceed it (not representable).
+template <int MC>
+__device__ __forceinline__ int suffix_sums(float* sU, float* sTot, int dk, int reverse) {
+  const int i = threadIdx.x;
+  int code = 0;
+  if (i < dk) {
+    const int pw = dk + 4;
+    float acc = 0.f, lo = 0.f, hi = 0.f;
+    for (int s = 0; s < MC; ++s) {
+      const int r = reverse ? s : (MC - 1 - s);
+      const float l = sU[r * pw + i];
+      sU[r * pw + i] = acc;
+      lo = fminf(lo, acc);
+      hi = fmaxf(hi, acc);
+      acc += l;
+    }
+    sTot[i] = acc;
+    lo = fminf(lo, acc);
+    hi = fmaxf(hi, acc);
+    if (!(lo >= -kRange) || !(hi <= kRange)) code |= 1;
+    if (!(hi <= kRange)) code |= 2;
+  }
+  return code;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 1: per-chunk K^T V (forward state) and Qbar^T dO (backward state).
+// ---------------------------------------------------------------------------
+template <typename TI, int MC>
+__global__ void __launch_bounds__(NT) gla_bwd_local(const BwdArgs<TI> a) {
+  extern __shared__ float4 smem_f4[];
+  float* smem = reinterpret_cast<float*>(smem_f4);
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int pk = a.dk + 4, pv = a.dv + 4;
+  float* sK = smem;
+  float* sQ = sK + MC * pk;
+  float* sU = sQ + MC * pk;
+  float* sV = sU + MC * pk;
+  float* sO = sV + MC * pv;
+  float* sTot = sO + MC * pv;
+
+  const int f0 = chunk_first_base_pos(a.g, c, MC);
+  stage<MC>(sK, a.k, a.dk, a.g, f0, b, h, a.H);
+  stage<MC>(sQ, a.q, a.dk, a.g, f0, b, h, a.H);
+  stage<MC>(sU, a.la, a.dk, a.g, f0, b, h, a.H);
+  stage<MC>(sV, a.v, a.dv, a.g, f0, b, h, a.H);
+  stage<MC>(sO, a.dout, a.dv, a.g, f0, b, h, a.H);
+  __syncthreads();
+  // Qbar = q e^{b}, b the inclusive prefix sum of the log-gates in scan order (formed
+  // directly, not as g - u, so that a -inf gate gives 0 rather than inf - inf).
+  for (int i = threadIdx.x; i < a.dk; i += NT) {
+    float acc = 0.f;
+    for (int s = 0; s < MC; ++s) {
+      const int r = a.g.reverse ? (MC - 1 - s) : s;
+      acc += sU[r * pk + i];
+      sQ[r * pk + i] *= expf(acc);
+    }
+  }
+  __syncthreads();
+  const int code = suffix_sums<MC>(sU, sTot, a.dk, a.g.reverse);
+  if (code & 2) report_status(GLA_ERR_RANGE);
+  const int wide = __syncthreads_or(code != 0);
+  // K^ = k e^{u}: the exponent is a sum of log-gates, so decays only shrink it.
+  for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
+    const int r = e / a.dk, i = e - r * a.dk;
+    sK[r * pk + i] *= expf(sU[r * pk + i]);
+  }
+  __syncthreads();
+  const int64_t cid = (int64_t)bh * a.NC + c;
+  float* sx = a.sx + cid * a.dk * a.dv;
+  float* dd = a.dd + cid * a.dk * a.dv;
+  for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+    const int i = e / a.dv, j = e - i * a.dv;
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll 8
+    for (int r = 0; r < MC; ++r) {
+      s1 = fmaf(sK[r * pk + i], sV[r * pv + j], s1);
+      s2 = fmaf(sQ[r * pk + i], sO[r * pv + j], s2);
+    }
+    sx[e] = s1;
+    dd[e] = s2;
+  }
+  if (threadIdx.x < a.dk) a.gamma[cid * a.dk + threadIdx.x] = expf(sTot[threadIdx.x]);
+  if (threadIdx.x == 0) a.flags[cid] = wide;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 2: per state element (i, j) of each head, the forward scan
+// S_in(c+1) = gamma_c S_in(c) + (K^T V)_c and the reverse scan
+// D(c-1) = gamma_c D(c) + (Qbar^T dO)_c, each written over its local term.
+// ---------------------------------------------------------------------------
+template <typename TI>
+__global__ void __launch_bounds__(256) gla_bwd_scan(const BwdArgs<TI> a) {
+  const int bh = blockIdx.y;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= a.dk * a.dv) return;
+  const int i = e / a.dv;
+  const size_t st = (size_t)a.dk * a.dv;
+  float* sx = a.sx + (size_t)bh * a.NC * st + e;
+  float* dd = a.dd + (size_t)bh * a.NC * st + e;
+  const float* gam = a.gamma + (size_t)bh * a.NC * a.dk + i;
+  // Batches of kBatch chunks: the loads of a batch are issued before its dependent
+  // chain of fmas, so the scan is not one memory latency per chunk.
+  constexpr int kBatch = 8;
+  float S = 0.f;
+  for (int c0 = 0; c0 < a.NC; c0 += kBatch) {
+    float x[kBatch], gm[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int c = c0 + u;
+      x[u] = c < a.NC ? sx[c * st] : 0.f;
+      gm[u] = c < a.NC ? gam[(size_t)c * a.dk] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int c = c0 + u;
+      if (c < a.NC) {
+        S = fmaf(gm[u], S, x[u]);
+        sx[c * st] = S;
+      }
+    }
+  }
+  float D = 0.f;
+  for (int c0 = a.NC - 1; c0 >= 0; c0 -= kBatch) {
+    float x[kBatch], gm[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int c = c0 - u;
+      x[u] = c >= 0 ? dd[c * st] : 0.f;
+      gm[u] = c >= 0 ? gam[(size_t)c * a.dk] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int c = c0 - u;
+      if (c >= 0) {
+        dd[c * st] = D;
+        D = fmaf(gm[u], D, x[u]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 3: per-chunk gradients.
+// ---------------------------------------------------------------------------
+template <typename TI>
+__device__ __forceinline__ int64_t row_off(const BwdArgs<TI>& a, int b, int h, int f, int d) {
+  return (((int64_t)b * a.g.T + base_pos_to_token(a.g, f)) * a.H + h) * d;
+}
+
+// Exact token-by-token reverse sweep through one chunk, from the state entering it
+// (S_in(c) = the scan's S_in written for chunk c-1, zero for the first chunk) and the
+// gradient D(c) leaving it.  Thread-private recomputation of S_{r-1} for every
+// position keeps every state element's recurrence in one thread.
+template <typename TI, int MC>
+__device__ void chunk_serial_bwd(const BwdArgs<TI>& a, float* sQ, float* sK, float* sU, float* sV, float* sO,
+                                 float* sGg, float* sW, int c, int b, int h, int f0) {
+  const int pk = a.dk + 4, pv = a.dv + 4;
+  const int64_t cid = (int64_t)blockIdx.y * a.NC + c;
+  const size_t st = (size_t)a.dk * a.dv;
+  const float* sin = c > 0 ? a.sx + (cid - 1) * st : nullptr;
+  const float* dd = a.dd + cid * st;
+  for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+    const int i = e / a.dv, j = e - i * a.dv;
+    sGg[i * pv + j] = dd[e];
+  }
+  for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
+    const int r = e / a.dk, i = e - r * a.dk;
+    sU[r * pk + i] = expf(sU[r * pk + i]);  // alpha
+  }
+  __syncthreads();
+  for (int step = MC - 1; step >= 0; --step) {
+    const int r = a.g.reverse ? (MC - 1 - step) : step;
+    const int f = f0 + r;
+    // S_{r-1}: the state before this position, recomputed from S_in; and the
+    // gradient of S_r picks up q_r^T dO_r.
+    for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+      const int i = e / a.dv, j = e - i * a.dv;
+      float w = sin ? sin[e] : 0.f;
+      for (int s2 = 0; s2 < step; ++s2) {
+        const int r2 = a.g.reverse ? (MC - 1 - s2) : s2;
+        w = fmaf(sU[r2 * pk + i], w, sK[r2 * pk + i] * sV[r2 * pv + j]);
+      }
+      sW[i * pv + j] = w;
+      sGg[i * pv + j] = fmaf(sQ[r * pk + i], sO[r * pv + j], sGg[i * pv + j]);
+    }
+    __syncthreads();
+    const bool real = f >= 0 && f < a.g.T;
+    for (int i = threadIdx.x; i < a.dk; i += NT) {
+      const float al = sU[r * pk + i], ki = sK[r * pk + i];
+      float gq = 0.f, gk = 0.f, gl = 0.f;
+      for (int j = 0; j < a.dv; ++j) {
+        const float sr = fmaf(al, sW[i * pv + j], ki * sV[r * pv + j]);  // S_r
+        gq = fmaf(sO[r * pv + j], sr, gq);
+        gk = fmaf(sGg[i * pv + j], sV[r * pv + j], gk);
+        gl = fmaf(sGg[i * pv + j], sW[i * pv + j], gl);
+      }
+      if (real) {
+        const int64_t o = row_off(a, b, h, f, a.dk);
+        store1(a.dq + o + i, gq);
+        store1(a.dk_out + o + i, gk);
+        a.dla[o + i] = al * gl;
+      }
+    }
+    for (int j = threadIdx.x; j < a.dv; j += NT) {
+      float gv = 0.f;
+      for (int i = 0; i < a.dk; ++i) gv = fmaf(sK[r * pk + i], sGg[i * pv + j], gv);
+      if (real) store1(a.dv_out + row_off(a, b, h, f, a.dv) + j, gv);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+      const int i = e / a.dv, j = e - i * a.dv;
+      sGg[i * pv + j] *= sU[r * pk + i];
+    }
+    __syncthreads();
+  }
+}
+
+template <typename TI, int MC>
+__global__ void __launch_bounds__(NT) gla_bwd_chunk(const BwdArgs<TI> a) {
+  extern __shared__ float4 smem_f4[];
+  float* smem = reinterpret_cast<float*>(smem_f4);
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int pk = a.dk + 4, pv = a.dv + 4, pa = MC + 1;
+  float* sQ = smem;
+  float* sK = sQ + MC * pk;
+  float* sU = sK + MC * pk;
+  float* sV = sU + MC * pk;
+  float* sO = sV + MC * pv;
+  float* sTot = sO + MC * pv;
+  float* sCarry = sTot + 128;
+  float* rest = sCarry + 128;
+  // factorised form
+  float* sDB = rest;                 // [MC][pk]   Q~ dQ~ - K^ dK^
+  float* sS = sDB + MC * pk;         // [dk][pv]   G, then D
+  float* sA = sS + a.dk * pv;        // [MC][MC+1] mask(dO V^T)
+  float* sP = sA + MC * pa;          // [MC][MC+1] mask(Q~ K^T)
+  // token-by-token form
+  float* sGg = rest;                 // [dk][pv]
+  float* sW = sGg + a.dk * pv;       // [dk][pv]
+
+  const int f0 = chunk_first_base_pos(a.g, c, MC);
+  stage<MC>(sQ, a.q, a.dk, a.g, f0, b, h, a.H);
+  stage<MC>(sK, a.k, a.dk, a.g, f0, b, h, a.H);
+  stage<MC>(sU, a.la, a.dk, a.g, f0, b, h, a.H);
+  stage<MC>(sV, a.v, a.dv, a.g, f0, b, h, a.H);
+  stage<MC>(sO, a.dout, a.dv, a.g, f0, b, h, a.H);
+  const int64_t cid = (int64_t)bh * a.NC + c;
+  __syncthreads();
+  if (a.flags[cid]) {
+    chunk_serial_bwd<TI, MC>(a, sQ, sK, sU, sV, sO, sGg, sW, c, b, h, f0);
+    return;
+  }
+  suffix_sums<MC>(sU, sTot, a.dk, a.g.reverse);
+  __syncthreads();
+  const size_t st = (size_t)a.dk * a.dv;
+  const float* sin = c > 0 ? a.sx + (cid - 1) * st : nullptr;
+  for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
+    const int r = e / a.dk, i = e - r * a.dk;
+    const float u = sU[r * pk + i];
+    sQ[r * pk + i] *= expf(-u);
+    sK[r * pk + i] *= expf(u);
+  }
+  for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+    const int i = e / a.dv, j = e - i * a.dv;
+    sS[i * pv + j] = sin ? expf(sTot[i]) * sin[e] : 0.f;
+  }
+  __syncthreads();
+  const bool rev = a.g.reverse;
+  for (int e = threadIdx.x; e < MC * MC; e += NT) {
+    const int r = e / MC, s = e - r * MC;
+    const bool keep = rev ? (s >= r) : (s <= r);
+    float x = 0.f, y = 0.f;
+    if (keep) {
+      for (int j = 0; j < a.dv; ++j) x = fmaf(sO[r * pv + j], sV[s * pv + j], x);
+      for (int i = 0; i < a.dk; ++i) y = fmaf(sQ[r * pk + i], sK[s * pk + i], y);
+    }
+    sA[r * pa + s] = x;
+    sP[r * pa + s] = y;
+  }
+  __syncthreads();
+  // dQ~ = dO G^T + A K^
+  for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
+    const int r = e / a.dk, i = e - r * a.dk;
+    float acc = 0.f;
+    for (int j = 0; j < a.dv; ++j) acc = fmaf(sO[r * pv + j], sS[i * pv + j], acc);
+    for (int s = 0; s < MC; ++s) acc = fmaf(sA[r * pa + s], sK[s * pk + i], acc);
+    sDB[r * pk + i] = sQ[r * pk + i] * acc;
+    const int f = f0 + r;
+    if (f >= 0 && f < a.g.T) store1(a.dq + row_off(a, b, h, f, a.dk) + i, expf(-sU[r * pk + i]) * acc);
+  }
+  __syncthreads();
+  const float* dd = a.dd + cid * st;
+  for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+    const int i = e / a.dv, j = e - i * a.dv;
+    sS[i * pv + j] = dd[e];
+  }
+  __syncthreads();
+  // dK^ = A^T Q~ + V D^T
+  for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
+    const int s = e / a.dk, i = e - s * a.dk;
+    float acc = 0.f;
+    for (int r = 0; r < MC; ++r) acc = fmaf(sA[r * pa + s], sQ[r * pk + i], acc);
+    for (int j = 0; j < a.dv; ++j) acc = fmaf(sV[s * pv + j], sS[i * pv + j], acc);
+    sDB[s * pk + i] = fmaf(-sK[s * pk + i], acc, sDB[s * pk + i]);
+    const int f = f0 + s;
+    if (f >= 0 && f < a.g.T) store1(a.dk_out + row_off(a, b, h, f, a.dk) + i, expf(sU[s * pk + i]) * acc);
+  }
+  // dV = P^T dO + K^ D
+  for (int e = threadIdx.x; e < MC * a.dv; e += NT) {
+    const int s = e / a.dv, j = e - s * a.dv;
+    float acc = 0.f;
+    for (int r = 0; r < MC; ++r) acc = fmaf(sP[r * pa + s], sO[r * pv + j], acc);
+    for (int i = 0; i < a.dk; ++i) acc = fmaf(sK[s * pk + i], sS[i * pv + j], acc);
+    const int f = f0 + s;
+    if (f >= 0 && f < a.g.T) store1(a.dv_out + row_off(a, b, h, f, a.dv) + j, acc);
+  }
+  // gradient of a gate at the chunk's end: sum_j D[i][j] S_in(c+1)[i][j]
+  {
+    const float* sout = a.sx + cid * st;
+    for (int i = threadIdx.x; i < a.dk; i += NT) {
+      float acc = 0.f;
+      for (int j = 0; j < a.dv; ++j) acc = fmaf(sS[i * pv + j], sout[(size_t)i * a.dv + j], acc);
+      sCarry[i] = acc;
+    }
+  }
+  __syncthreads();
+  // dlog_alpha_r = carry + sum of db over the chunk's positions at or after r
+  for (int i = threadIdx.x; i < a.dk; i += NT) {
+    float acc = sCarry[i];
+    for (int step = MC - 1; step >= 0; --step) {
+      const int r = rev ? (MC - 1 - step) : step;
+      acc += sDB[r * pk + i];
+      const int f = f0 + r;
+      if (f >= 0 && f < a.g.T) a.dla[row_off(a, b, h, f, a.dk) + i] = acc;
+    }
+  }
+}
+
+size_t rup(size_t x, size_t m) { return (x + m - 1) / m * m; }
+
+int chunk_rows(const GlaShape& s) { return (s.dk > 80 || s.dv > 80) ? 32 : 64; }
+
+template <int MC>
+size_t smem_local(const GlaShape& s) {
+  return ((size_t)MC * (s.dk + 4) * 3 + (size_t)MC * (s.dv + 4) * 2 + 128) * sizeof(float);
+}
+
+template <int MC>
+size_t smem_chunk(const GlaShape& s) {
+  const size_t pk = s.dk + 4, pv = s.dv + 4;
+  const size_t tiles = MC * pk * 3 + MC * pv * 2 + 256;
+  const size_t fact = MC * pk + s.dk * pv + 2 * (size_t)MC * (MC + 1);
+  const size_t serial = 2 * (size_t)s.dk * pv;
+  return (tiles + (fact > serial ? fact : serial)) * sizeof(float);
+}
+
+template <typename TI, int MC>
+cudaError_t launch_bwd(const BwdArgs<TI>& a, const GlaShape& s, cudaStream_t st) {
+  const size_t s1 = smem_local<MC>(s), s3 = smem_chunk<MC>(s);
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(gla_bwd_local<TI, MC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1)) !=
+      cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(gla_bwd_chunk<TI, MC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3)) !=
+      cudaSuccess)
+    return e;
+  const dim3 grid(a.NC, s.B * s.H);
+  gla_bwd_local<TI, MC><<<grid, NT, s1, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  gla_bwd_scan<TI><<<dim3((s.dk * s.dv + 255) / 256, s.B * s.H), 256, 0, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  gla_bwd_chunk<TI, MC><<<grid, NT, s3, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename TI>
+cudaError_t run_bwd(const void* q, const void* k, const void* v, const float* la, const void* dout, void* dq,
+                    void* dk, void* dv, float* dla, const GlaShape& s, void* workspace, cudaStream_t st) {
+  BwdArgs<TI> a;
+  a.q = static_cast<const TI*>(q);
+  a.k = static_cast<const TI*>(k);
+  a.v = static_cast<const TI*>(v);
+  a.la = la;
+  a.dout = static_cast<const TI*>(dout);
+  a.dq = static_cast<TI*>(dq);
+  a.dk_out = static_cast<TI*>(dk);
+  a.dv_out = static_cast<TI*>(dv);
+  a.dla = dla;
+  a.H = s.H;
+  a.dk = s.dk;
+  a.dv = s.dv;
+  const int MC = chunk_rows(s);
+  a.NC = (s.T() + MC - 1) / MC;
+  a.g = make_geom(s.Hg, s.Wg, s.dir);
+  const size_t BH = (size_t)s.B * s.H;
+  const size_t big = rup(BH * a.NC * s.dk * s.dv * 4, 256);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.sx = reinterpret_cast<float*>(ws);
+  a.dd = reinterpret_cast<float*>(ws + big);
+  a.gamma = reinterpret_cast<float*>(ws + 2 * big);
+  a.flags = reinterpret_cast<int*>(ws + 2 * big + rup(BH * a.NC * s.dk * 4, 256));
+  return MC == 64 ? launch_bwd<TI, 64>(a, s, st) : launch_bwd<TI, 32>(a, s, st);
+}
+
+}  // namespace
+
+size_t gla_bwd_workspace_bytes(const GlaShape& s) {
+  const int MC = chunk_rows(s);
+  const size_t NC = (size_t)(s.T() + MC - 1) / MC;
+  const size_t BH = (size_t)s.B * s.H;
+  return rup(BH * NC * s.dk * s.dv * 4, 256) * 2 + rup(BH * NC * s.dk * 4, 256) + rup(BH * NC * 4, 256);
+}
+
+cudaError_t gla_bwd_launch(const void* q, const void* k, const void* v, const float* la, const void* dout, void* dq,
+                           void* dk, void* dv, float* dla, const GlaShape& s, int bf16, void* workspace,
+                           cudaStream_t st) {
+  return bf16 ? run_bwd<__nv_bfloat16>(q, k, v, la, dout, dq, dk, dv, dla, s, workspace, st)
+              : run_bwd<float>(q, k, v, la, dout, dq, dk, dv, dla, s, workspace, st);
+}
+
+}  // namespace dig

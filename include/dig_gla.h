@@ -127,6 +127,39 @@ int gla_fwd_f32_noalloc(const float* q, const float* k, const float* v, const fl
                         int Hgrid, int Wgrid, int dk, int dv, int dir, float* out, cudaStream_t stream);
 
 /*
+ * gla_bwd -- gradients of the chunk-wise GLA forward, bf16 q, k, v, dout.
+ *
+ * DiG is trained like DiT (DiG paper notes, "损失函数 / 训练策略"), so every GLA
+ * layer is differentiated; the notes' complexity claim for the chunk-wise form
+ * ("硬件友好的效率设计") covers training.  Given dout = dL/dout for
+ * out = gla_fwd(q, k, v, log_alpha, ..., dir), writes the exact gradients of L
+ * (through the same recurrence, the same scan order and S_0 = 0):
+ *   dq, dk        [B][T][H][dk] bf16        dv [B][T][H][dv] bf16
+ *   dlog_alpha    [B][T][H][dk] fp32        (d L / d log_alpha, not d alpha)
+ * from q, k [B][T][H][dk] bf16, v and dout [B][T][H][dv] bf16 and log_alpha
+ * [B][T][H][dk] fp32, all at canonical token positions.
+ * Arithmetic: every product and sum in fp32 on CUDA cores, from the bf16 inputs
+ * widened exactly; dq, dk, dv rounded to nearest even on the store.  Chunks of 64
+ * scan positions (32 when dk or dv exceeds 80); a chunk whose gates decay by more
+ * than e^80 inside it (a full reset, -inf) is differentiated token by token (exact,
+ * slower).  Growth gates whose product exceeds e^80 inside a chunk record
+ * GLA_ERR_RANGE.  Shapes, dims, directions and errors as gla_fwd; no output may
+ * overlap an input or another output.  Workspace as gla_fwd (2 * B*H*ceil(T/64) *
+ * dk*dv fp32 values, plus per-chunk gates).
+ */
+int gla_bwd(const void* q, const void* k, const void* v, const float* log_alpha, const void* dout, int B, int H,
+            int Hgrid, int Wgrid, int dk, int dv, int dir, void* dq, void* dk_out, void* dv_out, float* dlog_alpha,
+            cudaStream_t stream);
+
+/*
+ * gla_bwd_f32 -- gla_bwd with fp32 q, k, v, dout, dq, dk, dv (same arithmetic, no
+ * rounding on the store).
+ */
+int gla_bwd_f32(const float* q, const float* k, const float* v, const float* log_alpha, const float* dout, int B,
+                int H, int Hgrid, int Wgrid, int dk, int dv, int dir, float* dq, float* dk_out, float* dv_out,
+                float* dlog_alpha, cudaStream_t stream);
+
+/*
  * srem_reorient -- SREM's change of scan direction as an explicit row gather
  * (DiG paper notes, SREM: the block ends by transposing the 2D token matrix and
  * flipping the sequence, both O(T) operations; DiG Block step (5)).

@@ -141,3 +141,16 @@ def conv_weight_device(C: int, seed: int, device, noise: float = 0.01):
     w = torch.randn((C, 3, 3), generator=gen, dtype=torch.float32, device=device) * noise
     w[:, 1, 1] += 1.0
     return w.contiguous()
+
+
+def gla_dout(w: Workload, seed: int = 0, scale: float | None = None):
+    """An upstream gradient d out [B][T][H][dv] for the GLA backward: N(0,1) * 1/sqrt(dv)
+    in the workload's dtype, from its own generator stream (seed + 3_000_003) so that it
+    does not change the forward inputs of the same seed."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(seed) + 3_000_003)
+    s = (1.0 / math.sqrt(w.dv)) if scale is None else scale
+    d = torch.randn((w.B, w.T, w.H, w.dv), generator=gen, dtype=torch.float32) * s
+    if w.dtype == "bf16":
+        d = d.to(torch.bfloat16)
+    return d.contiguous()
