@@ -12,6 +12,7 @@
  *    right-to-left, top-to-bottom, bottom-to-top -- obtained by transposing the
  *    2D token matrix and flipping the sequence.  Numbering follows the order in
  *    which the notes list them: 0 = L->R, 1 = R->L, 2 = T->B, 3 = B->T.
+ *    Codes 4..11 are the eight zigzag orders (see zigzag_order).
  *    oracle_scan_order() materialises the order literally: it builds the grid of
  *    raster token ids, transposes it for 2/3, flattens row by row, and reverses
  *    the flattened sequence for 1/3.
@@ -74,9 +75,53 @@
 /* ------------------------------------------------------------------------- */
 /* Scan order: the raster token id visited at each scan position.             */
 /* ------------------------------------------------------------------------- */
+/*
+ * Zigzag orders (ZigMa notes, "Zigzag 扫描方案": within every line the scan turns
+ * back, a snake path, so that tokens adjacent in the sequence are adjacent in the
+ * grid; eight schemes S_0..S_7 that differ in horizontal / vertical orientation,
+ * start and direction).  Scheme j: lines are the grid's rows for j < 4 and its
+ * columns (the transposed grid's rows) for j >= 4; the lines are visited first to
+ * last when bit 1 of j is clear and last to first when it is set; the first visited
+ * line is walked from its first entry when bit 0 of j is clear and from its last
+ * entry when it is set, and every following line in the opposite direction of the
+ * one before.  scan order code dir = 4 + j.
+ */
+static int zigzag_order(int j, int Hgrid, int Wgrid, int64_t *order)
+{
+    const int64_t T = (int64_t)Hgrid * Wgrid;
+    int64_t *grid = (int64_t *)malloc(sizeof(int64_t) * T);
+    if (!grid) return ORACLE_NOMEM;
+    int nl, len; /* lines and their length, in `grid` laid out line by line */
+    if (j < 4) {
+        nl = Hgrid;
+        len = Wgrid;
+        for (int y = 0; y < Hgrid; ++y)
+            for (int x = 0; x < Wgrid; ++x) grid[(int64_t)y * Wgrid + x] = (int64_t)y * Wgrid + x;
+    } else {
+        nl = Wgrid;
+        len = Hgrid;
+        for (int y = 0; y < Hgrid; ++y)
+            for (int x = 0; x < Wgrid; ++x) grid[(int64_t)x * Hgrid + y] = (int64_t)y * Wgrid + x;
+    }
+    const int lines_backwards = (j >> 1) & 1;
+    int from_end = j & 1; /* direction of the line being walked */
+    int64_t n = 0;
+    for (int s = 0; s < nl; ++s) {
+        const int line = lines_backwards ? nl - 1 - s : s;
+        for (int e = 0; e < len; ++e) {
+            const int at = from_end ? len - 1 - e : e;
+            order[n++] = grid[(int64_t)line * len + at];
+        }
+        from_end = !from_end; /* the snake turns back */
+    }
+    free(grid);
+    return ORACLE_OK;
+}
+
 int oracle_scan_order(int dir, int Hgrid, int Wgrid, int64_t *order)
 {
-    if (dir < 0 || dir > 3 || Hgrid <= 0 || Wgrid <= 0 || !order) return ORACLE_BAD_ARG;
+    if (dir < 0 || dir > 11 || Hgrid <= 0 || Wgrid <= 0 || !order) return ORACLE_BAD_ARG;
+    if (dir >= 4) return zigzag_order(dir - 4, Hgrid, Wgrid, order);
     const int64_t T = (int64_t)Hgrid * Wgrid;
 
     /* grid[y][x] holds the raster token id y*Wgrid + x */
@@ -256,7 +301,7 @@ static int gla_common(const double *q, const double *k, const double *v, const d
 {
     if (!q || !k || !v || !log_alpha || !out) return ORACLE_BAD_ARG;
     if (B <= 0 || H <= 0 || Hgrid <= 0 || Wgrid <= 0 || dk <= 0 || dv <= 0) return ORACLE_BAD_ARG;
-    if (dir < 0 || dir > 3) return ORACLE_BAD_ARG;
+    if (dir < 0 || dir > 11) return ORACLE_BAD_ARG;
     const int64_t T = (int64_t)Hgrid * Wgrid;
     const int64_t BH = (int64_t)B * H;
     if (bh_begin < 0) bh_begin = 0;
@@ -439,7 +484,7 @@ static int gla_bwd_common(const double *q, const double *k, const double *v, con
 {
     if (!q || !k || !v || !log_alpha || !dout || !dq || !dk_out || !dv_out || !dla) return ORACLE_BAD_ARG;
     if (B <= 0 || H <= 0 || Hgrid <= 0 || Wgrid <= 0 || dk <= 0 || dv <= 0) return ORACLE_BAD_ARG;
-    if (dir < 0 || dir > 3) return ORACLE_BAD_ARG;
+    if (dir < 0 || dir > 11) return ORACLE_BAD_ARG;
     const int64_t T = (int64_t)Hgrid * Wgrid;
     const int64_t BH = (int64_t)B * H;
     if (bh_begin < 0) bh_begin = 0;
@@ -547,7 +592,7 @@ int oracle_reorient(const void *x, int dir, int inverse, int B, int Hgrid, int W
                     void *y)
 {
     if (!x || !y || B <= 0 || Hgrid <= 0 || Wgrid <= 0 || row_bytes <= 0) return ORACLE_BAD_ARG;
-    if (dir < 0 || dir > 3 || (inverse != 0 && inverse != 1)) return ORACLE_BAD_ARG;
+    if (dir < 0 || dir > 11 || (inverse != 0 && inverse != 1)) return ORACLE_BAD_ARG;
     const int64_t T = (int64_t)Hgrid * Wgrid;
     int64_t *order = (int64_t *)malloc(sizeof(int64_t) * T);
     if (!order) return ORACLE_NOMEM;

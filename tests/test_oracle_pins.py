@@ -26,10 +26,27 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
 # --------------------------------------------------------------------------- helpers
+def zigzag_closed_form(j, Hg, Wg):
+    """Zigzag scheme j (scan order code 4 + j) from index formulas: line k of the walk
+    and position i along it, the line's grid index, the walking direction by parity."""
+    T = Hg * Wg
+    p = np.arange(T)
+    cols = j >= 4
+    nl, ln = (Wg, Hg) if cols else (Hg, Wg)
+    k, i = p // ln, p % ln
+    line = nl - 1 - k if (j >> 1) & 1 else k
+    backwards = (k % 2 == 1) ^ bool(j & 1)
+    at = np.where(backwards, ln - 1 - i, i)
+    y, x = (at, line) if cols else (line, at)
+    return y * Wg + x
+
+
 def closed_form_order(direction, Hg, Wg):
     """Scan position -> raster token id, from closed-form index formulas."""
     T = Hg * Wg
     p = np.arange(T)
+    if direction >= 4:
+        return zigzag_closed_form(direction - 4, Hg, Wg)
     if direction == 0:
         return p
     if direction == 1:
@@ -192,7 +209,9 @@ def test_scan_order_transpose_inverse_nonsquare():
 
 def test_scan_order_rejects_bad_args():
     with pytest.raises(RuntimeError):
-        oracle.scan_order(4, 2, 2)
+        oracle.scan_order(12, 2, 2)      # codes 0..3 SREM, 4..11 zigzag
+    with pytest.raises(RuntimeError):
+        oracle.scan_order(-1, 2, 2)
     with pytest.raises(RuntimeError):
         oracle.scan_order(0, 0, 2)
 
