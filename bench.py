@@ -20,7 +20,8 @@ Beside the headline (rank 0, unless --no-extras): a long window of c4 GLA launch
 (at least one second of device time, its own clock samples, median per direction),
 and the 28-layer DiG-XL/2 stack at 2048 resolution (gla_fwd -> dwconv3x3 ->
 srem_reorient per layer, fresh inputs per layer, dir = layer % 4), timed with and
-without the reorientation; and the GLA backward (gla_bwd) on c4 and c2.  Under torchrun (N > 1) every rank runs its own replica of the
+without the reorientation; the GLA backward (gla_bwd) on c4 and c2; and the c4 GLA forward
+along the eight zigzag orders.  Under torchrun (N > 1) every rank runs its own replica of the
 workload (no data exchange: heads and batches are independent), and rank 0
 prints the aggregate.
 """
@@ -382,11 +383,12 @@ def run_gpu(args):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     extra = other_configs(dig, dev, stream, hbm) if (rank == 0 and not args.no_other_configs) else None
     gla_avg_s = statistics.mean(gla_ms) / 1e3
-    window = stack = bwd = None
+    window = stack = bwd = zig = None
     if rank == 0 and not args.no_extras:
         window = long_window(dig, dev, stream, dev_in, outs, hbm, gla_us_hint=gla_avg_s * 1e6)
         stack = stack_c5(dig, dev, stream, hbm)
         bwd = bwd_configs(dig, dev, stream, hbm)
+        zig = zigzag_c4(dig, dev, stream, dev_in, outs, hbm)
     gla_bytes = GLA_BYTES_PER_TOKEN_HEAD * w.token_heads
     achieved = gla_bytes / gla_avg_s / 1e9
     traffic = recorded_traffic()
@@ -430,6 +432,7 @@ def run_gpu(args):
             "gla_long_window_c4": window,
             "stack_c5_28_layers": stack,
             "gla_bwd": bwd,
+            "gla_fwd_zigzag_c4": zig,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -605,6 +608,36 @@ def bwd_configs(dig, dev, stream, hbm, reps=5):
     if status != 0:
         raise RuntimeError(f"device status after the backward: {dig.status_string(status)}")
     return res
+
+
+def zigzag_c4(dig, dev, stream, dev_in, outs, hbm, reps=5):
+    """The c4 GLA forward along the eight zigzag orders (codes 4..11): each call gathers
+    q, k, v, log_alpha into the scan order, scans, and scatters the output back.  Median
+    of `reps` calls per scheme; the fraction is on the GLA's own algorithmic bytes (the
+    arranged copies are extra traffic)."""
+    w = WORKLOAD
+    q, k, v, la = dev_in[0]
+    per = []
+    for j in range(8):
+        dig.gla_fwd(q, k, v, la, w.Hgrid, w.Wgrid, 4 + j, out=outs[0])
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dig.gla_fwd(q, k, v, la, w.Hgrid, w.Wgrid, 4 + j, out=outs[0])
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        per.append(statistics.median(ts))
+    status = dig.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after the zigzag orders: {dig.status_string(status)}")
+    us = statistics.mean(per)
+    gla_bytes = GLA_BYTES_PER_TOKEN_HEAD * w.token_heads
+    copy_bytes = 2 * (2 * (2 * w.dk + w.dv) + 4 * w.dk + 2 * w.dv) * w.token_heads  # gathers + scatter
+    return {"us_per_scheme": per, "tokens_heads_per_s": w.token_heads / (us / 1e6),
+            "frac_of_hbm": gla_bytes / (us / 1e6) / 1e9 / hbm,
+            "bytes_moved_incl_arranging": gla_bytes + copy_bytes}
 
 
 def per_kernel(w, gla_ms, conv_ms, reor_ms, hbm):

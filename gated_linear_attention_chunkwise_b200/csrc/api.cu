@@ -17,6 +17,9 @@
 
 namespace dig {
 
+// Scan order codes: 0..3 the SREM orders, 4..11 the zigzag schemes.
+constexpr int kDirLast = 11;
+
 // First error a kernel recorded on this device (GLA_OK while none).
 __device__ int g_device_status = 0;
 
@@ -57,7 +60,7 @@ int validate_gla(const void* q, const void* k, const void* v, const void* la, co
                  int Hg, int Wg, int dk, int dv, int dir, size_t elt) {
   if (!q || !k || !v || !la || !out) return GLA_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || Hg <= 0 || Wg <= 0 || dk <= 0 || dv <= 0) return GLA_ERR_INVALID_ARG;
-  if (dir < 0 || dir > 3) return GLA_ERR_INVALID_ARG;
+  if (dir < 0 || dir > kDirLast) return GLA_ERR_INVALID_ARG;
   if (dk % 8 || dv % 8 || dk > 128 || dv > 128) return GLA_ERR_UNSUPPORTED;
   const int64_t T = (int64_t)Hg * Wg;
   if (T > (int64_t)1 << 30) return GLA_ERR_UNSUPPORTED;
@@ -202,14 +205,68 @@ struct GlaCall {
   GlaShape s;
   cudaStream_t st;
 };
-cudaError_t run_tc(void* ws, void* ctx) {
-  const GlaCall* c = static_cast<const GlaCall*>(ctx);
-  return dig::gla_ws_forward(c->q, c->k, c->v, c->la, c->out, c->s, ws, c->st);
+// ---- zigzag orders (codes 4..11) ------------------------------------------------
+// They run as the ZigMa notes write a layer ("异构逐层扫描": arrange the tokens into
+// the scheme's order, scan, arrange the result back): the token rows of every input
+// are gathered into scan order, the left-to-right scan runs over them as one line of
+// T tokens, and the output rows are scattered back to canonical positions.  The four
+// SREM orders need no copies: their order lives in the kernels' address math.
+size_t rup256(size_t x) { return (x + 255) / 256 * 256; }
+GlaShape line_shape(const GlaShape& s) { return GlaShape{s.B, s.H, 1, s.T(), s.dk, s.dv, 0}; }
+size_t rows_of(const GlaShape& s) { return (size_t)s.B * s.T() * s.H; }
+
+// Scratch of the arranged copies: n_k tensors of width dk and n_v of width dv in the
+// call's element type, and n_l fp32 tensors of width dk.
+size_t arranged_bytes(const GlaShape& s, size_t elt, int n_k, int n_v, int n_l) {
+  const size_t r = rows_of(s);
+  return n_k * rup256(r * s.dk * elt) + n_v * rup256(r * s.dv * elt) + n_l * rup256(r * s.dk * 4);
 }
-cudaError_t run_f32(void* ws, void* ctx) {
-  const GlaCall* c = static_cast<const GlaCall*>(ctx);
-  return dig::gla_f32_forward(static_cast<const float*>(c->q), static_cast<const float*>(c->k),
-                              static_cast<const float*>(c->v), c->la, static_cast<float*>(c->out), c->s, ws, c->st);
+
+// Gathers (inverse 0) or scatters (inverse 1) whole token rows [B][T][H*d].
+cudaError_t arrange(const void* x, void* y, const GlaShape& s, size_t row_bytes, int inverse, cudaStream_t st) {
+  return dig::srem_reorient_launch(x, y, s.dir, inverse, s.B, s.Hg, s.Wg, row_bytes, st);
+}
+
+cudaError_t fwd_line(const GlaCall& c, size_t elt, void* ws,
+                     cudaError_t (*fwd)(const GlaCall&, void*)) {
+  if (c.s.dir < 4) return fwd(c, ws);
+  const GlaShape& s = c.s;
+  const size_t r = rows_of(s);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  void* q2 = p;
+  p += rup256(r * s.dk * elt);
+  void* k2 = p;
+  p += rup256(r * s.dk * elt);
+  void* v2 = p;
+  p += rup256(r * s.dv * elt);
+  void* o2 = p;
+  p += rup256(r * s.dv * elt);
+  float* l2 = reinterpret_cast<float*>(p);
+  p += rup256(r * s.dk * 4);
+  const size_t rk = (size_t)s.H * s.dk * elt, rv = (size_t)s.H * s.dv * elt, rl = (size_t)s.H * s.dk * 4;
+  cudaError_t e;
+  if ((e = arrange(c.q, q2, s, rk, 0, c.st)) != cudaSuccess || (e = arrange(c.k, k2, s, rk, 0, c.st)) != cudaSuccess ||
+      (e = arrange(c.v, v2, s, rv, 0, c.st)) != cudaSuccess || (e = arrange(c.la, l2, s, rl, 0, c.st)) != cudaSuccess)
+    return e;
+  const GlaCall c2{q2, k2, v2, l2, o2, line_shape(s), c.st};
+  if ((e = fwd(c2, p)) != cudaSuccess) return e;
+  return arrange(o2, c.out, s, rv, 1, c.st);
+}
+
+cudaError_t tc_fwd(const GlaCall& c, void* ws) { return dig::gla_ws_forward(c.q, c.k, c.v, c.la, c.out, c.s, ws, c.st); }
+cudaError_t f32_fwd(const GlaCall& c, void* ws) {
+  return dig::gla_f32_forward(static_cast<const float*>(c.q), static_cast<const float*>(c.k),
+                              static_cast<const float*>(c.v), c.la, static_cast<float*>(c.out), c.s, ws, c.st);
+}
+cudaError_t run_tc(void* ws, void* ctx) { return fwd_line(*static_cast<const GlaCall*>(ctx), 2, ws, tc_fwd); }
+cudaError_t run_f32(void* ws, void* ctx) { return fwd_line(*static_cast<const GlaCall*>(ctx), 4, ws, f32_fwd); }
+size_t tc_ws_bytes(const GlaShape& s) {
+  return s.dir < 4 ? dig::gla_ws_workspace_bytes(s)
+                   : arranged_bytes(s, 2, 2, 2, 1) + dig::gla_ws_workspace_bytes(line_shape(s));
+}
+size_t f32_ws_bytes(const GlaShape& s) {
+  return s.dir < 4 ? dig::gla_f32_workspace_bytes(s)
+                   : arranged_bytes(s, 4, 2, 2, 1) + dig::gla_f32_workspace_bytes(line_shape(s));
 }
 struct BwdCall {
   const void *q, *k, *v;
@@ -223,8 +280,38 @@ struct BwdCall {
 };
 cudaError_t run_bwd(void* ws, void* ctx) {
   const BwdCall* c = static_cast<const BwdCall*>(ctx);
-  return dig::gla_bwd_launch(c->q, c->k, c->v, c->la, c->dout, c->dq, c->dk, c->dv, c->dla, c->s, c->bf16, ws,
-                             c->st);
+  const GlaShape& s = c->s;
+  if (s.dir < 4)
+    return dig::gla_bwd_launch(c->q, c->k, c->v, c->la, c->dout, c->dq, c->dk, c->dv, c->dla, s, c->bf16, ws, c->st);
+  // zigzag: arrange the five inputs, differentiate the line, scatter the four gradients
+  const size_t elt = c->bf16 ? 2 : 4;
+  const size_t r = rows_of(s);
+  const size_t nk = rup256(r * s.dk * elt), nv = rup256(r * s.dv * elt), nl = rup256(r * s.dk * 4);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  void *q2 = p, *k2 = p + nk, *dq2 = p + 2 * nk, *dk2 = p + 3 * nk;
+  p += 4 * nk;
+  void *v2 = p, *do2 = p + nv, *dv2 = p + 2 * nv;
+  p += 3 * nv;
+  float* l2 = reinterpret_cast<float*>(p);
+  float* dl2 = reinterpret_cast<float*>(p + nl);
+  p += 2 * nl;
+  const size_t rk = (size_t)s.H * s.dk * elt, rv = (size_t)s.H * s.dv * elt, rl = (size_t)s.H * s.dk * 4;
+  cudaError_t e;
+  if ((e = arrange(c->q, q2, s, rk, 0, c->st)) != cudaSuccess || (e = arrange(c->k, k2, s, rk, 0, c->st)) != cudaSuccess ||
+      (e = arrange(c->v, v2, s, rv, 0, c->st)) != cudaSuccess || (e = arrange(c->la, l2, s, rl, 0, c->st)) != cudaSuccess ||
+      (e = arrange(c->dout, do2, s, rv, 0, c->st)) != cudaSuccess)
+    return e;
+  if ((e = dig::gla_bwd_launch(q2, k2, v2, l2, do2, dq2, dk2, dv2, dl2, line_shape(s), c->bf16, p, c->st)) !=
+      cudaSuccess)
+    return e;
+  if ((e = arrange(dq2, c->dq, s, rk, 1, c->st)) != cudaSuccess || (e = arrange(dk2, c->dk, s, rk, 1, c->st)) != cudaSuccess ||
+      (e = arrange(dv2, c->dv, s, rv, 1, c->st)) != cudaSuccess)
+    return e;
+  return arrange(dl2, c->dla, s, rl, 1, c->st);
+}
+size_t bwd_ws_bytes(const GlaShape& s, int bf16) {
+  return s.dir < 4 ? dig::gla_bwd_workspace_bytes(s)
+                   : arranged_bytes(s, bf16 ? 2 : 4, 4, 3, 2) + dig::gla_bwd_workspace_bytes(line_shape(s));
 }
 int gla_bwd_common(const void* q, const void* k, const void* v, const float* la, const void* dout, int B, int H,
                    int Hgrid, int Wgrid, int dk, int dv, int dir, void* dq, void* dk_out, void* dv_out, float* dla,
@@ -234,7 +321,7 @@ int gla_bwd_common(const void* q, const void* k, const void* v, const float* la,
   if (rc != GLA_OK) return rc;
   if ((rc = dig::check_device()) != GLA_OK) return rc;
   BwdCall c{q, k, v, la, dout, dq, dk_out, dv_out, dla, GlaShape{B, H, Hgrid, Wgrid, dk, dv, dir}, bf16, stream};
-  return dig::run_with_workspace(dig::gla_bwd_workspace_bytes(c.s), stream, run_bwd, &c);
+  return dig::run_with_workspace(bwd_ws_bytes(c.s, bf16), stream, run_bwd, &c);
 }
 }  // namespace
 
@@ -260,7 +347,7 @@ int gla_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
   if (rc != GLA_OK) return rc;
   if ((rc = dig::check_device()) != GLA_OK) return rc;
   GlaCall c{q, k, v, log_alpha, out, GlaShape{B, H, Hgrid, Wgrid, dk, dv, dir}, stream};
-  return dig::run_with_workspace(dig::gla_ws_workspace_bytes(c.s), stream, run_tc, &c);
+  return dig::run_with_workspace(tc_ws_bytes(c.s), stream, run_tc, &c);
 }
 
 int gla_fwd_f32(const float* q, const float* k, const float* v, const float* log_alpha, int B, int H, int Hgrid,
@@ -269,7 +356,7 @@ int gla_fwd_f32(const float* q, const float* k, const float* v, const float* log
   if (rc != GLA_OK) return rc;
   if ((rc = dig::check_device()) != GLA_OK) return rc;
   GlaCall c{q, k, v, log_alpha, out, GlaShape{B, H, Hgrid, Wgrid, dk, dv, dir}, stream};
-  return dig::run_with_workspace(dig::gla_f32_workspace_bytes(c.s), stream, run_f32, &c);
+  return dig::run_with_workspace(f32_ws_bytes(c.s), stream, run_f32, &c);
 }
 
 int srem_reorient(const void* x, int dir, int inverse, int B, int Hgrid, int Wgrid, int C, int dtype, void* y,
@@ -277,7 +364,7 @@ int srem_reorient(const void* x, int dir, int inverse, int B, int Hgrid, int Wgr
   size_t rb = 0;
   int rc = dig::validate_grid(x, y, B, Hgrid, Wgrid, C, dtype, &rb);
   if (rc != GLA_OK) return rc;
-  if (dir < 0 || dir > 3 || (inverse != 0 && inverse != 1)) return GLA_ERR_INVALID_ARG;
+  if (dir < 0 || dir > dig::kDirLast || (inverse != 0 && inverse != 1)) return GLA_ERR_INVALID_ARG;
   if ((rc = dig::check_device()) != GLA_OK) return rc;
   return dig::srem_reorient_launch(x, y, dir, inverse, B, Hgrid, Wgrid, rb, stream) == cudaSuccess ? GLA_OK
                                                                                                    : GLA_ERR_CUDA;

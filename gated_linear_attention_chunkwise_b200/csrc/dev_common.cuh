@@ -215,6 +215,7 @@ struct ScanGeom {
   int T, Hg, Wg;
   int column_base;  // 1 for T->B / B->T
   int reverse;      // 1 for R->L / B->T
+  int zigzag;       // 0: one of the four SREM orders; 1 + j: zigzag scheme j (codes 4 + j)
 };
 
 __host__ __device__ __forceinline__ ScanGeom make_geom(int Hg, int Wg, int dir) {
@@ -222,9 +223,25 @@ __host__ __device__ __forceinline__ ScanGeom make_geom(int Hg, int Wg, int dir) 
   g.T = Hg * Wg;
   g.Hg = Hg;
   g.Wg = Wg;
-  g.column_base = (dir >= 2) ? 1 : 0;
+  g.zigzag = dir >= 4 ? dir - 3 : 0;
+  g.column_base = (dir == 2 || dir == 3) ? 1 : 0;
   g.reverse = (dir == 1 || dir == 3) ? 1 : 0;
   return g;
+}
+
+// Zigzag scheme j (ZigMa notes, "Zigzag 扫描方案": the scan turns back at the end of
+// every line): lines are rows for j < 4, columns for j >= 4; bit 1 of j visits the
+// lines last to first, bit 0 walks the first line from its end; every line reverses
+// the direction of the one before.  Token visited at scan position p.
+__device__ __forceinline__ int zigzag_token(const ScanGeom& g, int p) {
+  const int j = g.zigzag - 1;
+  const bool cols = j >= 4;
+  const int len = cols ? g.Hg : g.Wg, nl = cols ? g.Wg : g.Hg;
+  const int k = p / len, i = p - k * len;
+  const int line = (j & 2) ? nl - 1 - k : k;
+  const bool back = ((k & 1) != 0) != ((j & 1) != 0);
+  const int at = back ? len - 1 - i : i;
+  return cols ? at * g.Wg + line : line * g.Wg + at;
 }
 
 __device__ __forceinline__ int base_pos_to_token(const ScanGeom& g, int f) {
@@ -236,6 +253,7 @@ __device__ __forceinline__ int base_pos_to_token(const ScanGeom& g, int f) {
 
 // Token visited at scan position p.
 __device__ __forceinline__ int scan_pos_to_token(const ScanGeom& g, int p) {
+  if (g.zigzag) return zigzag_token(g, p);
   const int f = g.reverse ? (g.T - 1 - p) : p;
   return base_pos_to_token(g, f);
 }

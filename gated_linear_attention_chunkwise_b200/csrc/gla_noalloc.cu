@@ -65,6 +65,7 @@ extern "C" int gla_fwd_f32_noalloc(const float* q, const float* k, const float* 
                                    cudaStream_t stream) {
   int rc = dig::validate_gla(q, k, v, log_alpha, out, B, H, Hgrid, Wgrid, dk, dv, dir, 4);
   if (rc != GLA_OK) return rc;
+  if (dir > 3) return GLA_ERR_UNSUPPORTED;  // zigzag orders need arranged copies beyond the fixed scratch
   if ((rc = dig::check_device()) != GLA_OK) return rc;
   const dig::GlaShape s{B, H, Hgrid, Wgrid, dk, dv, dir};
   if (dig::gla_f32_workspace_bytes(s) > (size_t)DIG_GLA_NOALLOC_SCRATCH_BYTES) return GLA_ERR_UNSUPPORTED;

@@ -20,6 +20,17 @@
  *      GLA_DIR_R2L = 1: reversed raster order t = T-1-p
  *      GLA_DIR_T2B = 2: column-major order t = (p mod Hgrid)*Wgrid + p div Hgrid
  *      GLA_DIR_B2T = 3: reversed column-major order
+ *    Codes 4..11 are the eight zigzag orders S_0..S_7 of the ZigMa notes ("Zigzag
+ *    扫描方案": the scan turns back at the end of every line, so neighbours in the
+ *    sequence are neighbours in the grid), code GLA_DIR_ZIGZAG0 + j for scheme j:
+ *    lines are the grid's rows for j < 4 and its columns for j >= 4; bit 1 of j
+ *    visits the lines last to first; bit 0 walks the first line from its end; each
+ *    line then reverses the direction of the one before.  The GLA entry points run
+ *    them as the notes write a layer: the token rows are gathered into the scan order
+ *    (srem_reorient), scanned left to right as one line of T tokens, and the results
+ *    scattered back, so a zigzag call also moves every input and output through HBM
+ *    once more and needs that much more workspace.  gla_fwd_f32_noalloc takes codes
+ *    0..3 only.
  *  - Every call is asynchronous on `stream` (0 = the legacy default stream) and
  *    never synchronises it.  Argument errors are returned synchronously before
  *    anything is launched; a launch failure returns GLA_ERR_CUDA.  Conditions a
@@ -51,7 +62,7 @@ typedef enum {
                                (device status only; the output is not valid) */
 } gla_status_t;
 
-enum { GLA_DIR_L2R = 0, GLA_DIR_R2L = 1, GLA_DIR_T2B = 2, GLA_DIR_B2T = 3 };
+enum { GLA_DIR_L2R = 0, GLA_DIR_R2L = 1, GLA_DIR_T2B = 2, GLA_DIR_B2T = 3, GLA_DIR_ZIGZAG0 = 4 };
 enum { GLA_BF16 = 0, GLA_F32 = 1 };
 
 /*
@@ -70,7 +81,7 @@ enum { GLA_BF16 = 0, GLA_F32 = 1 };
  *   q, k       [B][T][H][dk] bf16        log_alpha [B][T][H][dk] fp32
  *   v          [B][T][H][dv] bf16        out       [B][T][H][dv] bf16 (written)
  *   dk, dv     multiples of 8 in [8, 128]
- *   dir        GLA_DIR_*
+ *   dir        GLA_DIR_* (0..3), or GLA_DIR_ZIGZAG0 + j (j = 0..7)
  * Arithmetic: tensor-core products of bf16 operands with fp32 accumulation; the
  * chunk state and all gate arithmetic are fp32; out is rounded to nearest even.
  * Gates: any log_alpha <= 0 is handled, -inf (a full reset of the channel)
@@ -165,7 +176,7 @@ int gla_bwd_f32(const float* q, const float* k, const float* v, const float* log
  * flipping the sequence, both O(T) operations; DiG Block step (5)).
  *   inverse = 0:  y[b][p][:] = x[b][order_dir(p)][:]   (canonical -> scan order)
  *   inverse = 1:  y[b][order_dir(p)][:] = x[b][p][:]   (scan order -> canonical)
- * where order_dir(p) is the raster token visited at scan position p.
+ * where order_dir(p) is the raster token visited at scan position p (dir 0..11).
  *   x, y   [B][T][C] elements of `dtype` (GLA_BF16 or GLA_F32); C*sizeof(elt)
  *          must be a multiple of 16 bytes.  Bit-exact copy.  y must not overlap x.
  */

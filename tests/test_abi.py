@@ -69,7 +69,7 @@ def test_gla_argument_validation(lib, fn):
     assert gla(lib, out=None, fn=fn) == INVALID
     assert gla(lib, B=0, fn=fn) == INVALID
     assert gla(lib, Hg=-1, fn=fn) == INVALID
-    assert gla(lib, d=4, fn=fn) == INVALID
+    assert gla(lib, d=12, fn=fn) == INVALID     # codes 0..3 SREM orders, 4..11 zigzag
     assert gla(lib, d=-1, fn=fn) == INVALID
     assert gla(lib, dk=60, fn=fn) == UNSUPPORTED       # not a multiple of 8
     assert gla(lib, dv=136, fn=fn) == UNSUPPORTED      # above 128
@@ -93,7 +93,7 @@ def test_gla_valid_arguments_reach_the_device_check(lib):
 def test_grid_op_validation(lib):
     X, Y, W = 0x100000, 0x900000, 0x1100000
     assert lib.srem_reorient(None, 0, 0, 1, 4, 4, 64, 0, Y, None) == INVALID
-    assert lib.srem_reorient(X, 4, 0, 1, 4, 4, 64, 0, Y, None) == INVALID
+    assert lib.srem_reorient(X, 12, 0, 1, 4, 4, 64, 0, Y, None) == INVALID
     assert lib.srem_reorient(X, 0, 2, 1, 4, 4, 64, 0, Y, None) == INVALID
     assert lib.srem_reorient(X, 0, 0, 1, 4, 4, 64, 7, Y, None) == INVALID
     assert lib.srem_reorient(X, 0, 0, 1, 4, 4, 12, 0, Y, None) == ALIGN     # 24-byte rows
