@@ -18,6 +18,9 @@ Functions and the passages they follow (see the C file for the full statement):
   gla_bwd          the exact gradient of that recurrence (dq, dk, dv, dlog_alpha
                    for a given d out), as reverse-mode differentiation of its steps
                    in reverse scan order (DiG notes, training like DiT).
+  gla_norm_fwd     the diffusers draft's normalised variant (page 4,
+                   "gated_linear_attention"): elu+1 features, sigmoid(q*k) gate,
+                   gated denominator, output divided by max(denominator, eps).
   dwconv3x3        DiG notes, SREM / DiG Block step (4): 3x3 depthwise conv on
                    the 2D token grid, zero padding.
   reorient         DiG notes, SREM: the O(T) transpose + flip as a row gather.
@@ -66,6 +69,10 @@ def _load():
         lib.oracle_gla_bwd_planted.argtypes = [dp] * 5 + [c_int] * 7 + [dp] * 4 + [c_int]
         lib.oracle_gla_bwd.restype = c_int
         lib.oracle_gla_bwd_planted.restype = c_int
+        lib.oracle_gla_norm_fwd.argtypes = [dp] * 3 + [c_int] * 7 + [ctypes.c_double, dp, c_int]
+        lib.oracle_gla_norm_fwd_planted.argtypes = [dp] * 3 + [c_int] * 7 + [ctypes.c_double, dp, c_int]
+        lib.oracle_gla_norm_fwd.restype = c_int
+        lib.oracle_gla_norm_fwd_planted.restype = c_int
         lib.oracle_dwconv3x3.argtypes = [dp, dp, c_int, c_int, c_int, c_int, dp, c_int]
         lib.oracle_reorient.argtypes = [ctypes.c_void_p, c_int, c_int, c_int, c_int, c_int, c_i64,
                                         ctypes.c_void_p]
@@ -158,6 +165,23 @@ def gla_bwd(q, k, v, log_alpha, dout, Hgrid: int, Wgrid: int, direction: int, nt
         lo, hi = (0, -1) if heads is None else (int(heads[0]), int(heads[1]))
         _check(lib.oracle_gla_bwd(*args, nthreads, lo, hi), "gla_bwd")
     return gq, gk, gv, gl
+
+
+def gla_norm_fwd(q, k, v, Hgrid: int, Wgrid: int, direction: int, eps: float = 1e-6, nthreads: int = 0,
+                 planted: int = 0) -> np.ndarray:
+    """fp64 normalised variant.  q, k: [B,T,H,dk]; v: [B,T,H,dv] -> out [B,T,H,dv]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    assert T == Hgrid * Wgrid and k.shape == q.shape and v.shape[:3] == q.shape[:3]
+    out = np.zeros((B, T, H, dv), dtype=np.float64)
+    lib = _load()
+    args = (_dp(q), _dp(k), _dp(v), B, H, Hgrid, Wgrid, dk, dv, direction, float(eps), _dp(out))
+    if planted:
+        _check(lib.oracle_gla_norm_fwd_planted(*args, planted), "gla_norm_fwd_planted")
+    else:
+        _check(lib.oracle_gla_norm_fwd(*args, nthreads), "gla_norm_fwd")
+    return out
 
 
 def dwconv3x3(x, w, nthreads: int = 0) -> np.ndarray:

@@ -56,9 +56,19 @@
  *    The forward states S_p of the head are kept (T * dk * dv values) so that the
  *    reverse sweep reads them exactly.
  *
+ *  - Normalised variant (the diffusers draft, page 4, `gated_linear_attention`): the
+ *    features are elu(x) + 1 of q and k, the per-key-channel forget gate is
+ *    sigmoid(q * k) of the raw q and k, and a gated denominator runs beside the
+ *    state.  Per (batch, head), from S = 0 and z = 0, at every scan position:
+ *        S <- Diag(g_t) S + phi(k_t)^T v_t,   z <- g_t * z + phi(k_t)
+ *        o_t = (phi(q_t) S) / max(phi(q_t) . z, eps)
+ *    all in fp64 (the draft computes in fp32 or wider).  Same scan orders and
+ *    canonical output positions as the forward above.
+ *
  * Planted mistakes: oracle_gla_fwd_planted() runs the same recurrence with one
  * deliberate error selected by `planted` (1..7), and oracle_gla_bwd_planted()
- * the backward sweep with one of 1..6.  Tests use them to show that the oracle's
+ * the backward sweep with one of 1..6, oracle_gla_norm_fwd_planted() the
+ * normalised variant with one of 1..5.  Tests use them to show that the oracle's
  * pins catch each kind of mistake; the method itself is planted == 0.
  */
 #include <math.h>
@@ -544,6 +554,112 @@ int oracle_gla_bwd_planted(const double *q, const double *k, const double *v, co
     if (planted < 0 || planted > 6) return ORACLE_BAD_ARG;
     return gla_bwd_common(q, k, v, log_alpha, dout, B, H, Hgrid, Wgrid, dk, dv, dir, dq, dk_out, dv_out, dla, 1,
                           planted, 0, -1);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Normalised variant (elu+1 features, sigmoid(q*k) gate, gated denominator). */
+/* ------------------------------------------------------------------------- */
+typedef struct {
+    const double *q, *k, *v;
+    double *out;
+    const int64_t *order;
+    int64_t T;
+    int H, dk, dv;
+    double eps;
+    int planted; /* 0 = the method; 1..5 = a planted mistake (tests only) */
+    int status;
+} norm_ctx;
+
+static double feature(double x, int planted)
+{
+    if (planted == 1) return x > 0.0 ? x : 0.0; /* planted: relu in place of elu + 1 */
+    return x > 0.0 ? x + 1.0 : exp(x);         /* elu(x) + 1 = e^x for x <= 0 */
+}
+
+static void norm_head(void *vctx, int64_t bh)
+{
+    norm_ctx *c = (norm_ctx *)vctx;
+    const int64_t b = bh / c->H, h = bh % c->H;
+    const int dk = c->dk, dv = c->dv;
+    double *S = (double *)calloc((size_t)dk * dv, sizeof(double));
+    double *z = (double *)calloc((size_t)dk, sizeof(double));
+    double *fq = (double *)malloc(sizeof(double) * dk);
+    double *fk = (double *)malloc(sizeof(double) * dk);
+    if (!S || !z || !fq || !fk) {
+        free(S);
+        free(z);
+        free(fq);
+        free(fk);
+        c->status = ORACLE_NOMEM;
+        return;
+    }
+    for (int64_t p = 0; p < c->T; ++p) {
+        const int64_t t = c->order[p];
+        const double *qt = c->q + tok_off(b, t, h, c->T, c->H, dk);
+        const double *kt = c->k + tok_off(b, t, h, c->T, c->H, dk);
+        const double *vt = c->v + tok_off(b, t, h, c->T, c->H, dv);
+        double *ot = c->out + tok_off(b, t, h, c->T, c->H, dv);
+        for (int i = 0; i < dk; ++i) {
+            fq[i] = feature(qt[i], c->planted);
+            fk[i] = feature(kt[i], c->planted);
+        }
+        for (int i = 0; i < dk; ++i) {
+            /* the gate: sigmoid of the raw q * k (planted 2: of the features' product) */
+            const double x = (c->planted == 2) ? fq[i] * fk[i] : qt[i] * kt[i];
+            const double g = 1.0 / (1.0 + exp(-x));
+            for (int j = 0; j < dv; ++j) S[(int64_t)i * dv + j] = g * S[(int64_t)i * dv + j] + fk[i] * vt[j];
+            /* planted 3: the denominator is not gated */
+            z[i] = (c->planted == 3 ? 1.0 : g) * z[i] + fk[i];
+        }
+        double den = 0.0;
+        for (int i = 0; i < dk; ++i) den += fq[i] * z[i];
+        if (c->planted != 4 && den < c->eps) den = c->eps; /* planted 4: no clamp */
+        for (int j = 0; j < dv; ++j) {
+            double num = 0.0;
+            for (int i = 0; i < dk; ++i) num += fq[i] * S[(int64_t)i * dv + j];
+            ot[j] = (c->planted == 5) ? num : num / den; /* planted 5: not normalised */
+        }
+    }
+    free(S);
+    free(z);
+    free(fq);
+    free(fk);
+}
+
+static int norm_common(const double *q, const double *k, const double *v, int B, int H, int Hgrid, int Wgrid,
+                       int dk, int dv, int dir, double eps, double *out, int nthreads, int planted)
+{
+    if (!q || !k || !v || !out || B <= 0 || H <= 0 || Hgrid <= 0 || Wgrid <= 0 || dk <= 0 || dv <= 0)
+        return ORACLE_BAD_ARG;
+    if (dir < 0 || dir > 11 || !(eps > 0.0)) return ORACLE_BAD_ARG;
+    const int64_t T = (int64_t)Hgrid * Wgrid;
+    int64_t *order = (int64_t *)malloc(sizeof(int64_t) * T);
+    if (!order) return ORACLE_NOMEM;
+    int rc = oracle_scan_order(dir, Hgrid, Wgrid, order);
+    if (rc != ORACLE_OK) {
+        free(order);
+        return rc;
+    }
+    norm_ctx c = {q, k, v, out, order, T, H, dk, dv, eps, planted, ORACLE_OK};
+    int used = run_pool(norm_head, &c, (int64_t)B * H, nthreads);
+    free(order);
+    if (c.status != ORACLE_OK) return c.status;
+    return used;
+}
+
+/* q, k: [B][T][H][dk]; v, out: [B][T][H][dv].  Returns the threads used or an error. */
+int oracle_gla_norm_fwd(const double *q, const double *k, const double *v, int B, int H, int Hgrid, int Wgrid,
+                        int dk, int dv, int dir, double eps, double *out, int nthreads)
+{
+    return norm_common(q, k, v, B, H, Hgrid, Wgrid, dk, dv, dir, eps, out, nthreads, 0);
+}
+
+/* The normalised variant with one deliberate mistake (tests of the pins only). */
+int oracle_gla_norm_fwd_planted(const double *q, const double *k, const double *v, int B, int H, int Hgrid,
+                                int Wgrid, int dk, int dv, int dir, double eps, double *out, int planted)
+{
+    if (planted < 0 || planted > 5) return ORACLE_BAD_ARG;
+    return norm_common(q, k, v, B, H, Hgrid, Wgrid, dk, dv, dir, eps, out, 1, planted);
 }
 
 /* ------------------------------------------------------------------------- */
