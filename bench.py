@@ -20,8 +20,8 @@ Beside the headline (rank 0, unless --no-extras): a long window of c4 GLA launch
 (at least one second of device time, its own clock samples, median per direction),
 and the 28-layer DiG-XL/2 stack at 2048 resolution (gla_fwd -> dwconv3x3 ->
 srem_reorient per layer, fresh inputs per layer, dir = layer % 4), timed with and
-without the reorientation; the GLA backward (gla_bwd) on c4 and c2; and the c4 GLA forward
-along the eight zigzag orders.  Under torchrun (N > 1) every rank runs its own replica of the
+without the reorientation; the GLA backward (gla_bwd) on c4 and c2; the c4 GLA forward
+along the eight zigzag orders; and the draft's normalised variant on c4 and c2.  Under torchrun (N > 1) every rank runs its own replica of the
 workload (no data exchange: heads and batches are independent), and rank 0
 prints the aggregate.
 """
@@ -383,12 +383,13 @@ def run_gpu(args):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     extra = other_configs(dig, dev, stream, hbm) if (rank == 0 and not args.no_other_configs) else None
     gla_avg_s = statistics.mean(gla_ms) / 1e3
-    window = stack = bwd = zig = None
+    window = stack = bwd = zig = nrm = None
     if rank == 0 and not args.no_extras:
         window = long_window(dig, dev, stream, dev_in, outs, hbm, gla_us_hint=gla_avg_s * 1e6)
         stack = stack_c5(dig, dev, stream, hbm)
         bwd = bwd_configs(dig, dev, stream, hbm)
         zig = zigzag_c4(dig, dev, stream, dev_in, outs, hbm)
+        nrm = norm_configs(dig, dev, stream, hbm)
     gla_bytes = GLA_BYTES_PER_TOKEN_HEAD * w.token_heads
     achieved = gla_bytes / gla_avg_s / 1e9
     traffic = recorded_traffic()
@@ -433,6 +434,7 @@ def run_gpu(args):
             "stack_c5_28_layers": stack,
             "gla_bwd": bwd,
             "gla_fwd_zigzag_c4": zig,
+            "gla_norm_fwd": nrm,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -638,6 +640,39 @@ def zigzag_c4(dig, dev, stream, dev_in, outs, hbm, reps=5):
     return {"us_per_scheme": per, "tokens_heads_per_s": w.token_heads / (us / 1e6),
             "frac_of_hbm": gla_bytes / (us / 1e6) / 1e9 / hbm,
             "bytes_moved_incl_arranging": gla_bytes + copy_bytes}
+
+
+def norm_configs(dig, dev, stream, hbm, reps=5):
+    """The normalised variant (gla_norm_fwd, bf16) on c4 and c2: median of `reps` calls
+    per direction; the fraction is on its algorithmic bytes (q, k, v read once, out
+    written once, bf16)."""
+    res = {}
+    for name in ("c4", "c2"):
+        cw = workloads.WORKLOADS[name]
+        q, k, v, _ = [t.to(dev) for t in workloads.gla_inputs(cw, seed=13)]
+        per_th = 2 * (2 * cw.dk + cw.dv) + 2 * cw.dv
+        per_dir = []
+        for d in range(4):
+            dig.gla_norm_fwd(q, k, v, cw.Hgrid, cw.Wgrid, d)
+            ts = []
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                dig.gla_norm_fwd(q, k, v, cw.Hgrid, cw.Wgrid, d)
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                ts.append(e0.elapsed_time(e1) * 1e3)
+            per_dir.append(statistics.median(ts))
+        us = statistics.mean(per_dir)
+        res[name] = {"workload": cw.name, "kernels": "prep + fp32 chunk-wise GLA (3) + post",
+                     "us_per_dir": per_dir, "bytes_per_token_head": per_th,
+                     "tokens_heads_per_s": cw.token_heads / (us / 1e6),
+                     "frac_of_hbm": per_th * cw.token_heads / (us / 1e6) / 1e9 / hbm}
+        del q, k, v
+    status = dig.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after the normalised variant: {dig.status_string(status)}")
+    return res
 
 
 def per_kernel(w, gla_ms, conv_ms, reor_ms, hbm):

@@ -7,7 +7,8 @@ the library's sm_100a kernels; there is no CPU or PyTorch fallback, and
 importing this package fails if the library has not been built
 (`python gated_linear_attention_chunkwise_b200/build.py`).
 
-Names follow the C ABI: gla_fwd, gla_fwd_f32, gla_bwd, gla_bwd_f32, srem_reorient, dwconv3x3,
+Names follow the C ABI: gla_fwd, gla_fwd_f32, gla_bwd, gla_bwd_f32, gla_norm_fwd,
+gla_norm_fwd_f32, srem_reorient, dwconv3x3,
 device_status (dig_gla_device_status), status_string (dig_gla_status_string).
 """
 from __future__ import annotations
@@ -17,7 +18,7 @@ import os
 
 import torch
 
-__all__ = ["gla_fwd", "gla_fwd_f32", "gla_bwd", "gla_bwd_f32", "srem_reorient", "dwconv3x3", "device_status", "status_string",
+__all__ = ["gla_fwd", "gla_fwd_f32", "gla_bwd", "gla_bwd_f32", "gla_norm_fwd", "gla_norm_fwd_f32", "srem_reorient", "dwconv3x3", "device_status", "status_string",
            "GlaError", "lib", "LIB_PATH", "DIR_L2R", "DIR_R2L", "DIR_T2B", "DIR_B2T"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdig_gla.so")
@@ -31,6 +32,8 @@ _lib.gla_fwd.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 7 + [_vp, _u]
 _lib.gla_fwd_f32.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 7 + [_vp, _u]
 _lib.gla_bwd.argtypes = [_vp] * 5 + [_i] * 7 + [_vp] * 4 + [_u]
 _lib.gla_bwd_f32.argtypes = [_vp] * 5 + [_i] * 7 + [_vp] * 4 + [_u]
+_lib.gla_norm_fwd.argtypes = [_vp] * 3 + [_i] * 7 + [ctypes.c_float, _vp, _u]
+_lib.gla_norm_fwd_f32.argtypes = [_vp] * 3 + [_i] * 7 + [ctypes.c_float, _vp, _u]
 _lib.srem_reorient.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _i, _vp, _u]
 _lib.dwconv3x3.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _u]
 _lib.dig_gla_device_status.argtypes = [_u]
@@ -40,7 +43,8 @@ _lib.dig_gla_release.argtypes = []
 _lib.dig_gla_release.restype = None
 _lib.dig_gla_test_skip_items.argtypes = [_i]
 _lib.dig_gla_test_skip_items.restype = None
-for _fn in (_lib.gla_fwd, _lib.gla_fwd_f32, _lib.gla_bwd, _lib.gla_bwd_f32, _lib.srem_reorient, _lib.dwconv3x3, _lib.dig_gla_device_status):
+for _fn in (_lib.gla_fwd, _lib.gla_fwd_f32, _lib.gla_bwd, _lib.gla_bwd_f32, _lib.gla_norm_fwd, _lib.gla_norm_fwd_f32,
+            _lib.srem_reorient, _lib.dwconv3x3, _lib.dig_gla_device_status):
     _fn.restype = ctypes.c_int
 
 DIR_L2R, DIR_R2L, DIR_T2B, DIR_B2T = 0, 1, 2, 3
@@ -150,6 +154,39 @@ def gla_bwd(q, k, v, log_alpha, dout, Hgrid: int, Wgrid: int, direction: int, st
 def gla_bwd_f32(q, k, v, log_alpha, dout, Hgrid: int, Wgrid: int, direction: int, stream=None):
     """fp32 GLA backward (see include/dig_gla.h, gla_bwd_f32).  Returns (dq, dk, dv, dlog_alpha) fp32."""
     return _bwd("gla_bwd_f32", q, k, v, log_alpha, dout, Hgrid, Wgrid, direction, stream, torch.float32)
+
+
+def _norm(fn_name, q, k, v, Hgrid, Wgrid, direction, eps, out, stream, dtype):
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, dtype, dev)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise ValueError("expected q, k [B,T,H,dk] and v [B,T,H,dv]")
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    if T != Hgrid * Wgrid:
+        raise ValueError(f"T={T} does not match the grid {Hgrid}x{Wgrid}")
+    if out is None:
+        out = torch.empty_like(v)
+    else:
+        _need(out, "out", dtype, dev)
+        if out.shape != v.shape:
+            raise ValueError("out must be [B,T,H,dv]")
+    with torch.cuda.device(dev):
+        rc = getattr(_lib, fn_name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, Hgrid, Wgrid, dk, dv,
+                                    int(direction), float(eps), out.data_ptr(), _stream_handle(dev, stream))
+    _check(fn_name, rc)
+    return out
+
+
+def gla_norm_fwd(q, k, v, Hgrid: int, Wgrid: int, direction: int, eps: float = 1e-6, out=None, stream=None):
+    """The draft's normalised GLA, bf16 (see include/dig_gla.h, gla_norm_fwd)."""
+    return _norm("gla_norm_fwd", q, k, v, Hgrid, Wgrid, direction, eps, out, stream, torch.bfloat16)
+
+
+def gla_norm_fwd_f32(q, k, v, Hgrid: int, Wgrid: int, direction: int, eps: float = 1e-6, out=None, stream=None):
+    """The draft's normalised GLA, fp32 (see include/dig_gla.h, gla_norm_fwd_f32)."""
+    return _norm("gla_norm_fwd_f32", q, k, v, Hgrid, Wgrid, direction, eps, out, stream, torch.float32)
 
 
 def _grid_dtype(x: torch.Tensor) -> int:

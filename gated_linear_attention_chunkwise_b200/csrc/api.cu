@@ -100,6 +100,24 @@ int validate_gla_bwd(const void* q, const void* k, const void* v, const void* la
   return GLA_OK;
 }
 
+// The normalised variant: q, k, v, out as the forward's (no log_alpha: the gate comes
+// from q and k); eps positive; dv at most 120, leaving room for the ones column.
+int validate_gla_norm(const void* q, const void* k, const void* v, const void* out, int B, int H, int Hg, int Wg,
+                      int dk, int dv, int dir, float eps, size_t elt) {
+  if (!q || !k || !v || !out) return GLA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Hg <= 0 || Wg <= 0 || dk <= 0 || dv <= 0) return GLA_ERR_INVALID_ARG;
+  if (dir < 0 || dir > kDirLast || !(eps > 0.f)) return GLA_ERR_INVALID_ARG;
+  if (dk % 8 || dv % 8 || dk > 128 || dv > 120) return GLA_ERR_UNSUPPORTED;
+  const int64_t T = (int64_t)Hg * Wg;
+  if (T > (int64_t)1 << 30 || (int64_t)B * H > 65535) return GLA_ERR_UNSUPPORTED;
+  const int64_t rows = (int64_t)B * T * H;
+  if (rows > ((int64_t)1 << 40) / 128) return GLA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GLA_ERR_ALIGNMENT;
+  const size_t nq = (size_t)rows * dk * elt, nv = (size_t)rows * dv * elt;
+  if (overlaps(out, nv, q, nq) || overlaps(out, nv, k, nq) || overlaps(out, nv, v, nv)) return GLA_ERR_INVALID_ARG;
+  return GLA_OK;
+}
+
 namespace {
 
 int validate_grid(const void* x, const void* y, int B, int Hg, int Wg, int C, int dtype, size_t* row_bytes) {
@@ -323,9 +341,67 @@ int gla_bwd_common(const void* q, const void* k, const void* v, const float* la,
   BwdCall c{q, k, v, la, dout, dq, dk_out, dv_out, dla, GlaShape{B, H, Hgrid, Wgrid, dk, dv, dir}, bf16, stream};
   return dig::run_with_workspace(bwd_ws_bytes(c.s, bf16), stream, run_bwd, &c);
 }
+// ---- the normalised variant ----------------------------------------------------
+struct NormCall {
+  const void *q, *k, *v;
+  void* out;
+  GlaShape s;
+  float eps;
+  int bf16;
+  cudaStream_t st;
+};
+int norm_width(int dv) { return dv + 8; }  // v, a column of ones, zero padding to a multiple of 8
+size_t norm_ws_bytes(const GlaShape& s) {
+  const size_t r = rows_of(s);
+  const GlaShape sa{s.B, s.H, s.Hg, s.Wg, s.dk, norm_width(s.dv), s.dir};
+  return 3 * rup256(r * s.dk * 4) + 2 * rup256(r * sa.dv * 4) + f32_ws_bytes(sa);
+}
+cudaError_t run_norm(void* ws, void* ctx) {
+  const NormCall* c = static_cast<const NormCall*>(ctx);
+  const GlaShape& s = c->s;
+  const int dva = norm_width(s.dv);
+  const GlaShape sa{s.B, s.H, s.Hg, s.Wg, s.dk, dva, s.dir};
+  const size_t r = rows_of(s);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  float* fq = reinterpret_cast<float*>(p);
+  p += rup256(r * s.dk * 4);
+  float* fk = reinterpret_cast<float*>(p);
+  p += rup256(r * s.dk * 4);
+  float* la = reinterpret_cast<float*>(p);
+  p += rup256(r * s.dk * 4);
+  float* va = reinterpret_cast<float*>(p);
+  p += rup256(r * dva * 4);
+  float* oa = reinterpret_cast<float*>(p);
+  p += rup256(r * dva * 4);
+  cudaError_t e;
+  if ((e = dig::gla_norm_prep_launch(c->q, c->k, c->v, fq, fk, la, va, (int64_t)r, s.dk, s.dv, dva, c->bf16, c->st)) !=
+      cudaSuccess)
+    return e;
+  const GlaCall g{fq, fk, va, la, oa, sa, c->st};
+  if ((e = fwd_line(g, 4, p, f32_fwd)) != cudaSuccess) return e;
+  return dig::gla_norm_post_launch(oa, c->out, (int64_t)r, s.dv, dva, c->eps, c->bf16, c->st);
+}
+int gla_norm_common(const void* q, const void* k, const void* v, int B, int H, int Hgrid, int Wgrid, int dk, int dv,
+                    int dir, float eps, void* out, int bf16, cudaStream_t stream) {
+  int rc = dig::validate_gla_norm(q, k, v, out, B, H, Hgrid, Wgrid, dk, dv, dir, eps, bf16 ? 2 : 4);
+  if (rc != GLA_OK) return rc;
+  if ((rc = dig::check_device()) != GLA_OK) return rc;
+  NormCall c{q, k, v, out, GlaShape{B, H, Hgrid, Wgrid, dk, dv, dir}, eps, bf16, stream};
+  return dig::run_with_workspace(norm_ws_bytes(c.s), stream, run_norm, &c);
+}
 }  // namespace
 
 extern "C" {
+
+int gla_norm_fwd(const void* q, const void* k, const void* v, int B, int H, int Hgrid, int Wgrid, int dk, int dv,
+                 int dir, float eps, void* out, cudaStream_t stream) {
+  return gla_norm_common(q, k, v, B, H, Hgrid, Wgrid, dk, dv, dir, eps, out, 1, stream);
+}
+
+int gla_norm_fwd_f32(const float* q, const float* k, const float* v, int B, int H, int Hgrid, int Wgrid, int dk,
+                     int dv, int dir, float eps, float* out, cudaStream_t stream) {
+  return gla_norm_common(q, k, v, B, H, Hgrid, Wgrid, dk, dv, dir, eps, out, 0, stream);
+}
 
 int gla_bwd(const void* q, const void* k, const void* v, const float* log_alpha, const void* dout, int B, int H,
             int Hgrid, int Wgrid, int dk, int dv, int dir, void* dq, void* dk_out, void* dv_out, float* dlog_alpha,

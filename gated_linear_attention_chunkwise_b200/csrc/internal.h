@@ -35,6 +35,12 @@ cudaError_t gla_bwd_launch(const void* q, const void* k, const void* v, const fl
                            void* dk, void* dv, float* dla, const GlaShape& s, int bf16, void* workspace,
                            cudaStream_t st);
 
+// ---- normalised variant: element-wise prep / post around the fp32 forward ----
+cudaError_t gla_norm_prep_launch(const void* q, const void* k, const void* v, float* fq, float* fk, float* la,
+                                 float* va, int64_t rows, int dk, int dv, int dva, int bf16, cudaStream_t s);
+cudaError_t gla_norm_post_launch(const float* oa, void* out, int64_t rows, int dv, int dva, float eps, int bf16,
+                                 cudaStream_t s);
+
 // cuTensorMapEncodeTiled, reached through the runtime's driver entry point
 // (nullptr when the driver does not provide it).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

@@ -171,6 +171,28 @@ int gla_bwd_f32(const float* q, const float* k, const float* v, const float* log
                 float* dlog_alpha, cudaStream_t stream);
 
 /*
+ * gla_norm_fwd -- the normalised variant of the diffusers draft (page 4,
+ * `gated_linear_attention`), bf16 q, k, v, out.
+ *
+ * Per (batch, head), over the scan order of `dir`, from S = 0 (dk x dv), z = 0 (dk):
+ *   phi(x) = elu(x) + 1 (x + 1 above zero, e^x otherwise), g_t = sigmoid(q_t * k_t)
+ *   per key channel (of the raw q and k), S <- Diag(g_t) S + phi(k_t)^T v_t,
+ *   z <- g_t * z + phi(k_t),  out_t = (phi(q_t) S) / max(phi(q_t) . z, eps).
+ * q, k [B][T][H][dk] bf16; v, out [B][T][H][dv] bf16; dk multiple of 8 in [8, 128],
+ * dv multiple of 8 in [8, 120]; eps > 0 (the draft uses 1e-6); dir as gla_fwd.
+ * Arithmetic: fp32 throughout (features, gates and the chunk-wise recurrence, whose
+ * denominator is a ones column appended to v); out rounded to nearest even.
+ * Workspace: about (3*dk + 2*(dv+8)) fp32 values per token-head plus the fp32
+ * forward's.  `out` must not overlap an input.  Errors as gla_fwd.
+ */
+int gla_norm_fwd(const void* q, const void* k, const void* v, int B, int H, int Hgrid, int Wgrid, int dk, int dv,
+                 int dir, float eps, void* out, cudaStream_t stream);
+
+/* gla_norm_fwd_f32 -- the same with fp32 q, k, v, out. */
+int gla_norm_fwd_f32(const float* q, const float* k, const float* v, int B, int H, int Hgrid, int Wgrid, int dk,
+                     int dv, int dir, float eps, float* out, cudaStream_t stream);
+
+/*
  * srem_reorient -- SREM's change of scan direction as an explicit row gather
  * (DiG paper notes, SREM: the block ends by transposing the 2D token matrix and
  * flipping the sequence, both O(T) operations; DiG Block step (5)).
