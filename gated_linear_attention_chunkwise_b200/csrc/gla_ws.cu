@@ -832,6 +832,13 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         mbar_arrive(BAR(kBarMail));
         ++jb;
         if (wide) continue;  // evaluated serially by the output group, which frees the stage
+        // The score columns still hold the previous chunk's P, the TMEM A operand of its
+        // P V, and S overwrites them: a later MMA's writes are not ordered after an
+        // earlier MMA's operand reads, so S waits for that P V to complete.
+        if (kb > 0 &&
+            !wait_bar(BAR(kBarBatch + (kb - 1) % a.nO), (uint32_t)(((kb - 1) / a.nO) & 1), abort_flag))
+          break;
+        tc_fence_after();
         // S = Q~ K^T (masked into P by the gate warps meanwhile)
         umma_ss(tbase + kColS, dQ + so, dK + so, id_s, 0u);
 #pragma unroll
