@@ -74,13 +74,17 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float* d) {
 __device__ __forceinline__ void store1(float* p, float x) { *p = x; }
 __device__ __forceinline__ void store1(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
+// Shared-memory tiles have an odd row pitch (d + 1 floats): a warp reading one column
+// of many rows then touches as many banks as rows.
+__host__ __device__ __forceinline__ int pitch_of(int d) { return d + 1; }
+
 // Rows f0 .. f0+MC-1 (base positions) of head h, batch b of a [B][T][H][d] tensor
-// into an fp32 tile with a pitch of d+4 floats; rows outside the sequence are zero.
+// into an fp32 tile of pitch pitch_of(d); rows outside the sequence are zero.
 template <int MC, typename TE>
 __device__ __forceinline__ void stage(float* dst, const TE* src, int d, const ScanGeom& g, int f0, int b, int h,
                                       int H) {
   const int cpr = d / 8;
-  const int pitch = d + 4;
+  const int pitch = pitch_of(d);
   for (int idx = threadIdx.x; idx < MC * cpr; idx += NT) {
     const int r = idx / cpr;
     const int cc = idx - r * cpr;
@@ -88,9 +92,38 @@ __device__ __forceinline__ void stage(float* dst, const TE* src, int d, const Sc
     float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (f >= 0 && f < g.T) load8(src + (((int64_t)b * g.T + base_pos_to_token(g, f)) * H + h) * d + cc * 8, x);
     float* o = dst + r * pitch + cc * 8;
-    *reinterpret_cast<float4*>(o) = make_float4(x[0], x[1], x[2], x[3]);
-    *reinterpret_cast<float4*>(o + 4) = make_float4(x[4], x[5], x[6], x[7]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = x[e];
   }
+}
+
+// A 4 x 8 block of a matrix product in registers:
+//   acc[i][j] += sum_{k < K} A[i*ar + k*ak] * B[k*bk + j*bc]
+// (A and B point at the block's first row / column; the strides pick the layout of
+// each operand).  Twelve shared-memory loads feed 32 multiply-adds.
+__device__ __forceinline__ void mt48(float (&acc)[4][8], const float* A, int ar, int ak, const float* B, int bk,
+                                     int bc, int K) {
+#pragma unroll 2
+  for (int k = 0; k < K; ++k) {
+    float x[4], y[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = A[i * ar];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = B[j * bc];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(x[i], y[j], acc[i][j]);
+    A += ak;
+    B += bk;
+  }
+}
+
+__device__ __forceinline__ void zero48(float (&acc)[4][8]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 }
 
 // Threads i < dk: the log-gate tile becomes, in place, the exclusive suffix sums u
@@ -102,7 +135,7 @@ __device__ __forceinline__ int suffix_sums(float* sU, float* sTot, int dk, int r
   const int i = threadIdx.x;
   int code = 0;
   if (i < dk) {
-    const int pw = dk + 4;
+    const int pw = pitch_of(dk);
     float acc = 0.f, lo = 0.f, hi = 0.f;
     for (int s = 0; s < MC; ++s) {
       const int r = reverse ? s : (MC - 1 - s);
@@ -130,7 +163,7 @@ __global__ void __launch_bounds__(NT) gla_bwd_local(const BwdArgs<TI> a) {
   float* smem = reinterpret_cast<float*>(smem_f4);
   const int c = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
-  const int pk = a.dk + 4, pv = a.dv + 4;
+  const int pk = pitch_of(a.dk), pv = pitch_of(a.dv);
   float* sK = smem;
   float* sQ = sK + MC * pk;
   float* sU = sQ + MC * pk;
@@ -168,16 +201,19 @@ __global__ void __launch_bounds__(NT) gla_bwd_local(const BwdArgs<TI> a) {
   const int64_t cid = (int64_t)bh * a.NC + c;
   float* sx = a.sx + cid * a.dk * a.dv;
   float* dd = a.dd + cid * a.dk * a.dv;
-  for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
-    const int i = e / a.dv, j = e - i * a.dv;
-    float s1 = 0.f, s2 = 0.f;
-#pragma unroll 8
-    for (int r = 0; r < MC; ++r) {
-      s1 = fmaf(sK[r * pk + i], sV[r * pv + j], s1);
-      s2 = fmaf(sQ[r * pk + i], sO[r * pv + j], s2);
-    }
-    sx[e] = s1;
-    dd[e] = s2;
+  // 4 x 8 blocks of K^T V (blocks 0 .. nb-1) and of Qbar^T dO (nb .. 2nb-1), dk x dv.
+  const int ncg = a.dv / 8, nb = (a.dk / 4) * ncg;
+  for (int t = threadIdx.x; t < 2 * nb; t += NT) {
+    const int which = t >= nb, tt = which ? t - nb : t;
+    const int i0 = 4 * (tt / ncg), j0 = 8 * (tt % ncg);
+    float acc[4][8];
+    zero48(acc);
+    mt48(acc, (which ? sQ : sK) + i0, 1, pk, (which ? sO : sV) + j0, pv, 1, MC);
+    float* dst = which ? dd : sx;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dst[(i0 + i) * a.dv + j0 + j] = acc[i][j];
   }
   if (threadIdx.x < a.dk) a.gamma[cid * a.dk + threadIdx.x] = expf(sTot[threadIdx.x]);
   if (threadIdx.x == 0) a.flags[cid] = wide;
@@ -254,7 +290,7 @@ __device__ __forceinline__ int64_t row_off(const BwdArgs<TI>& a, int b, int h, i
 template <typename TI, int MC>
 __device__ void chunk_serial_bwd(const BwdArgs<TI>& a, float* sQ, float* sK, float* sU, float* sV, float* sO,
                                  float* sGg, float* sW, int c, int b, int h, int f0) {
-  const int pk = a.dk + 4, pv = a.dv + 4;
+  const int pk = pitch_of(a.dk), pv = pitch_of(a.dv);
   const int64_t cid = (int64_t)blockIdx.y * a.NC + c;
   const size_t st = (size_t)a.dk * a.dv;
   const float* sin = c > 0 ? a.sx + (cid - 1) * st : nullptr;
@@ -321,7 +357,7 @@ __global__ void __launch_bounds__(NT) gla_bwd_chunk(const BwdArgs<TI> a) {
   float* smem = reinterpret_cast<float*>(smem_f4);
   const int c = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
-  const int pk = a.dk + 4, pv = a.dv + 4, pa = MC + 1;
+  const int pk = pitch_of(a.dk), pv = pitch_of(a.dv), pa = MC + 1;
   float* sQ = smem;
   float* sK = sQ + MC * pk;
   float* sU = sK + MC * pk;
@@ -367,27 +403,62 @@ __global__ void __launch_bounds__(NT) gla_bwd_chunk(const BwdArgs<TI> a) {
   }
   __syncthreads();
   const bool rev = a.g.reverse;
-  for (int e = threadIdx.x; e < MC * MC; e += NT) {
-    const int r = e / MC, s = e - r * MC;
-    const bool keep = rev ? (s >= r) : (s <= r);
-    float x = 0.f, y = 0.f;
-    if (keep) {
-      for (int j = 0; j < a.dv; ++j) x = fmaf(sO[r * pv + j], sV[s * pv + j], x);
-      for (int i = 0; i < a.dk; ++i) y = fmaf(sQ[r * pk + i], sK[s * pk + i], y);
+  // Positions s <= r in scan order are tile rows s <= r, or s >= r for reversed
+  // directions: the nonzero range of a row block of A or P, and of a column block.
+  auto lo_of_rows = [&](int r0) { return rev ? r0 : 0; };
+  auto hi_of_rows = [&](int r0) { return rev ? MC : r0 + 4; };
+  auto lo_of_cols = [&](int s0) { return rev ? 0 : s0; };
+  auto hi_of_cols = [&](int s0) { return rev ? s0 + 4 : MC; };
+  // A = mask(dO V^T) (blocks 0 .. nm-1) and P = mask(Q~ K^T) (nm .. 2nm-1), MC x MC.
+  {
+    const int ncg = MC / 8, nm = (MC / 4) * ncg;
+    for (int t = threadIdx.x; t < 2 * nm; t += NT) {
+      const int which = t >= nm, tt = which ? t - nm : t;
+      const int r0 = 4 * (tt / ncg), s0 = 8 * (tt % ncg);
+      float acc[4][8];
+      zero48(acc);
+      const bool empty = rev ? (s0 + 7 < r0) : (s0 > r0 + 3);
+      if (!empty) {
+        if (which)
+          mt48(acc, sQ + r0 * pk, pk, 1, sK + s0 * pk, 1, pk, a.dk);
+        else
+          mt48(acc, sO + r0 * pv, pv, 1, sV + s0 * pv, 1, pv, a.dv);
+      }
+      float* dst = which ? sP : sA;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int r = r0 + i, s2 = s0 + j;
+          const bool keep = rev ? (s2 >= r) : (s2 <= r);
+          dst[r * pa + s2] = keep ? acc[i][j] : 0.f;
+        }
     }
-    sA[r * pa + s] = x;
-    sP[r * pa + s] = y;
   }
   __syncthreads();
-  // dQ~ = dO G^T + A K^
-  for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
-    const int r = e / a.dk, i = e - r * a.dk;
-    float acc = 0.f;
-    for (int j = 0; j < a.dv; ++j) acc = fmaf(sO[r * pv + j], sS[i * pv + j], acc);
-    for (int s = 0; s < MC; ++s) acc = fmaf(sA[r * pa + s], sK[s * pk + i], acc);
-    sDB[r * pk + i] = sQ[r * pk + i] * acc;
-    const int f = f0 + r;
-    if (f >= 0 && f < a.g.T) store1(a.dq + row_off(a, b, h, f, a.dk) + i, expf(-sU[r * pk + i]) * acc);
+  // dQ~ = dO G^T + A K^ (MC x dk)
+  {
+    const int ncg = a.dk / 8, nb = (MC / 4) * ncg;
+    for (int t = threadIdx.x; t < nb; t += NT) {
+      const int r0 = 4 * (t / ncg), i0 = 8 * (t % ncg);
+      float acc[4][8];
+      zero48(acc);
+      mt48(acc, sO + r0 * pv, pv, 1, sS + i0 * pv, 1, pv, a.dv);
+      const int lo = lo_of_rows(r0), hi = hi_of_rows(r0);
+      mt48(acc, sA + r0 * pa + lo, pa, 1, sK + lo * pk + i0, pk, 1, hi - lo);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = r0 + i, f = f0 + r;
+        const bool real = f >= 0 && f < a.g.T;
+        const int64_t o = real ? row_off(a, b, h, f, a.dk) : 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int ii = i0 + j;
+          sDB[r * pk + ii] = sQ[r * pk + ii] * acc[i][j];
+          if (real) store1(a.dq + o + ii, expf(-sU[r * pk + ii]) * acc[i][j]);
+        }
+      }
+    }
   }
   __syncthreads();
   const float* dd = a.dd + cid * st;
@@ -396,24 +467,44 @@ __global__ void __launch_bounds__(NT) gla_bwd_chunk(const BwdArgs<TI> a) {
     sS[i * pv + j] = dd[e];
   }
   __syncthreads();
-  // dK^ = A^T Q~ + V D^T
-  for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
-    const int s = e / a.dk, i = e - s * a.dk;
-    float acc = 0.f;
-    for (int r = 0; r < MC; ++r) acc = fmaf(sA[r * pa + s], sQ[r * pk + i], acc);
-    for (int j = 0; j < a.dv; ++j) acc = fmaf(sV[s * pv + j], sS[i * pv + j], acc);
-    sDB[s * pk + i] = fmaf(-sK[s * pk + i], acc, sDB[s * pk + i]);
-    const int f = f0 + s;
-    if (f >= 0 && f < a.g.T) store1(a.dk_out + row_off(a, b, h, f, a.dk) + i, expf(sU[s * pk + i]) * acc);
-  }
-  // dV = P^T dO + K^ D
-  for (int e = threadIdx.x; e < MC * a.dv; e += NT) {
-    const int s = e / a.dv, j = e - s * a.dv;
-    float acc = 0.f;
-    for (int r = 0; r < MC; ++r) acc = fmaf(sP[r * pa + s], sO[r * pv + j], acc);
-    for (int i = 0; i < a.dk; ++i) acc = fmaf(sK[s * pk + i], sS[i * pv + j], acc);
-    const int f = f0 + s;
-    if (f >= 0 && f < a.g.T) store1(a.dv_out + row_off(a, b, h, f, a.dv) + j, acc);
+  // dK^ = A^T Q~ + V D^T (MC x dk, blocks 0 .. nk-1) and dV = P^T dO + K^ D (MC x dv,
+  // blocks nk .. nk+nv-1)
+  {
+    const int nck = a.dk / 8, ncv = a.dv / 8, nk = (MC / 4) * nck, nv = (MC / 4) * ncv;
+    for (int t = threadIdx.x; t < nk + nv; t += NT) {
+      const bool isv = t >= nk;
+      const int tt = isv ? t - nk : t;
+      const int nc = isv ? ncv : nck;
+      const int s0 = 4 * (tt / nc), c0 = 8 * (tt % nc);
+      const int lo = lo_of_cols(s0), hi = hi_of_cols(s0);
+      float acc[4][8];
+      zero48(acc);
+      if (!isv) {
+        mt48(acc, sA + lo * pa + s0, 1, pa, sQ + lo * pk + c0, pk, 1, hi - lo);
+        mt48(acc, sV + s0 * pv, pv, 1, sS + c0 * pv, 1, pv, a.dv);
+      } else {
+        mt48(acc, sP + lo * pa + s0, 1, pa, sO + lo * pv + c0, pv, 1, hi - lo);
+        mt48(acc, sK + s0 * pk, pk, 1, sS + c0, pv, 1, a.dk);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int s2 = s0 + i, f = f0 + s2;
+        const bool real = f >= 0 && f < a.g.T;
+        if (!isv) {
+          const int64_t o = real ? row_off(a, b, h, f, a.dk) : 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int ii = c0 + j;
+            sDB[s2 * pk + ii] = fmaf(-sK[s2 * pk + ii], acc[i][j], sDB[s2 * pk + ii]);
+            if (real) store1(a.dk_out + o + ii, expf(sU[s2 * pk + ii]) * acc[i][j]);
+          }
+        } else if (real) {
+          const int64_t o = row_off(a, b, h, f, a.dv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) store1(a.dv_out + o + c0 + j, acc[i][j]);
+        }
+      }
+    }
   }
   // gradient of a gate at the chunk's end: sum_j D[i][j] S_in(c+1)[i][j]
   {
@@ -443,12 +534,12 @@ int chunk_rows(const GlaShape& s) { return (s.dk > 80 || s.dv > 80) ? 32 : 64; }
 
 template <int MC>
 size_t smem_local(const GlaShape& s) {
-  return ((size_t)MC * (s.dk + 4) * 3 + (size_t)MC * (s.dv + 4) * 2 + 128) * sizeof(float);
+  return ((size_t)MC * pitch_of(s.dk) * 3 + (size_t)MC * pitch_of(s.dv) * 2 + 128) * sizeof(float);
 }
 
 template <int MC>
 size_t smem_chunk(const GlaShape& s) {
-  const size_t pk = s.dk + 4, pv = s.dv + 4;
+  const size_t pk = pitch_of(s.dk), pv = pitch_of(s.dv);
   const size_t tiles = MC * pk * 3 + MC * pv * 2 + 256;
   const size_t fact = MC * pk + s.dk * pv + 2 * (size_t)MC * (MC + 1);
   const size_t serial = 2 * (size_t)s.dk * pv;

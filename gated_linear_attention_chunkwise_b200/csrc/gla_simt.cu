@@ -37,12 +37,16 @@ struct F32Args {
   ScanGeom g;
 };
 
+// Shared-memory tiles have an odd row pitch (d + 1 floats): a warp reading one column
+// of many rows then touches as many banks as rows.
+__host__ __device__ __forceinline__ int pitch_of(int d) { return d + 1; }
+
 // Rows f0..f0+MC-1 of head h, batch b of a [B][T][H][d] fp32 tensor into a
-// plain tile with a pitch of d+4 floats; rows outside the sequence are zero.
+// plain tile of pitch pitch_of(d); rows outside the sequence are zero.
 __device__ __forceinline__ void stage_rows(float* dst, const float* src, int d, const ScanGeom& g, int f0, int b,
                                            int h, int H) {
   const int cpr = d / 4;
-  const int pitch = d + 4;
+  const int pitch = pitch_of(d);
   for (int idx = threadIdx.x; idx < MC * cpr; idx += NT) {
     const int r = idx / cpr;
     const int cc = idx - r * cpr;
@@ -51,8 +55,41 @@ __device__ __forceinline__ void stage_rows(float* dst, const float* src, int d, 
     if (f >= 0 && f < g.T)
       val = *reinterpret_cast<const float4*>(src + (((int64_t)b * g.T + base_pos_to_token(g, f)) * H + h) * d +
                                              cc * 4);
-    *reinterpret_cast<float4*>(dst + r * pitch + cc * 4) = val;
+    float* o = dst + r * pitch + cc * 4;
+    o[0] = val.x;
+    o[1] = val.y;
+    o[2] = val.z;
+    o[3] = val.w;
   }
+}
+
+// A 4 x 8 block of a matrix product in registers:
+//   acc[i][j] += sum_{k < K} A[i*ar + k*ak] * B[k*bk + j*bc]
+// (A and B point at the block's first row / column; the strides pick the layout of
+// each operand).  Twelve shared-memory loads feed 32 multiply-adds.
+__device__ __forceinline__ void mt48(float (&acc)[4][8], const float* A, int ar, int ak, const float* B, int bk,
+                                     int bc, int K) {
+#pragma unroll 2
+  for (int k = 0; k < K; ++k) {
+    float x[4], y[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = A[i * ar];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = B[j * bc];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(x[i], y[j], acc[i][j]);
+    A += ak;
+    B += bk;
+  }
+}
+
+__device__ __forceinline__ void zero48(float (&acc)[4][8]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 }
 
 // Threads i < dk: exclusive suffix sums of the log-gate along the scan order, in
@@ -62,7 +99,7 @@ __device__ __forceinline__ int suffix64(float* sLA, float* sBL, int dk, int reve
   const int i = threadIdx.x;
   int code = 0;
   if (i < dk) {
-    const int pw = dk + 4;
+    const int pw = pitch_of(dk);
     float acc = 0.f, lo = 0.f, hi = 0.f;
     for (int s = 0; s < MC; ++s) {
       const int r = reverse ? s : (MC - 1 - s);
@@ -85,7 +122,7 @@ __global__ void __launch_bounds__(NT) gla_f32_chunk_state(const F32Args a) {
   float* smem = reinterpret_cast<float*>(smem_f4);
   const int c = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
-  const int pk = a.dk + 4, pv = a.dv + 4;
+  const int pk = pitch_of(a.dk), pv = pitch_of(a.dv);
   float* sK = smem;
   float* sV = sK + MC * pk;
   float* sLA = sV + MC * pv;
@@ -105,12 +142,20 @@ __global__ void __launch_bounds__(NT) gla_f32_chunk_state(const F32Args a) {
   }
   __syncthreads();
   const int64_t cid = (int64_t)bh * a.NC + c;
-  for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
-    const int j = e / a.dk, i = e - j * a.dk;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < MC; ++s) acc = fmaf(sK[s * pk + i], sV[s * pv + j], acc);
-    a.s_locT[(cid * a.dv + j) * a.dk + i] = acc;
+  // 4 x 8 blocks of K^T V (dk x dv), stored transposed ([dv][dk])
+  {
+    const int ncg = a.dv / 8, nb = (a.dk / 4) * ncg;
+    float* dst = a.s_locT + cid * a.dv * a.dk;
+    for (int t = threadIdx.x; t < nb; t += NT) {
+      const int i0 = 4 * (t / ncg), j0 = 8 * (t % ncg);
+      float acc[4][8];
+      zero48(acc);
+      mt48(acc, sK + i0, 1, pk, sV + j0, pv, 1, MC);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dst[(int64_t)(j0 + j) * a.dk + i0 + i] = acc[i][j];
+    }
   }
   if (threadIdx.x < a.dk) a.gamma[cid * a.dk + threadIdx.x] = expf(sBL[threadIdx.x]);
   if (threadIdx.x == 0) a.flags[cid] = wide;
@@ -137,12 +182,12 @@ __global__ void __launch_bounds__(NT) gla_f32_output(const F32Args a) {
   float* smem = reinterpret_cast<float*>(smem_f4);
   const int c = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
-  const int pk = a.dk + 4, pv = a.dv + 4, pa = MC + 1;
+  const int pk = pitch_of(a.dk), pv = pitch_of(a.dv), pa = MC + 1;
   float* sQ = smem;
   float* sK = sQ + MC * pk;
   float* sLA = sK + MC * pk;
   float* sV = sLA + MC * pk;
-  float* sG = sV + MC * pv;          // [dv][dk+4]: G^T
+  float* sG = sV + MC * pv;          // [dv][pitch_of(dk)]: G^T
   float* sA = sG + a.dv * pk;        // [MC][MC+1]
   float* sBL = sA + MC * pa;
 
@@ -154,11 +199,9 @@ __global__ void __launch_bounds__(NT) gla_f32_output(const F32Args a) {
   const int64_t cid = (int64_t)bh * a.NC + c;
   {
     const float* src = a.GT + cid * a.dv * a.dk;
-    const int cpr = a.dk / 4;
-    for (int idx = threadIdx.x; idx < a.dv * cpr; idx += NT) {
-      const int j = idx / cpr, cc = idx - j * cpr;
-      *reinterpret_cast<float4*>(sG + j * pk + cc * 4) =
-          *reinterpret_cast<const float4*>(src + (int64_t)j * a.dk + cc * 4);
+    for (int e = threadIdx.x; e < a.dv * a.dk; e += NT) {
+      const int j = e / a.dk, i = e - j * a.dk;
+      sG[j * pk + i] = src[e];
     }
   }
   __syncthreads();
@@ -202,24 +245,44 @@ __global__ void __launch_bounds__(NT) gla_f32_output(const F32Args a) {
     sK[r * pk + i] *= expf(u);
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < MC * MC; e += NT) {
-    const int t = e / MC, s = e - t * MC;
-    const bool keep = a.g.reverse ? (s >= t) : (s <= t);
-    float acc = 0.f;
-    if (keep) {
-      for (int i = 0; i < a.dk; ++i) acc = fmaf(sQ[t * pk + i], sK[s * pk + i], acc);
+  const bool rev = a.g.reverse;
+  // A = mask(Q~ K^T): position s <= t in scan order is tile row s <= t (s >= t reversed)
+  {
+    const int ncg = MC / 8, nm = (MC / 4) * ncg;
+    for (int e = threadIdx.x; e < nm; e += NT) {
+      const int t0 = 4 * (e / ncg), s0 = 8 * (e % ncg);
+      float acc[4][8];
+      zero48(acc);
+      if (!(rev ? (s0 + 7 < t0) : (s0 > t0 + 3))) mt48(acc, sQ + t0 * pk, pk, 1, sK + s0 * pk, 1, pk, a.dk);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int t = t0 + i, s2 = s0 + j;
+          sA[t * pa + s2] = (rev ? (s2 >= t) : (s2 <= t)) ? acc[i][j] : 0.f;
+        }
     }
-    sA[t * pa + s] = acc;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < MC * a.dv; e += NT) {
-    const int t = e / a.dv, j = e - t * a.dv;
-    const int f = f0 + t;
-    if (f < 0 || f >= a.g.T) continue;
-    float acc = 0.f;
-    for (int s = 0; s < MC; ++s) acc = fmaf(sA[t * pa + s], sV[s * pv + j], acc);
-    for (int i = 0; i < a.dk; ++i) acc = fmaf(sQ[t * pk + i], sG[j * pk + i], acc);
-    a.out[(((int64_t)b * a.g.T + base_pos_to_token(a.g, f)) * a.H + h) * a.dv + j] = acc;
+  // O = A V + Q~ G (G held transposed: sG[j][i])
+  {
+    const int ncg = a.dv / 8, nb = (MC / 4) * ncg;
+    for (int e = threadIdx.x; e < nb; e += NT) {
+      const int t0 = 4 * (e / ncg), j0 = 8 * (e % ncg);
+      const int lo = rev ? t0 : 0, hi = rev ? MC : t0 + 4;
+      float acc[4][8];
+      zero48(acc);
+      mt48(acc, sA + t0 * pa + lo, pa, 1, sV + lo * pv + j0, pv, 1, hi - lo);
+      mt48(acc, sQ + t0 * pk, pk, 1, sG + j0 * pk, 1, pk, a.dk);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int f = f0 + t0 + i;
+        if (f < 0 || f >= a.g.T) continue;
+        float* orow = a.out + (((int64_t)b * a.g.T + base_pos_to_token(a.g, f)) * a.H + h) * a.dv + j0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) orow[j] = acc[i][j];
+      }
+    }
   }
 }
 
@@ -254,7 +317,7 @@ cudaError_t gla_f32_forward(const float* q, const float* k, const float* v, cons
   a.gamma = reinterpret_cast<float*>(ws + 2 * sl);
   a.flags = reinterpret_cast<int*>(ws + 2 * sl + rup(BH * a.NC * s.dk * 4, 256));
 
-  const size_t pk = s.dk + 4, pv = s.dv + 4;
+  const size_t pk = pitch_of(s.dk), pv = pitch_of(s.dv);
   const size_t smem_state = (MC * pk * 2 + MC * pv + s.dk) * sizeof(float);
   const size_t smem_out = (MC * pk * 3 + MC * pv + s.dv * pk + MC * (MC + 1) + s.dk) * sizeof(float);
   cudaError_t e;
