@@ -15,6 +15,8 @@ Functions and the passages they follow (see the C file for the full statement):
   gla_fwd          the GLA recurrence S_t = Diag(alpha_t) S_{t-1} + k_t^T v_t,
                    o_t = q_t S_t over the scan order, zero initial state, update
                    before read (diffusers draft "gated_linear_attention").
+  gla_fwd_glogit   the forward with the gate given as logits g:
+                   log_alpha = logsigmoid(g) / gate_norm (the configurations' gate).
   gla_bwd          the exact gradient of that recurrence (dq, dk, dv, dlog_alpha
                    for a given d out), as reverse-mode differentiation of its steps
                    in reverse scan order (DiG notes, training like DiT).
@@ -69,6 +71,8 @@ def _load():
         lib.oracle_gla_bwd_planted.argtypes = [dp] * 5 + [c_int] * 7 + [dp] * 4 + [c_int]
         lib.oracle_gla_bwd.restype = c_int
         lib.oracle_gla_bwd_planted.restype = c_int
+        lib.oracle_gla_fwd_glogit.argtypes = [dp] * 4 + [c_int] * 7 + [ctypes.c_double, dp, c_int]
+        lib.oracle_gla_fwd_glogit.restype = c_int
         lib.oracle_gla_norm_fwd.argtypes = [dp] * 3 + [c_int] * 7 + [ctypes.c_double, dp, c_int]
         lib.oracle_gla_norm_fwd_planted.argtypes = [dp] * 3 + [c_int] * 7 + [ctypes.c_double, dp, c_int]
         lib.oracle_gla_norm_fwd.restype = c_int
@@ -139,6 +143,19 @@ def gla_fwd(q, k, v, log_alpha, Hgrid: int, Wgrid: int, direction: int, nthreads
     else:
         rc = _check(lib.oracle_gla_fwd(*args, nthreads), "gla_fwd")
     return (out, rc) if return_threads else out
+
+
+def gla_fwd_glogit(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, gate_norm: float = 16.0,
+                   nthreads: int = 0) -> np.ndarray:
+    """fp64 forward with gate logits g [B,T,H,dk]: log_alpha = logsigmoid(g) / gate_norm."""
+    q, k, v, g = _f64(q), _f64(k), _f64(v), _f64(g)
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    assert T == Hgrid * Wgrid and k.shape == q.shape and g.shape == q.shape and v.shape[:3] == q.shape[:3]
+    out = np.zeros((B, T, H, dv), dtype=np.float64)
+    _check(_load().oracle_gla_fwd_glogit(_dp(q), _dp(k), _dp(v), _dp(g), B, H, Hgrid, Wgrid, dk, dv, direction,
+                                         float(gate_norm), _dp(out), nthreads), "gla_fwd_glogit")
+    return out
 
 
 def gla_bwd(q, k, v, log_alpha, dout, Hgrid: int, Wgrid: int, direction: int, nthreads: int = 0,

@@ -372,6 +372,27 @@ int oracle_gla_fwd_heads(const double *q, const double *k, const double *v, cons
                       bh_end);
 }
 
+/*
+ * The forward with the gate given as logits g (same layout as q): log_alpha =
+ * logsigmoid(g) / gate_norm, the gate definition of the GLA configurations
+ * (logsigmoid(g) = min(g, 0) - log(1 + e^{-|g|}), in fp64), then the recurrence.
+ */
+int oracle_gla_fwd_glogit(const double *q, const double *k, const double *v, const double *g, int B, int H,
+                          int Hgrid, int Wgrid, int dk, int dv, int dir, double gate_norm, double *out, int nthreads)
+{
+    if (!g || !(gate_norm > 0.0) || B <= 0 || H <= 0 || Hgrid <= 0 || Wgrid <= 0 || dk <= 0) return ORACLE_BAD_ARG;
+    const int64_t n = (int64_t)B * Hgrid * Wgrid * H * dk;
+    double *la = (double *)malloc(sizeof(double) * (size_t)n);
+    if (!la) return ORACLE_NOMEM;
+    for (int64_t e = 0; e < n; ++e) {
+        const double x = g[e];
+        la[e] = ((x < 0.0 ? x : 0.0) - log1p(exp(-fabs(x)))) / gate_norm;
+    }
+    int rc = gla_common(q, k, v, la, B, H, Hgrid, Wgrid, dk, dv, dir, out, nthreads, 0, 0, -1);
+    free(la);
+    return rc;
+}
+
 /* The recurrence with one deliberate mistake (tests of the pins only). */
 int oracle_gla_fwd_planted(const double *q, const double *k, const double *v, const double *log_alpha,
                            int B, int H, int Hgrid, int Wgrid, int dk, int dv, int dir, double *out,
