@@ -21,7 +21,8 @@ Beside the headline (rank 0, unless --no-extras): a long window of c4 GLA launch
 and the 28-layer DiG-XL/2 stack at 2048 resolution (gla_fwd -> dwconv3x3 ->
 srem_reorient per layer, fresh inputs per layer, dir = layer % 4), timed with and
 without the reorientation; the GLA backward (gla_bwd) on c4 and c2; the c4 GLA forward
-along the eight zigzag orders; and the draft's normalised variant on c4 and c2.  Under torchrun (N > 1) every rank runs its own replica of the
+along the eight zigzag orders; the draft's normalised variant on c4 and c2;
+and the c4 forward with bf16 gate logits (gla_fwd_glogit).  Under torchrun (N > 1) every rank runs its own replica of the
 workload (no data exchange: heads and batches are independent), and rank 0
 prints the aggregate.
 """
@@ -383,13 +384,14 @@ def run_gpu(args):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     extra = other_configs(dig, dev, stream, hbm) if (rank == 0 and not args.no_other_configs) else None
     gla_avg_s = statistics.mean(gla_ms) / 1e3
-    window = stack = bwd = zig = nrm = None
+    window = stack = bwd = zig = nrm = glg = None
     if rank == 0 and not args.no_extras:
         window = long_window(dig, dev, stream, dev_in, outs, hbm, gla_us_hint=gla_avg_s * 1e6)
         stack = stack_c5(dig, dev, stream, hbm)
         bwd = bwd_configs(dig, dev, stream, hbm)
         zig = zigzag_c4(dig, dev, stream, dev_in, outs, hbm)
         nrm = norm_configs(dig, dev, stream, hbm)
+        glg = glogit_c4(dig, dev, stream, hbm)
     gla_bytes = GLA_BYTES_PER_TOKEN_HEAD * w.token_heads
     achieved = gla_bytes / gla_avg_s / 1e9
     traffic = recorded_traffic()
@@ -435,6 +437,7 @@ def run_gpu(args):
             "gla_bwd": bwd,
             "gla_fwd_zigzag_c4": zig,
             "gla_norm_fwd": nrm,
+            "gla_fwd_glogit_c4": glg,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -673,6 +676,36 @@ def norm_configs(dig, dev, stream, hbm, reps=5):
     if status != 0:
         raise RuntimeError(f"device status after the normalised variant: {dig.status_string(status)}")
     return res
+
+
+def glogit_c4(dig, dev, stream, hbm, reps=10):
+    """The c4 GLA forward with bf16 gate logits (gla_fwd_glogit: log_alpha =
+    logsigmoid(g)/16 inside the kernel), median of `reps` calls per direction; its
+    algorithmic bytes are q, k, v, g and out in bf16 (720 B per token-head at d = 72)."""
+    w = WORKLOAD
+    q, k, v, g = [t.to(dev) for t in workloads.gla_inputs_glogit(w, seed=17)]
+    out = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+    per_th = 2 * (2 * w.dk + w.dv) + 2 * w.dk + 2 * w.dv
+    per_dir = []
+    for d in range(4):
+        for _ in range(2):
+            dig.gla_fwd_glogit(q, k, v, g, w.Hgrid, w.Wgrid, d, out=out)
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dig.gla_fwd_glogit(q, k, v, g, w.Hgrid, w.Wgrid, d, out=out)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        per_dir.append(statistics.median(ts))
+    status = dig.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after the gate-logit forward: {dig.status_string(status)}")
+    us = statistics.mean(per_dir)
+    return {"us_per_dir": per_dir, "bytes_per_token_head": per_th,
+            "tokens_heads_per_s": w.token_heads / (us / 1e6),
+            "frac_of_hbm": per_th * w.token_heads / (us / 1e6) / 1e9 / hbm}
 
 
 def per_kernel(w, gla_ms, conv_ms, reor_ms, hbm):

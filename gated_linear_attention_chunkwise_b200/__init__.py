@@ -7,7 +7,7 @@ the library's sm_100a kernels; there is no CPU or PyTorch fallback, and
 importing this package fails if the library has not been built
 (`python gated_linear_attention_chunkwise_b200/build.py`).
 
-Names follow the C ABI: gla_fwd, gla_fwd_f32, gla_bwd, gla_bwd_f32, gla_norm_fwd,
+Names follow the C ABI: gla_fwd, gla_fwd_glogit, gla_fwd_f32, gla_bwd, gla_bwd_f32, gla_norm_fwd,
 gla_norm_fwd_f32, srem_reorient, dwconv3x3,
 device_status (dig_gla_device_status), status_string (dig_gla_status_string).
 """
@@ -18,7 +18,7 @@ import os
 
 import torch
 
-__all__ = ["gla_fwd", "gla_fwd_f32", "gla_bwd", "gla_bwd_f32", "gla_norm_fwd", "gla_norm_fwd_f32", "srem_reorient", "dwconv3x3", "device_status", "status_string",
+__all__ = ["gla_fwd", "gla_fwd_glogit", "gla_fwd_f32", "gla_bwd", "gla_bwd_f32", "gla_norm_fwd", "gla_norm_fwd_f32", "srem_reorient", "dwconv3x3", "device_status", "status_string",
            "GlaError", "lib", "LIB_PATH", "DIR_L2R", "DIR_R2L", "DIR_T2B", "DIR_B2T"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdig_gla.so")
@@ -32,6 +32,7 @@ _lib.gla_fwd.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 7 + [_vp, _u]
 _lib.gla_fwd_f32.argtypes = [_vp, _vp, _vp, _vp] + [_i] * 7 + [_vp, _u]
 _lib.gla_bwd.argtypes = [_vp] * 5 + [_i] * 7 + [_vp] * 4 + [_u]
 _lib.gla_bwd_f32.argtypes = [_vp] * 5 + [_i] * 7 + [_vp] * 4 + [_u]
+_lib.gla_fwd_glogit.argtypes = [_vp] * 4 + [_i] * 7 + [ctypes.c_float, _vp, _u]
 _lib.gla_norm_fwd.argtypes = [_vp] * 3 + [_i] * 7 + [ctypes.c_float, _vp, _u]
 _lib.gla_norm_fwd_f32.argtypes = [_vp] * 3 + [_i] * 7 + [ctypes.c_float, _vp, _u]
 _lib.srem_reorient.argtypes = [_vp, _i, _i, _i, _i, _i, _i, _i, _vp, _u]
@@ -43,7 +44,7 @@ _lib.dig_gla_release.argtypes = []
 _lib.dig_gla_release.restype = None
 _lib.dig_gla_test_skip_items.argtypes = [_i]
 _lib.dig_gla_test_skip_items.restype = None
-for _fn in (_lib.gla_fwd, _lib.gla_fwd_f32, _lib.gla_bwd, _lib.gla_bwd_f32, _lib.gla_norm_fwd, _lib.gla_norm_fwd_f32,
+for _fn in (_lib.gla_fwd, _lib.gla_fwd_glogit, _lib.gla_fwd_f32, _lib.gla_bwd, _lib.gla_bwd_f32, _lib.gla_norm_fwd, _lib.gla_norm_fwd_f32,
             _lib.srem_reorient, _lib.dwconv3x3, _lib.dig_gla_device_status):
     _fn.restype = ctypes.c_int
 
@@ -115,6 +116,30 @@ def _gla(fn_name: str, q, k, v, log_alpha, Hgrid, Wgrid, direction, out, stream,
 def gla_fwd(q, k, v, log_alpha, Hgrid: int, Wgrid: int, direction: int, out=None, stream=None):
     """bf16 GLA forward (see include/dig_gla.h, gla_fwd).  Returns `out` [B,T,H,dv] bf16."""
     return _gla("gla_fwd", q, k, v, log_alpha, Hgrid, Wgrid, direction, out, stream, torch.bfloat16)
+
+
+def gla_fwd_glogit(q, k, v, g, Hgrid: int, Wgrid: int, direction: int, gate_norm: float = 16.0, out=None,
+                   stream=None):
+    """bf16 GLA forward with bf16 gate logits g (log_alpha = logsigmoid(g) / gate_norm in
+    the kernel; see include/dig_gla.h, gla_fwd_glogit).  Returns `out` [B,T,H,dv] bf16."""
+    dev = q.device
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g")):
+        _need(t, n, torch.bfloat16, dev)
+    if q.dim() != 4 or k.shape != q.shape or g.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise ValueError("expected q, k, g [B,T,H,dk] and v [B,T,H,dv]")
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    if T != Hgrid * Wgrid:
+        raise ValueError(f"T={T} does not match the grid {Hgrid}x{Wgrid}")
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    else:
+        _need(out, "out", torch.bfloat16, dev)
+    with torch.cuda.device(dev):
+        rc = _lib.gla_fwd_glogit(q.data_ptr(), k.data_ptr(), v.data_ptr(), g.data_ptr(), B, H, Hgrid, Wgrid, dk, dv,
+                                 int(direction), float(gate_norm), out.data_ptr(), _stream_handle(dev, stream))
+    _check("gla_fwd_glogit", rc)
+    return out
 
 
 def gla_fwd_f32(q, k, v, log_alpha, Hgrid: int, Wgrid: int, direction: int, out=None, stream=None):

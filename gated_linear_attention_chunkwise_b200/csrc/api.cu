@@ -118,6 +118,22 @@ int validate_gla_norm(const void* q, const void* k, const void* v, const void* o
   return GLA_OK;
 }
 
+// The gate-logit forward: q, k, v, g (bf16, g shaped like q), out; dk at most 120
+// (the logit tile's padded TMA box); the four SREM orders; gate_norm positive.
+int validate_gla_glogit(const void* q, const void* k, const void* v, const void* g, const void* out, int B, int H,
+                        int Hg, int Wg, int dk, int dv, int dir, float gate_norm) {
+  if (!g) return GLA_ERR_INVALID_ARG;
+  int rc = validate_gla_norm(q, k, v, out, B, H, Hg, Wg, dk, dv, dir > 3 ? 0 : dir, 1.f, 2);
+  if (rc != GLA_OK) return rc;
+  if (dir > 3) return GLA_ERR_UNSUPPORTED;
+  if (!(gate_norm > 0.f)) return GLA_ERR_INVALID_ARG;
+  if (dk > 120 || dv > 128) return GLA_ERR_UNSUPPORTED;
+  if (!aligned16(g)) return GLA_ERR_ALIGNMENT;
+  const size_t rows = (size_t)B * Hg * Wg * H;
+  if (overlaps(out, rows * dv * 2, g, rows * dk * 2)) return GLA_ERR_INVALID_ARG;
+  return GLA_OK;
+}
+
 namespace {
 
 int validate_grid(const void* x, const void* y, int B, int Hg, int Wg, int C, int dtype, size_t* row_bytes) {
@@ -341,6 +357,19 @@ int gla_bwd_common(const void* q, const void* k, const void* v, const float* la,
   BwdCall c{q, k, v, la, dout, dq, dk_out, dv_out, dla, GlaShape{B, H, Hgrid, Wgrid, dk, dv, dir}, bf16, stream};
   return dig::run_with_workspace(bwd_ws_bytes(c.s, bf16), stream, run_bwd, &c);
 }
+// ---- gate logits in place of log_alpha ------------------------------------------
+struct GlogitCall {
+  const void *q, *k, *v, *g;
+  float gate_norm;
+  void* out;
+  GlaShape s;
+  cudaStream_t st;
+};
+cudaError_t run_glogit(void* ws, void* ctx) {
+  const GlogitCall* c = static_cast<const GlogitCall*>(ctx);
+  return dig::gla_ws_forward_glogit(c->q, c->k, c->v, c->g, c->gate_norm, c->out, c->s, ws, c->st);
+}
+
 // ---- the normalised variant ----------------------------------------------------
 struct NormCall {
   const void *q, *k, *v;
@@ -392,6 +421,15 @@ int gla_norm_common(const void* q, const void* k, const void* v, int B, int H, i
 }  // namespace
 
 extern "C" {
+
+int gla_fwd_glogit(const void* q, const void* k, const void* v, const void* g, int B, int H, int Hgrid, int Wgrid,
+                   int dk, int dv, int dir, float gate_norm, void* out, cudaStream_t stream) {
+  int rc = dig::validate_gla_glogit(q, k, v, g, out, B, H, Hgrid, Wgrid, dk, dv, dir, gate_norm);
+  if (rc != GLA_OK) return rc;
+  if ((rc = dig::check_device()) != GLA_OK) return rc;
+  GlogitCall c{q, k, v, g, gate_norm, out, GlaShape{B, H, Hgrid, Wgrid, dk, dv, dir}, stream};
+  return dig::run_with_workspace(dig::gla_ws_workspace_bytes(c.s), stream, run_glogit, &c);
+}
 
 int gla_norm_fwd(const void* q, const void* k, const void* v, int B, int H, int Hgrid, int Wgrid, int dk, int dv,
                  int dir, float eps, void* out, cudaStream_t stream) {

@@ -100,6 +100,8 @@ struct WsArgs {
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
   const float* la;
+  const __nv_bfloat16* glog;  // gate logits [B][T][H][dk] when set: log_alpha = logsigmoid(g) / gate_norm
+  float inv_gate_norm;        // 1 / gate_norm
   __nv_bfloat16* out;
   float* agg_S;   // [BH][NS][dv/4][dk][4]  segment aggregates (quads of value columns)
   float* agg_g;   // [BH][NS][dk]           exp(segment log-gate sums)
@@ -269,6 +271,20 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// log2(alpha) for a gate logit g: logsigmoid(g) / gate_norm in log2 units,
+//   logsigmoid(g) = min(g, 0) - ln(1 + e^{-|g|}),
+// so log2 alpha = (min(g, 0) log2 e - log2(1 + 2^{-|g| log2 e})) / gate_norm; the
+// exponential never exceeds 1.
+__device__ __forceinline__ float log2_gate(float g, float inv_norm) {
+  return (fminf(g, 0.f) * kLog2e - lg2_approx(1.f + exp2_approx(-fabsf(g) * kLog2e))) * inv_norm;
+}
+
 // Lane-wise product of two packed bf16 pairs, rounded to bf16.
 __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t x, uint32_t y) {
   __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&x), *reinterpret_cast<__nv_bfloat162*>(&y));
@@ -330,6 +346,21 @@ __device__ __forceinline__ int row_token(const WsArgs& a, int cf, int r) {
   }
   const int x = cf / a.ppr, y = (cf - x * a.ppr) * MC + r;
   return y < a.g.Hg ? y * a.g.Wg + x : -1;
+}
+
+// Rows of forward chunk cf's tile that hold tokens: always a prefix [0, n) of the tile
+// (the end of the sequence, the columns past Wg, or the end of a column piece).
+__device__ __forceinline__ int chunk_valid_rows(const WsArgs& a, int cf) {
+  int n;
+  if (a.mode == 0) {
+    n = a.g.T - cf * MC;
+  } else if (a.mode == 1) {
+    n = (a.g.Wg - cf * a.rpc) * a.g.Hg;
+  } else {
+    const int x = cf / a.ppr;
+    n = a.g.Hg - (cf - x * a.ppr) * MC;
+  }
+  return n < MC ? n : MC;
 }
 
 // TMA coordinates (run position, run index) of forward chunk cf's box.
@@ -405,7 +436,12 @@ __device__ void chunk_serial(const WsArgs& a, const uint8_t* st, float* red, uin
       qi = 0.f;
       if (t >= 0 && i < a.dk) {
         const int64_t o = (((int64_t)b * a.g.T + t) * a.H + h) * a.dk + i;
-        al = __expf(__ldg(a.la + o));
+        if (a.glog) {
+          const float gg = __bfloat162float(a.glog[o]);
+          al = expf((fminf(gg, 0.f) - log1pf(expf(-fabsf(gg)))) * a.inv_gate_norm);
+        } else {
+          al = __expf(__ldg(a.la + o));
+        }
         kq = __bfloat162float(a.k[o]);
         qi = __bfloat162float(a.q[o]);
       }
@@ -627,6 +663,9 @@ __device__ __forceinline__ uint32_t align1024(uint32_t x) { return (x + 1023u) &
 // k % 2, which holds its aggregate after pass 1, its incoming state after the
 // look-back and its running state during pass 2.
 // ---------------------------------------------------------------------------
+// kGlogit: the gates arrive as bf16 logits (a.glog) and the suffix warps turn them into
+// log2 gates; a separate instance so that the fp32-gate kernel carries none of that code.
+template <bool kGlogit>
 __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsArgs a, const __grid_constant__ TensorMaps tm) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -913,16 +952,52 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
         const int dr = a.g.reverse ? (pw >> 1) : -(pw >> 1);  // in float2
         float2* pa = reinterpret_cast<float2*>(lag + (a.g.reverse ? 64 * sw : 64 * sw + 31) * pw) + lane;
         float2* pb = pa + 16 * pw;  // the other quarter: 32 rows on
+        // Gate logits arrive as bf16 at the start of each fp32 row (the box is padded to
+        // the row pitch), one packed pair per lane: a row's logits are read before the
+        // same row's sums overwrite them, and rows never overlap.
+        const uint32_t* ua =
+            reinterpret_cast<const uint32_t*>(lag + (a.g.reverse ? 64 * sw : 64 * sw + 31) * pw) + lane;
+        const uint32_t* ub = ua + 32 * pw;  // the other quarter: 32 rows on
+        const int du = 2 * dr;  // 4-byte words per row step
+        const float mul = kGlogit ? 1.f : kLog2e;  // logits are converted straight to log2 units
+        // Rows past the chunk's tokens hold the box's zero fill: a zero logit is not a
+        // neutral gate (logsigmoid(0) < 0), so those rows get gate 0 explicitly.
+        int nvalid = MC;
+        if (kGlogit) {
+          const Item itj = decode_item(a, sJob[4 * s + 1]);
+          const int cj = pass1 ? itj.c0 + itj.n - 1 - j : itj.c0 + j;  // pass 1 walks its chunks backwards
+          nvalid = chunk_valid_rows(a, fwd_chunk(a, cj));
+        }
+        const int row_a0 = a.g.reverse ? 64 * sw : 64 * sw + 31, row_step = a.g.reverse ? 1 : -1;
+        auto gate2 = [&](uint32_t w) {
+          const float2 g = unpack_bf16x2(w);
+          return make_float2(log2_gate(g.x, a.inv_gate_norm), log2_gate(g.y, a.inv_gate_norm));
+        };
         float2 a0 = make_float2(0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
 #pragma unroll 1
         for (int h8 = 0; h8 < 4; ++h8) {
           float2 xa[8], xb[8], ya[8], yb[8];
+          if (kGlogit) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            xa[q] = act0 ? pa[q * dr] : make_float2(0.f, 0.f);
-            xb[q] = act0 ? pb[q * dr] : make_float2(0.f, 0.f);
-            ya[q] = act1 ? pa[q * dr + 32] : make_float2(0.f, 0.f);
-            yb[q] = act1 ? pb[q * dr + 32] : make_float2(0.f, 0.f);
+            for (int q = 0; q < 8; ++q) {
+              const float2 z = make_float2(0.f, 0.f);
+              const int ra = row_a0 + row_step * (8 * h8 + q);  // row of quarter a; quarter b is 32 on
+              const bool va = ra < nvalid, vb = ra + 32 < nvalid;
+              xa[q] = act0 && va ? gate2(ua[q * du]) : z;
+              xb[q] = act0 && vb ? gate2(ub[q * du]) : z;
+              ya[q] = act1 && va ? gate2(ua[q * du + 32]) : z;
+              yb[q] = act1 && vb ? gate2(ub[q * du + 32]) : z;
+            }
+            ua += 8 * du;
+            ub += 8 * du;
+          } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              xa[q] = act0 ? pa[q * dr] : make_float2(0.f, 0.f);
+              xb[q] = act0 ? pb[q * dr] : make_float2(0.f, 0.f);
+              ya[q] = act1 ? pa[q * dr + 32] : make_float2(0.f, 0.f);
+              yb[q] = act1 ? pb[q * dr + 32] : make_float2(0.f, 0.f);
+            }
           }
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
@@ -934,14 +1009,14 @@ __global__ void __launch_bounds__(NT, 1) gla_ws_fwd(const __grid_constant__ WsAr
               pa[q * dr + 32] = a1;
               pb[q * dr + 32] = b1;
             }
-            a0.x = fmaf(xa[q].x, kLog2e, a0.x);
-            a0.y = fmaf(xa[q].y, kLog2e, a0.y);
-            b0.x = fmaf(xb[q].x, kLog2e, b0.x);
-            b0.y = fmaf(xb[q].y, kLog2e, b0.y);
-            a1.x = fmaf(ya[q].x, kLog2e, a1.x);
-            a1.y = fmaf(ya[q].y, kLog2e, a1.y);
-            b1.x = fmaf(yb[q].x, kLog2e, b1.x);
-            b1.y = fmaf(yb[q].y, kLog2e, b1.y);
+            a0.x = fmaf(xa[q].x, mul, a0.x);
+            a0.y = fmaf(xa[q].y, mul, a0.y);
+            b0.x = fmaf(xb[q].x, mul, b0.x);
+            b0.y = fmaf(xb[q].y, mul, b0.y);
+            a1.x = fmaf(ya[q].x, mul, a1.x);
+            a1.y = fmaf(ya[q].y, mul, a1.y);
+            b1.x = fmaf(yb[q].x, mul, b1.x);
+            b1.y = fmaf(yb[q].y, mul, b1.y);
           }
           pa += 8 * dr;
           pb += 8 * dr;
@@ -1453,15 +1528,21 @@ size_t gla_ws_workspace_bytes(const GlaShape& s) {
   return L.flag_bytes + 2 * L.agg_bytes + L.aggg_bytes;
 }
 
-cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const float* la, void* out, const GlaShape& s,
-                           void* workspace, cudaStream_t st) {
+namespace {
+// glog != nullptr: the gates are bf16 logits g and log_alpha = logsigmoid(g) / gate_norm
+// (la unused); the logit tile's TMA box is padded to the fp32 tile's row pitch.
+cudaError_t ws_forward(const void* q, const void* k, const void* v, const float* la, const void* glog,
+                       float gate_norm, void* out, const GlaShape& s, void* workspace, cudaStream_t st) {
   const WsLayout L = ws_layout(s);
   if (L.smem > kMaxSmem) return cudaErrorInvalidValue;
+  if (glog && 2 * (s.dk + 4) > 256) return cudaErrorInvalidValue;  // TMA box of at most 256 elements
   WsArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k = static_cast<const __nv_bfloat16*>(k);
   a.v = static_cast<const __nv_bfloat16*>(v);
   a.la = la;
+  a.glog = static_cast<const __nv_bfloat16*>(glog);
+  a.inv_gate_norm = glog ? 1.f / gate_norm : 1.f;
   a.out = static_cast<__nv_bfloat16*>(out);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t BH = (size_t)s.B * s.H;
@@ -1521,7 +1602,10 @@ cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const fl
   if (!(encode_map(&tm.q, q, false, s.dk, 16, CU_TENSOR_MAP_SWIZZLE_32B, s, column, box_rows, box_runs) &&
         encode_map(&tm.k, k, false, s.dk, 16, CU_TENSOR_MAP_SWIZZLE_32B, s, column, box_rows, box_runs) &&
         encode_map(&tm.v, v, false, s.dv, 16, CU_TENSOR_MAP_SWIZZLE_32B, s, column, box_rows, box_runs) &&
-        encode_map(&tm.la, la, true, s.dk, s.dk + 4, CU_TENSOR_MAP_SWIZZLE_NONE, s, column, box_rows, box_runs)))
+        (glog ? encode_map(&tm.la, glog, false, s.dk, 2 * (s.dk + 4), CU_TENSOR_MAP_SWIZZLE_NONE, s, column, box_rows,
+                           box_runs)
+              : encode_map(&tm.la, la, true, s.dk, s.dk + 4, CU_TENSOR_MAP_SWIZZLE_NONE, s, column, box_rows,
+                           box_runs))))
     return cudaErrorInvalidValue;
   a.nak = a.nav = 0;
   if (L.mode == 0) {
@@ -1533,7 +1617,8 @@ cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const fl
   }
   cudaError_t e = cudaMemsetAsync(ws, 0, L.flag_bytes, st);  // flags and the ticket counter
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(gla_ws_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
+  auto kernel = glog ? gla_ws_fwd<true> : gla_ws_fwd<false>;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   e = cudaGetDevice(&dev);
@@ -1541,8 +1626,19 @@ cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const fl
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const size_t grid = (size_t)a.items < (size_t)sms ? (size_t)a.items : (size_t)sms;
-  gla_ws_fwd<<<(unsigned)grid, NT, L.smem, st>>>(a, tm);
+  kernel<<<(unsigned)grid, NT, L.smem, st>>>(a, tm);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const float* la, void* out, const GlaShape& s,
+                           void* workspace, cudaStream_t st) {
+  return ws_forward(q, k, v, la, nullptr, 1.f, out, s, workspace, st);
+}
+
+cudaError_t gla_ws_forward_glogit(const void* q, const void* k, const void* v, const void* g, float gate_norm, void* out,
+                                  const GlaShape& s, void* workspace, cudaStream_t st) {
+  return ws_forward(q, k, v, nullptr, g, gate_norm, out, s, workspace, st);
 }
 
 }  // namespace dig

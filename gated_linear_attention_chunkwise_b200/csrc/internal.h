@@ -23,6 +23,11 @@ size_t gla_ws_workspace_bytes(const GlaShape& s);
 cudaError_t gla_ws_forward(const void* q, const void* k, const void* v, const float* la, void* out, const GlaShape& s,
                            void* workspace, cudaStream_t st);
 
+// The same kernel with bf16 gate logits g in place of log_alpha:
+// log_alpha = logsigmoid(g) / gate_norm, computed in the kernel (dk <= 120).
+cudaError_t gla_ws_forward_glogit(const void* q, const void* k, const void* v, const void* g, float gate_norm, void* out,
+                                  const GlaShape& s, void* workspace, cudaStream_t st);
+
 // ---- fp32 SIMT path (chunks of 64 scan positions) ----
 constexpr int kChunkF32 = 64;
 size_t gla_f32_workspace_bytes(const GlaShape& s);

@@ -97,6 +97,23 @@ int gla_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
             int Wgrid, int dk, int dv, int dir, void* out, cudaStream_t stream);
 
 /*
+ * gla_fwd_glogit -- gla_fwd with the forget gate given as bf16 logits g instead of
+ * fp32 log_alpha: log_alpha = logsigmoid(g) / gate_norm, computed inside the kernel
+ * from the bf16 tile (the gate definition of the GLA configurations, gate_norm = 16),
+ * so log_alpha is never written or read in fp32: the gate costs 2 bytes per key
+ * channel per token instead of 4.
+ *   g          [B][T][H][dk] bf16 (the layout of q)
+ *   gate_norm  > 0
+ *   dk, dv     multiples of 8 in [8, 120]; dir 0..3 (the SREM orders)
+ * Everything else -- shapes, arithmetic, output, errors, workspace -- as gla_fwd.
+ * The logsigmoid is evaluated with the hardware base-2 exponential and logarithm
+ * (relative error about 2^-22) in the suffix-sum warps; the token-serial fallback
+ * uses expf / log1pf.  No output may overlap an input.
+ */
+int gla_fwd_glogit(const void* q, const void* k, const void* v, const void* g, int B, int H, int Hgrid, int Wgrid,
+                   int dk, int dv, int dir, float gate_norm, void* out, cudaStream_t stream);
+
+/*
  * gla_fwd_f32 -- the same recurrence with fp32 q, k, v and out (all arithmetic
  * fp32, no tensor-core rounding).  Same shapes, directions and errors as gla_fwd.
  */

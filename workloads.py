@@ -154,3 +154,19 @@ def gla_dout(w: Workload, seed: int = 0, scale: float | None = None):
     if w.dtype == "bf16":
         d = d.to(torch.bfloat16)
     return d.contiguous()
+
+
+def gla_inputs_glogit(w: Workload, seed: int = 0):
+    """(q, k, v, g) with the same draws as gla_inputs (g before its logsigmoid), g cast to
+    bf16: the gate-logit form of the same workload (log_alpha = logsigmoid(g) / 16 of the
+    bf16 g)."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(seed))
+    scale = 1.0 / math.sqrt(w.dk)
+    shp_k = (w.B, w.T, w.H, w.dk)
+    shp_v = (w.B, w.T, w.H, w.dv)
+    q = torch.randn(shp_k, generator=gen, dtype=torch.float32) * scale
+    k = torch.randn(shp_k, generator=gen, dtype=torch.float32) * scale
+    v = torch.randn(shp_v, generator=gen, dtype=torch.float32) * scale
+    g = torch.randn(shp_k, generator=gen, dtype=torch.float32) + w.g_mean
+    return tuple(t.to(torch.bfloat16).contiguous() for t in (q, k, v, g))
