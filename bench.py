@@ -481,6 +481,17 @@ def other_configs(dig, dev, stream, hbm, reps=10):
     return res
 
 
+def oracle_beside(fn, token_heads, sample):
+    """The fp64 oracle timed on the host's threads on a bounded sample of an extra
+    entry point's workload: {value (token-heads/s), unit, cores, kind, sample}."""
+    import oracle
+    t0 = time.perf_counter()
+    fn()
+    secs = time.perf_counter() - t0
+    return {"value": token_heads / secs, "unit": UNIT, "cores": oracle.hardware_threads(), "kind": "oracle",
+            "sample": sample, "seconds": secs}
+
+
 def stack_c5(dig, dev, stream, hbm, reps=5):
     """The 28-layer DiG-XL/2 stack at 2048 resolution (128x128 grid, B=1, H=16, d=72):
     layer l runs gla_fwd(dir = l % 4) -> dwconv3x3 -> srem_reorient(dir = (l+1) % 4)
@@ -604,6 +615,13 @@ def bwd_configs(dig, dev, stream, hbm, reps=5):
                 ts.append(e0.elapsed_time(e1) * 1e3)
             per_dir.append(statistics.median(ts))
         us = statistics.mean(per_dir)
+        if name == "c2":
+            import oracle
+            hq, hk, hv, hla = workloads.gla_inputs(cw, seed=11)
+            hdo = workloads.gla_dout(cw, seed=11)
+            res["cpu_baseline"] = oracle_beside(
+                lambda: oracle.gla_bwd(hq, hk, hv, hla, hdo, cw.Hgrid, cw.Wgrid, 0), cw.token_heads,
+                "fp64 oracle reverse sweep, c2 whole (48 heads), direction 0, all host threads")
         res[name] = {"workload": cw.name, "kernel": "gla_bwd (3 launches: local terms, chunk scans, gradients)",
                      "us_per_dir": per_dir, "bytes": nbytes, "bytes_per_token_head": per_th,
                      "tokens_heads_per_s": cw.token_heads / (us / 1e6),
@@ -637,12 +655,16 @@ def zigzag_c4(dig, dev, stream, dev_in, outs, hbm, reps=5):
     status = dig.device_status()
     if status != 0:
         raise RuntimeError(f"device status after the zigzag orders: {dig.status_string(status)}")
+    import oracle
+    hq, hk, hv, hla = (t.double().numpy() for t in workloads.gla_inputs(w, seed=0))
+    cpu = oracle_beside(lambda: oracle.gla_fwd(hq, hk, hv, hla, w.Hgrid, w.Wgrid, 4, heads=(0, 16)),
+                        16 * w.T, "fp64 oracle, c4 heads 0..15 of 32 along zigzag scheme 0, all host threads")
     us = statistics.mean(per)
     gla_bytes = GLA_BYTES_PER_TOKEN_HEAD * w.token_heads
     copy_bytes = 2 * (2 * (2 * w.dk + w.dv) + 4 * w.dk + 2 * w.dv) * w.token_heads  # gathers + scatter
     return {"us_per_scheme": per, "tokens_heads_per_s": w.token_heads / (us / 1e6),
             "frac_of_hbm": gla_bytes / (us / 1e6) / 1e9 / hbm,
-            "bytes_moved_incl_arranging": gla_bytes + copy_bytes}
+            "bytes_moved_incl_arranging": gla_bytes + copy_bytes, "cpu_baseline": cpu}
 
 
 def norm_configs(dig, dev, stream, hbm, reps=5):
@@ -667,6 +689,12 @@ def norm_configs(dig, dev, stream, hbm, reps=5):
                 ts.append(e0.elapsed_time(e1) * 1e3)
             per_dir.append(statistics.median(ts))
         us = statistics.mean(per_dir)
+        if name == "c2":
+            import oracle
+            hq, hk, hv, _ = workloads.gla_inputs(cw, seed=13)
+            res["cpu_baseline"] = oracle_beside(
+                lambda: oracle.gla_norm_fwd(hq, hk, hv, cw.Hgrid, cw.Wgrid, 0), cw.token_heads,
+                "fp64 oracle of the normalised variant, c2 whole (48 heads), direction 0, all host threads")
         res[name] = {"workload": cw.name, "kernels": "prep + fp32 chunk-wise GLA (3) + post",
                      "us_per_dir": per_dir, "bytes_per_token_head": per_th,
                      "tokens_heads_per_s": cw.token_heads / (us / 1e6),
@@ -702,8 +730,12 @@ def glogit_c4(dig, dev, stream, hbm, reps=10):
     status = dig.device_status()
     if status != 0:
         raise RuntimeError(f"device status after the gate-logit forward: {dig.status_string(status)}")
+    import oracle
+    hq, hk, hv, hg = workloads.gla_inputs_glogit(w, seed=17)
+    cpu = oracle_beside(lambda: oracle.gla_fwd_glogit(hq, hk, hv, hg, w.Hgrid, w.Wgrid, 0, 16.0), w.token_heads,
+                        "fp64 oracle with gate logits, c4 whole (32 heads), direction 0, all host threads")
     us = statistics.mean(per_dir)
-    return {"us_per_dir": per_dir, "bytes_per_token_head": per_th,
+    return {"cpu_baseline": cpu, "us_per_dir": per_dir, "bytes_per_token_head": per_th,
             "tokens_heads_per_s": w.token_heads / (us / 1e6),
             "frac_of_hbm": per_th * w.token_heads / (us / 1e6) / 1e9 / hbm}
 
