@@ -167,13 +167,13 @@ int gla_fwd_f32_noalloc(const float* q, const float* k, const float* v, const fl
  * from q, k [B][T][H][dk] bf16, v and dout [B][T][H][dv] bf16 and log_alpha
  * [B][T][H][dk] fp32, all at canonical token positions.
  * Arithmetic: every product and sum in fp32 on CUDA cores, from the bf16 inputs
- * widened exactly; dq, dk, dv rounded to nearest even on the store.  Chunks of 64
- * scan positions (32 when dk or dv exceeds 80); a chunk whose gates decay by more
- * than e^80 inside it (a full reset, -inf) is differentiated token by token (exact,
- * slower).  Growth gates whose product exceeds e^80 inside a chunk record
+ * widened exactly; dq, dk, dv rounded to nearest even on the store.  Chunks of 32
+ * scan positions; a chunk whose gates decay by more than e^80 inside it (a full
+ * reset, -inf) is differentiated token by token (exact, slower).  Growth gates whose product exceeds e^80 inside a chunk record
  * GLA_ERR_RANGE.  Shapes, dims, directions and errors as gla_fwd; no output may
- * overlap an input or another output.  Workspace as gla_fwd (2 * B*H*ceil(T/64) *
- * dk*dv fp32 values, plus per-chunk gates).
+ * overlap an input or another output.  Workspace: 2 * B*H*ceil(T/32) * dk*dv fp32
+ * values plus per-chunk gates (520 MB for B=2, H=16, T=12544, d=72), stream-ordered
+ * from the library's pool as gla_fwd's.
  */
 int gla_bwd(const void* q, const void* k, const void* v, const float* log_alpha, const void* dout, int B, int H,
             int Hgrid, int Wgrid, int dk, int dv, int dir, void* dq, void* dk_out, void* dv_out, float* dlog_alpha,

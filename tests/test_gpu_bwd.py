@@ -97,14 +97,14 @@ def test_bwd_bf16_c2(dig, direction):
 @pytest.mark.parametrize("direction", [0, 1, 2, 3])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_bwd_ragged_d72(dig, direction, dtype):
-    """d = 72 (the DiG-XL/2 head width), a 9x23 grid: 207 tokens, three full
-    chunks of 64 and a ragged one; columns of 9 split across chunks."""
+    """d = 72 (the DiG-XL/2 head width), a 9x23 grid: 207 tokens, six full chunks of
+    32 and a ragged one; columns of 9 split across chunks."""
     run_case(dig, workloads.custom(2, 3, 9, 23, 72, 72, dtype), direction, seed=4)
 
 
 @pytest.mark.parametrize("dims", [(128, 128), (32, 96), (88, 40)])
-def test_bwd_wide_heads_32_row_chunks(dig, dims):
-    """dk or dv above 80 switch to chunks of 32 positions."""
+def test_bwd_wide_heads(dig, dims):
+    """Heads wider than 80 channels (the largest shared-memory footprint) and dk != dv."""
     dk, dv = dims
     for direction in (0, 3):
         run_case(dig, workloads.custom(1, 2, 7, 11, dk, dv, "bf16"), direction, seed=5)
