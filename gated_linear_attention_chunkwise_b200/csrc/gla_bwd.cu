@@ -101,17 +101,18 @@ __device__ __forceinline__ void stage(float* dst, const TE* src, int d, const Sc
 //   acc[i][j] += sum_{k < K} A[i*ar + k*ak] * B[k*bk + j*bc]
 // (A and B point at the block's first row / column; the strides pick the layout of
 // each operand).  Twelve shared-memory loads feed 32 multiply-adds.
-__device__ __forceinline__ void mt48(float (&acc)[4][8], const float* A, int ar, int ak, const float* B, int bk,
+template <int R>
+__device__ __forceinline__ void mt48(float (&acc)[R][8], const float* A, int ar, int ak, const float* B, int bk,
                                      int bc, int K) {
 #pragma unroll 2
   for (int k = 0; k < K; ++k) {
-    float x[4], y[8];
+    float x[R], y[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = A[i * ar];
+    for (int i = 0; i < R; ++i) x[i] = A[i * ar];
 #pragma unroll
     for (int j = 0; j < 8; ++j) y[j] = B[j * bc];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < R; ++i)
 #pragma unroll
       for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(x[i], y[j], acc[i][j]);
     A += ak;
@@ -119,12 +120,15 @@ __device__ __forceinline__ void mt48(float (&acc)[4][8], const float* A, int ar,
   }
 }
 
-__device__ __forceinline__ void zero48(float (&acc)[4][8]) {
+template <int R>
+__device__ __forceinline__ void zero48(float (&acc)[R][8]) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < R; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 }
+
+
 
 // Threads i < dk: the log-gate tile becomes, in place, the exclusive suffix sums u
 // along the scan order; the chunk total goes to sTot[i].  Returns bit 1 if |u| or
@@ -207,8 +211,8 @@ __global__ void __launch_bounds__(NT) gla_bwd_local(const BwdArgs<TI> a) {
     const int which = t >= nb, tt = which ? t - nb : t;
     const int i0 = 4 * (tt / ncg), j0 = 8 * (tt % ncg);
     float acc[4][8];
-    zero48(acc);
-    mt48(acc, (which ? sQ : sK) + i0, 1, pk, (which ? sO : sV) + j0, pv, 1, MC);
+    zero48<4>(acc);
+    mt48<4>(acc, (which ? sQ : sK) + i0, 1, pk, (which ? sO : sV) + j0, pv, 1, MC);
     float* dst = which ? dd : sx;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -351,7 +355,9 @@ __device__ void chunk_serial_bwd(const BwdArgs<TI>& a, float* sQ, float* sK, flo
   }
 }
 
-template <typename TI, int MC>
+// kTR: rows per register block of the product phases -- 2 when the largest phase
+// (dK^ and dV together) still has at most one block per thread, else 4.
+template <typename TI, int MC, int kTR>
 __global__ void __launch_bounds__(NT) gla_bwd_chunk(const BwdArgs<TI> a) {
   extern __shared__ float4 smem_f4[];
   float* smem = reinterpret_cast<float*>(smem_f4);
@@ -406,27 +412,27 @@ __global__ void __launch_bounds__(NT) gla_bwd_chunk(const BwdArgs<TI> a) {
   // Positions s <= r in scan order are tile rows s <= r, or s >= r for reversed
   // directions: the nonzero range of a row block of A or P, and of a column block.
   auto lo_of_rows = [&](int r0) { return rev ? r0 : 0; };
-  auto hi_of_rows = [&](int r0) { return rev ? MC : r0 + 4; };
+  auto hi_of_rows = [&](int r0) { return rev ? MC : r0 + kTR; };
   auto lo_of_cols = [&](int s0) { return rev ? 0 : s0; };
-  auto hi_of_cols = [&](int s0) { return rev ? s0 + 4 : MC; };
+  auto hi_of_cols = [&](int s0) { return rev ? s0 + kTR : MC; };
   // A = mask(dO V^T) (blocks 0 .. nm-1) and P = mask(Q~ K^T) (nm .. 2nm-1), MC x MC.
   {
-    const int ncg = MC / 8, nm = (MC / 4) * ncg;
+    const int ncg = MC / 8, nm = (MC / kTR) * ncg;
     for (int t = threadIdx.x; t < 2 * nm; t += NT) {
       const int which = t >= nm, tt = which ? t - nm : t;
-      const int r0 = 4 * (tt / ncg), s0 = 8 * (tt % ncg);
-      float acc[4][8];
-      zero48(acc);
-      const bool empty = rev ? (s0 + 7 < r0) : (s0 > r0 + 3);
+      const int r0 = kTR * (tt / ncg), s0 = 8 * (tt % ncg);
+      float acc[kTR][8];
+      zero48<kTR>(acc);
+      const bool empty = rev ? (s0 + 7 < r0) : (s0 > r0 + kTR - 1);
       if (!empty) {
         if (which)
-          mt48(acc, sQ + r0 * pk, pk, 1, sK + s0 * pk, 1, pk, a.dk);
+          mt48<kTR>(acc, sQ + r0 * pk, pk, 1, sK + s0 * pk, 1, pk, a.dk);
         else
-          mt48(acc, sO + r0 * pv, pv, 1, sV + s0 * pv, 1, pv, a.dv);
+          mt48<kTR>(acc, sO + r0 * pv, pv, 1, sV + s0 * pv, 1, pv, a.dv);
       }
       float* dst = which ? sP : sA;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < kTR; ++i)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int r = r0 + i, s2 = s0 + j;
@@ -438,16 +444,16 @@ __global__ void __launch_bounds__(NT) gla_bwd_chunk(const BwdArgs<TI> a) {
   __syncthreads();
   // dQ~ = dO G^T + A K^ (MC x dk)
   {
-    const int ncg = a.dk / 8, nb = (MC / 4) * ncg;
+    const int ncg = a.dk / 8, nb = (MC / kTR) * ncg;
     for (int t = threadIdx.x; t < nb; t += NT) {
-      const int r0 = 4 * (t / ncg), i0 = 8 * (t % ncg);
-      float acc[4][8];
-      zero48(acc);
-      mt48(acc, sO + r0 * pv, pv, 1, sS + i0 * pv, 1, pv, a.dv);
+      const int r0 = kTR * (t / ncg), i0 = 8 * (t % ncg);
+      float acc[kTR][8];
+      zero48<kTR>(acc);
+      mt48<kTR>(acc, sO + r0 * pv, pv, 1, sS + i0 * pv, 1, pv, a.dv);
       const int lo = lo_of_rows(r0), hi = hi_of_rows(r0);
-      mt48(acc, sA + r0 * pa + lo, pa, 1, sK + lo * pk + i0, pk, 1, hi - lo);
+      mt48<kTR>(acc, sA + r0 * pa + lo, pa, 1, sK + lo * pk + i0, pk, 1, hi - lo);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kTR; ++i) {
         const int r = r0 + i, f = f0 + r;
         const bool real = f >= 0 && f < a.g.T;
         const int64_t o = real ? row_off(a, b, h, f, a.dk) : 0;
@@ -470,24 +476,24 @@ __global__ void __launch_bounds__(NT) gla_bwd_chunk(const BwdArgs<TI> a) {
   // dK^ = A^T Q~ + V D^T (MC x dk, blocks 0 .. nk-1) and dV = P^T dO + K^ D (MC x dv,
   // blocks nk .. nk+nv-1)
   {
-    const int nck = a.dk / 8, ncv = a.dv / 8, nk = (MC / 4) * nck, nv = (MC / 4) * ncv;
+    const int nck = a.dk / 8, ncv = a.dv / 8, nk = (MC / kTR) * nck, nv = (MC / kTR) * ncv;
     for (int t = threadIdx.x; t < nk + nv; t += NT) {
       const bool isv = t >= nk;
       const int tt = isv ? t - nk : t;
       const int nc = isv ? ncv : nck;
-      const int s0 = 4 * (tt / nc), c0 = 8 * (tt % nc);
+      const int s0 = kTR * (tt / nc), c0 = 8 * (tt % nc);
       const int lo = lo_of_cols(s0), hi = hi_of_cols(s0);
-      float acc[4][8];
-      zero48(acc);
+      float acc[kTR][8];
+      zero48<kTR>(acc);
       if (!isv) {
-        mt48(acc, sA + lo * pa + s0, 1, pa, sQ + lo * pk + c0, pk, 1, hi - lo);
-        mt48(acc, sV + s0 * pv, pv, 1, sS + c0 * pv, 1, pv, a.dv);
+        mt48<kTR>(acc, sA + lo * pa + s0, 1, pa, sQ + lo * pk + c0, pk, 1, hi - lo);
+        mt48<kTR>(acc, sV + s0 * pv, pv, 1, sS + c0 * pv, 1, pv, a.dv);
       } else {
-        mt48(acc, sP + lo * pa + s0, 1, pa, sO + lo * pv + c0, pv, 1, hi - lo);
-        mt48(acc, sK + s0 * pk, pk, 1, sS + c0, pv, 1, a.dk);
+        mt48<kTR>(acc, sP + lo * pa + s0, 1, pa, sO + lo * pv + c0, pv, 1, hi - lo);
+        mt48<kTR>(acc, sK + s0 * pk, pk, 1, sS + c0, pv, 1, a.dk);
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kTR; ++i) {
         const int s2 = s0 + i, f = f0 + s2;
         const bool real = f >= 0 && f < a.g.T;
         if (!isv) {
@@ -552,19 +558,20 @@ size_t smem_chunk(const GlaShape& s) {
 template <typename TI, int MC>
 cudaError_t launch_bwd(const BwdArgs<TI>& a, const GlaShape& s, cudaStream_t st) {
   const size_t s1 = smem_local<MC>(s), s3 = smem_chunk<MC>(s);
+  const bool two_rows = (MC / 2) * (s.dk / 8 + s.dv / 8) <= NT;
+  auto chunk_kernel = two_rows ? gla_bwd_chunk<TI, MC, 2> : gla_bwd_chunk<TI, MC, 4>;
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(gla_bwd_local<TI, MC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1)) !=
       cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(gla_bwd_chunk<TI, MC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3)) !=
-      cudaSuccess)
+  if ((e = cudaFuncSetAttribute(chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3)) != cudaSuccess)
     return e;
   const dim3 grid(a.NC, s.B * s.H);
   gla_bwd_local<TI, MC><<<grid, NT, s1, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   gla_bwd_scan<TI><<<dim3((s.dk * s.dv + 255) / 256, s.B * s.H), 256, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  gla_bwd_chunk<TI, MC><<<grid, NT, s3, st>>>(a);
+  chunk_kernel<<<grid, NT, s3, st>>>(a);
   return cudaGetLastError();
 }
 
