@@ -130,6 +130,19 @@ __device__ __forceinline__ void zero48(float (&acc)[R][8]) {
 
 
 
+// carry[i] = sum_j D[i][j] S_out[i][j] for i < dk (both [dk][dv] fp32 rows in global
+// memory): one warp per row i, lanes over j (coalesced), a fixed shuffle-tree sum.
+__device__ __forceinline__ void chunk_carry(const float* D, const float* Sout, int dk, int dv, float* carry) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int i = warp; i < dk; i += nw) {
+    float acc = 0.f;
+    for (int j = lane; j < dv; j += 32) acc = fmaf(D[(size_t)i * dv + j], Sout[(size_t)i * dv + j], acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) carry[i] = acc;
+  }
+}
+
 // Threads i < dk: the log-gate tile becomes, in place, the exclusive suffix sums u
 // along the scan order; the chunk total goes to sTot[i].  Returns bit 1 if |u| or
 // the total leave the fp32-safe range (evaluate token by token), bit 2 if growth
@@ -513,14 +526,7 @@ __global__ void __launch_bounds__(NT) gla_bwd_chunk(const BwdArgs<TI> a) {
     }
   }
   // gradient of a gate at the chunk's end: sum_j D[i][j] S_in(c+1)[i][j]
-  {
-    const float* sout = a.sx + cid * st;
-    for (int i = threadIdx.x; i < a.dk; i += NT) {
-      float acc = 0.f;
-      for (int j = 0; j < a.dv; ++j) acc = fmaf(sS[i * pv + j], sout[(size_t)i * a.dv + j], acc);
-      sCarry[i] = acc;
-    }
-  }
+  chunk_carry(a.dd + cid * st, a.sx + cid * st, a.dk, a.dv, sCarry);
   __syncthreads();
   // dlog_alpha_r = carry + sum of db over the chunk's positions at or after r
   for (int i = threadIdx.x; i < a.dk; i += NT) {
@@ -533,6 +539,385 @@ __global__ void __launch_bounds__(NT) gla_bwd_chunk(const BwdArgs<TI> a) {
     }
   }
 }
+
+// ---------------------------------------------------------------------------
+// Kernel 3 on tensor cores (bf16 inputs, dk and dv at most 80): chunks of 128 rows,
+// one CTA per chunk, every product a tcgen05 MMA (M = 128) from bf16 tiles in shared
+// memory into fp32 TMEM accumulators:
+//   A = dO V^T, P = Q~ K^^T                     (then masked and rounded to bf16)
+//   dQ~ = dO G^T + A K^,  dK^ = A^T Q~ + V D^T,  dV = P^T dO + K^ D
+// Tiles use the 32-byte swizzle in 16-channel blocks of `rows` rows; one tile serves as
+// a K-major operand (rows = M or N, K = channels) and, transposed, as an MN-major one
+// (K = rows).  The masked A and P are written back to shared memory once and read both
+// ways.  Chunks flagged by kernel 1 take an exact token-by-token sweep instead.
+// ---------------------------------------------------------------------------
+constexpr int kTcRows = 128;
+constexpr uint32_t kLayoutSW32b = 6;  // UMMA layout type of the 32-byte swizzle
+
+__device__ __forceinline__ uint32_t sw32_at(uint32_t rows, uint32_t r, uint32_t ch) {
+  return (ch >> 4) * (rows * 32u) + r * 32u + (((((ch >> 3) & 1u) ^ (r >> 2)) & 1u) << 4) + (ch & 7u) * 2u;
+}
+// K-major operand of a tile with `rows` rows: K step kk = channels 16kk..16kk+15.
+__device__ __forceinline__ uint64_t dkm(uint32_t tile, uint32_t rows, int kk) {
+  return umma_desc(tile + (uint32_t)kk * rows * 32u, 16u, 256u, kLayoutSW32b);
+}
+// MN-major operand (MN = channels, K = rows) of a tile with `rows` rows: K step kk =
+// rows 16kk..16kk+15.
+__device__ __forceinline__ uint64_t dmn(uint32_t tile, uint32_t rows, int kk) {
+  return umma_desc(tile + (uint32_t)kk * 512u, rows * 32u, 256u, kLayoutSW32b);
+}
+
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) { tmem_ld16(taddr, v); }
+
+// Exact sweep of a flagged chunk from fp32 tiles (alpha, k, v) staged in shared
+// memory; q and dout rows are read from global memory one position at a time.
+__device__ void tc_chunk_serial(const BwdArgs<__nv_bfloat16>& a, float* smem, int c, int b, int h, int f0) {
+  constexpr int MC = kTcRows;
+  const int pk = pitch_of(a.dk), pv = pitch_of(a.dv);
+  float* sAl = smem;                 // [MC][pk] alpha
+  float* sK = sAl + MC * pk;         // [MC][pk]
+  float* sV = sK + MC * pk;          // [MC][pv]
+  float* sGg = sV + MC * pv;         // [dk][pv] gradient of the state
+  float* sW = sGg + a.dk * pv;       // [dk][pv] S_{r-1}
+  stage<MC>(sAl, a.la, a.dk, a.g, f0, b, h, a.H);
+  stage<MC>(sK, a.k, a.dk, a.g, f0, b, h, a.H);
+  stage<MC>(sV, a.v, a.dv, a.g, f0, b, h, a.H);
+  const int64_t cid = (int64_t)blockIdx.y * a.NC + c;
+  const size_t st = (size_t)a.dk * a.dv;
+  const float* sin = c > 0 ? a.sx + (cid - 1) * st : nullptr;
+  const float* dd = a.dd + cid * st;
+  for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+    const int i = e / a.dv, j = e - i * a.dv;
+    sGg[i * pv + j] = dd[e];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
+    const int r = e / a.dk, i = e - r * a.dk;
+    sAl[r * pk + i] = expf(sAl[r * pk + i]);
+  }
+  __syncthreads();
+  for (int step = MC - 1; step >= 0; --step) {
+    const int r = a.g.reverse ? (MC - 1 - step) : step;
+    const int f = f0 + r;
+    const bool real = f >= 0 && f < a.g.T;
+    const int64_t ok = real ? row_off(a, b, h, f, a.dk) : 0;
+    const int64_t ov = real ? row_off(a, b, h, f, a.dv) : 0;
+    for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+      const int i = e / a.dv, j = e - i * a.dv;
+      float w = sin ? sin[e] : 0.f;
+      for (int s2 = 0; s2 < step; ++s2) {
+        const int r2 = a.g.reverse ? (MC - 1 - s2) : s2;
+        w = fmaf(sAl[r2 * pk + i], w, sK[r2 * pk + i] * sV[r2 * pv + j]);
+      }
+      sW[i * pv + j] = w;
+      if (real) {
+        const float qi = __bfloat162float(a.q[ok + i]), oj = __bfloat162float(a.dout[ov + j]);
+        sGg[i * pv + j] = fmaf(qi, oj, sGg[i * pv + j]);
+      }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < a.dk; i += NT) {
+      const float al = sAl[r * pk + i], ki = sK[r * pk + i];
+      float gq = 0.f, gk = 0.f, gl = 0.f;
+      for (int j = 0; j < a.dv; ++j) {
+        const float sr = fmaf(al, sW[i * pv + j], ki * sV[r * pv + j]);
+        if (real) gq = fmaf(__bfloat162float(a.dout[ov + j]), sr, gq);
+        gk = fmaf(sGg[i * pv + j], sV[r * pv + j], gk);
+        gl = fmaf(sGg[i * pv + j], sW[i * pv + j], gl);
+      }
+      if (real) {
+        store1(a.dq + ok + i, gq);
+        store1(a.dk_out + ok + i, gk);
+        a.dla[ok + i] = al * gl;
+      }
+    }
+    for (int j = threadIdx.x; j < a.dv; j += NT) {
+      float gv = 0.f;
+      for (int i = 0; i < a.dk; ++i) gv = fmaf(sK[r * pk + i], sGg[i * pv + j], gv);
+      if (real) store1(a.dv_out + ov + j, gv);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+      const int i = e / a.dv, j = e - i * a.dv;
+      sGg[i * pv + j] *= sAl[r * pk + i];
+    }
+    __syncthreads();
+  }
+}
+
+struct TcLayout {
+  uint32_t oQ, oK, oV, oO, oA, oP, oG, oD, oU, oMisc, bytes;
+};
+__host__ __device__ inline TcLayout tc_layout(int dk, int dv) {
+  const uint32_t Kp = (uint32_t)(dk + 15) / 16 * 16, Np = (uint32_t)(dv + 15) / 16 * 16;
+  TcLayout L;
+  L.oQ = 0;
+  L.oK = L.oQ + Kp / 16 * kTcRows * 32u;
+  L.oV = L.oK + Kp / 16 * kTcRows * 32u;
+  L.oO = L.oV + Np / 16 * kTcRows * 32u;
+  L.oA = L.oO + Np / 16 * kTcRows * 32u;
+  L.oP = L.oA + 8u * kTcRows * 32u;
+  L.oG = L.oP + 8u * kTcRows * 32u;
+  L.oD = L.oG + (Np / 16) * Kp * 32u;
+  L.oU = L.oD + (Np / 16) * Kp * 32u;
+  L.oMisc = (L.oU + (uint32_t)kTcRows * (uint32_t)(dk + 1) * 4u + 15u) / 16u * 16u;
+  L.bytes = L.oMisc + 1024u + 64u + 1024u;  // gate totals, carry, barrier, TMEM address; alignment slack
+  return L;
+}
+
+__global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfloat16> a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw_tc[];
+  // Swizzled operand tiles start on a 1024-byte boundary.
+  uint8_t* smem_tc = smem_raw_tc + ((1024u - (smem_u32(smem_raw_tc) & 1023u)) & 1023u);
+  constexpr int MC = kTcRows;
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const TcLayout L = tc_layout(a.dk, a.dv);
+  const uint32_t Kp = (uint32_t)(a.dk + 15) / 16 * 16, Np = (uint32_t)(a.dv + 15) / 16 * 16;
+  const uint32_t sb = smem_u32(smem_tc);
+  float* sU = reinterpret_cast<float*>(smem_tc + L.oU);   // [MC][dk+1]: log-gates, u, then db
+  float* sTot = reinterpret_cast<float*>(smem_tc + L.oMisc);
+  float* sCarry = sTot + 128;
+  uint64_t* sBar = reinterpret_cast<uint64_t*>(sCarry + 128);
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(sBar + 1);
+  const int pu = a.dk + 1;
+  const int f0 = chunk_first_base_pos(a.g, c, MC);
+  const int64_t cid = (int64_t)bh * a.NC + c;
+  const bool rev = a.g.reverse;
+
+  if (a.flags[cid]) {
+    tc_chunk_serial(a, reinterpret_cast<float*>(smem_tc), c, b, h, f0);
+    return;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) {
+    tmem_alloc(smem_u32(sTmem), 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(sBar), 1);
+    fence_mbar_init();
+  }
+  // ---- staging: log-gates (fp32), q, k, v, dout (bf16, swizzled, zero past the
+  // channels and rows), G = Diag(e^g) S_in and D (bf16, [Kp][Np] tiles)
+  stage<MC>(sU, a.la, a.dk, a.g, f0, b, h, a.H);
+  {
+    const int cq = (int)Kp / 8, cv = (int)Np / 8;
+    for (int idx = threadIdx.x; idx < MC * (2 * cq + 2 * cv); idx += NT) {
+      const int r = idx % MC, w = idx / MC;  // consecutive threads: consecutive rows
+      int which, cc;
+      if (w < cq) which = 0, cc = w;
+      else if (w < 2 * cq) which = 1, cc = w - cq;
+      else if (w < 2 * cq + cv) which = 2, cc = w - 2 * cq;
+      else which = 3, cc = w - 2 * cq - cv;
+      const int d = which < 2 ? a.dk : a.dv;
+      const __nv_bfloat16* src = which == 0 ? a.q : which == 1 ? a.k : which == 2 ? a.v : a.dout;
+      const uint32_t tile = which == 0 ? L.oQ : which == 1 ? L.oK : which == 2 ? L.oV : L.oO;
+      const int f = f0 + r;
+      uint4 val = make_uint4(0u, 0u, 0u, 0u);
+      if (f >= 0 && f < a.g.T && cc * 8 < d)
+        val = *reinterpret_cast<const uint4*>(src + row_off(a, b, h, f, d) + cc * 8);
+      *reinterpret_cast<uint4*>(smem_tc + tile + sw32_at(MC, (uint32_t)r, (uint32_t)(cc * 8))) = val;
+    }
+  }
+  __syncthreads();
+  suffix_sums<MC>(sU, sTot, a.dk, rev);
+  __syncthreads();
+  {
+    const size_t st = (size_t)a.dk * a.dv;
+    const float* sin = c > 0 ? a.sx + (cid - 1) * st : nullptr;
+    const float* dd = a.dd + cid * st;
+    // Q~ = q e^{-u}, K^ = k e^{u} in place (8 channels per thread), padding stays 0
+    const int cq = (int)Kp / 8;
+    for (int idx = threadIdx.x; idx < MC * cq; idx += NT) {
+      const int r = idx % MC, cc = idx / MC;
+      if (cc * 8 >= a.dk) continue;
+      uint4* pq = reinterpret_cast<uint4*>(smem_tc + L.oQ + sw32_at(MC, (uint32_t)r, (uint32_t)(cc * 8)));
+      uint4* pk = reinterpret_cast<uint4*>(smem_tc + L.oK + sw32_at(MC, (uint32_t)r, (uint32_t)(cc * 8)));
+      uint4 wq = *pq, wk = *pk;
+      uint32_t* uq = reinterpret_cast<uint32_t*>(&wq);
+      uint32_t* uk = reinterpret_cast<uint32_t*>(&wk);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float u0 = sU[r * pu + cc * 8 + 2 * e], u1 = sU[r * pu + cc * 8 + 2 * e + 1];
+        const float2 xq = unpack_bf16x2(uq[e]), xk = unpack_bf16x2(uk[e]);
+        uq[e] = pack_bf16x2(xq.x * expf(-u0), xq.y * expf(-u1));
+        uk[e] = pack_bf16x2(xk.x * expf(u0), xk.y * expf(u1));
+      }
+      *pq = wq;
+      *pk = wk;
+    }
+    // G[i][j] = e^{g_i} S_in[i][j] and D[i][j], bf16, rows i < Kp, channels j < Np
+    for (int e = threadIdx.x; e < (int)(Kp * Np); e += NT) {
+      const int i = e / (int)Np, j = e - i * (int)Np;
+      float gv = 0.f, dv_ = 0.f;
+      if (i < a.dk && j < a.dv) {
+        const size_t o = (size_t)i * a.dv + j;
+        gv = sin ? expf(sTot[i]) * sin[o] : 0.f;
+        dv_ = dd[o];
+      }
+      *reinterpret_cast<__nv_bfloat16*>(smem_tc + L.oG + sw32_at(Kp, (uint32_t)i, (uint32_t)j)) =
+          __float2bfloat16_rn(gv);
+      *reinterpret_cast<__nv_bfloat16*>(smem_tc + L.oD + sw32_at(Kp, (uint32_t)i, (uint32_t)j)) =
+          __float2bfloat16_rn(dv_);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *sTmem;
+  const uint32_t cA = 0, cP = 128, cDQ = 256, cDK = 256 + Kp, cDV = 256 + 2 * Kp;
+  const uint32_t bar = smem_u32(sBar);
+  bool ok = true;
+  // ---- A = dO V^T, P = Q~ K^^T
+  if (threadIdx.x == 0) {
+    const uint32_t idS = idesc_bf16_f32(MC, MC, false, false);
+    for (int kk = 0; kk < (int)Np / 16; ++kk)
+      umma_ss(tbase + cA, dkm(sb + L.oO, MC, kk), dkm(sb + L.oV, MC, kk), idS, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < (int)Kp / 16; ++kk)
+      umma_ss(tbase + cP, dkm(sb + L.oQ, MC, kk), dkm(sb + L.oK, MC, kk), idS, kk > 0 ? 1u : 0u);
+    umma_commit(bar);
+  }
+  ok = __syncthreads_and(mbar_wait(bar, 0u));
+  if (!ok && threadIdx.x == 0) report_status(GLA_ERR_TIMEOUT);
+  tc_fence_after();
+  // ---- mask and round: lane = row r (TMEM lane), warp pair splits the 128 columns
+  const int qd = warp & 3, hf = warp >> 2;
+  const int r = 32 * qd + lane;
+  const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
+  if (ok) {
+    for (int which = 0; which < 2; ++which) {
+      const uint32_t col = which ? cP : cA;
+      const uint32_t tile = which ? L.oP : L.oA;
+      for (int g = 0; g < 4; ++g) {
+        const int s0 = 64 * hf + 16 * g;
+        float x[16];
+        tc_ld16(tbase + lane_base + col + (uint32_t)s0, x);
+        uint32_t w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int sa = s0 + 2 * e, sbb = sa + 1;
+          const float x0 = (rev ? sa >= r : sa <= r) ? x[2 * e] : 0.f;
+          const float x1 = (rev ? sbb >= r : sbb <= r) ? x[2 * e + 1] : 0.f;
+          w[e] = pack_bf16x2(x0, x1);
+        }
+        *reinterpret_cast<uint4*>(smem_tc + tile + sw32_at(MC, (uint32_t)r, (uint32_t)s0)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(smem_tc + tile + sw32_at(MC, (uint32_t)r, (uint32_t)(s0 + 8))) =
+            make_uint4(w[4], w[5], w[6], w[7]);
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // ---- dQ~ = dO G^T + A K^,  dK^ = A^T Q~ + V D^T,  dV = P^T dO + K^ D
+  if (threadIdx.x == 0 && ok) {
+    const uint32_t idKK = idesc_bf16_f32(MC, (int)Kp, false, false);  // both K-major
+    const uint32_t idKM = idesc_bf16_f32(MC, (int)Kp, false, true);   // B MN-major
+    const uint32_t idMM = idesc_bf16_f32(MC, (int)Kp, true, true);    // both MN-major
+    const uint32_t idVM = idesc_bf16_f32(MC, (int)Np, true, true);
+    const uint32_t idVK = idesc_bf16_f32(MC, (int)Np, false, true);   // A K-major, B MN-major
+    for (int kk = 0; kk < (int)Np / 16; ++kk)
+      umma_ss(tbase + cDQ, dkm(sb + L.oO, MC, kk), dkm(sb + L.oG, Kp, kk), idKK, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < MC / 16; ++kk)
+      umma_ss(tbase + cDQ, dkm(sb + L.oA, MC, kk), dmn(sb + L.oK, MC, kk), idKM, 1u);
+    for (int kk = 0; kk < MC / 16; ++kk)
+      umma_ss(tbase + cDK, dmn(sb + L.oA, MC, kk), dmn(sb + L.oQ, MC, kk), idMM, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < (int)Np / 16; ++kk)
+      umma_ss(tbase + cDK, dkm(sb + L.oV, MC, kk), dkm(sb + L.oD, Kp, kk), idKK, 1u);
+    for (int kk = 0; kk < MC / 16; ++kk)
+      umma_ss(tbase + cDV, dmn(sb + L.oP, MC, kk), dmn(sb + L.oO, MC, kk), idVM, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < (int)Kp / 16; ++kk)
+      umma_ss(tbase + cDV, dkm(sb + L.oK, MC, kk), dmn(sb + L.oD, Kp, kk), idVK, 1u);
+    umma_commit(bar);
+  }
+  if (ok) {
+    ok = __syncthreads_and(mbar_wait(bar, 1u));
+    if (!ok && threadIdx.x == 0) report_status(GLA_ERR_TIMEOUT);
+  }
+  tc_fence_after();
+  // ---- epilogue: row r, 16-channel groups g with g % 2 == hf
+  const int f = f0 + r;
+  const bool real = f >= 0 && f < a.g.T;
+  if (ok) {
+    // q dq - k dk = Q~ dQ~ - K^ dK^, with Q~ and K^ the bf16 tiles of the MMAs.
+    const int64_t ok_ = real ? row_off(a, b, h, f, a.dk) : 0;
+    for (int g = hf; g < (int)Kp / 16; g += 2) {
+      float xq[16], xk[16];
+      tc_ld16(tbase + lane_base + cDQ + (uint32_t)(16 * g), xq);
+      tc_ld16(tbase + lane_base + cDK + (uint32_t)(16 * g), xk);
+      for (int half = 0; half < 2; ++half) {
+        const int i0 = 16 * g + 8 * half;
+        if (i0 >= a.dk) break;
+        const uint4 wq = *reinterpret_cast<const uint4*>(smem_tc + L.oQ + sw32_at(MC, (uint32_t)r, (uint32_t)i0));
+        const uint4 wk = *reinterpret_cast<const uint4*>(smem_tc + L.oK + sw32_at(MC, (uint32_t)r, (uint32_t)i0));
+        const uint32_t* uq = reinterpret_cast<const uint32_t*>(&wq);
+        const uint32_t* uk = reinterpret_cast<const uint32_t*>(&wk);
+        uint32_t pq[4], pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = i0 + 2 * e;
+          const float2 tq = unpack_bf16x2(uq[e]), tk = unpack_bf16x2(uk[e]);
+          const float a0 = xq[8 * half + 2 * e], a1 = xq[8 * half + 2 * e + 1];
+          const float b0 = xk[8 * half + 2 * e], b1 = xk[8 * half + 2 * e + 1];
+          const float u0 = sU[r * pu + i], u1 = sU[r * pu + i + 1];
+          pq[e] = pack_bf16x2(expf(-u0) * a0, expf(-u1) * a1);
+          pk[e] = pack_bf16x2(expf(u0) * b0, expf(u1) * b1);
+          sU[r * pu + i] = real ? tq.x * a0 - tk.x * b0 : 0.f;
+          sU[r * pu + i + 1] = real ? tq.y * a1 - tk.y * b1 : 0.f;
+        }
+        if (real) {
+          *reinterpret_cast<uint4*>(a.dq + ok_ + i0) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
+          *reinterpret_cast<uint4*>(a.dk_out + ok_ + i0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+    }
+    const int64_t ov_ = real ? row_off(a, b, h, f, a.dv) : 0;
+    for (int g = hf; g < (int)Np / 16; g += 2) {
+      float xv[16];
+      tc_ld16(tbase + lane_base + cDV + (uint32_t)(16 * g), xv);
+      for (int half = 0; half < 2; ++half) {
+        const int j0 = 16 * g + 8 * half;
+        if (j0 >= a.dv || !real) break;
+        *reinterpret_cast<uint4*>(a.dv_out + ov_ + j0) =
+            make_uint4(pack_bf16x2(xv[8 * half], xv[8 * half + 1]), pack_bf16x2(xv[8 * half + 2], xv[8 * half + 3]),
+                       pack_bf16x2(xv[8 * half + 4], xv[8 * half + 5]), pack_bf16x2(xv[8 * half + 6], xv[8 * half + 7]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (!ok && threadIdx.x == 0) {
+    // A wait ran out: let every MMA issued so far complete (bounded) before TMEM goes.
+    umma_commit(bar);
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, 0u) && !mbar_try_wait(bar, 1u) && clock64() - t0 < kWaitCycles) {
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tbase, 512);
+  if (!ok) return;
+  {
+    const size_t st = (size_t)a.dk * a.dv;
+    chunk_carry(a.dd + cid * st, a.sx + cid * st, a.dk, a.dv, sCarry);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < a.dk; i += NT) {
+    float acc = sCarry[i];
+    for (int step = MC - 1; step >= 0; --step) {
+      const int rr = rev ? (MC - 1 - step) : step;
+      acc += sU[rr * pu + i];
+      const int ff = f0 + rr;
+      if (ff >= 0 && ff < a.g.T) a.dla[row_off(a, b, h, ff, a.dk) + i] = acc;
+    }
+  }
+}
+
+bool use_tc(const GlaShape& s, int bf16) { return bf16 && s.dk <= 80 && s.dv <= 80; }
 
 size_t rup(size_t x, size_t m) { return (x + m - 1) / m * m; }
 
@@ -575,6 +960,26 @@ cudaError_t launch_bwd(const BwdArgs<TI>& a, const GlaShape& s, cudaStream_t st)
   return cudaGetLastError();
 }
 
+// The tensor-core path: kernels 1 and 2 with 128-row chunks, then gla_bwd_tc_chunk.
+cudaError_t launch_bwd_tc(const BwdArgs<__nv_bfloat16>& a, const GlaShape& s, cudaStream_t st) {
+  const size_t s1 = smem_local<kTcRows>(s);
+  const TcLayout L = tc_layout(s.dk, s.dv);
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(gla_bwd_local<__nv_bfloat16, kTcRows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)s1)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(gla_bwd_tc_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.bytes)) !=
+      cudaSuccess)
+    return e;
+  const dim3 grid(a.NC, s.B * s.H);
+  gla_bwd_local<__nv_bfloat16, kTcRows><<<grid, NT, s1, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  gla_bwd_scan<__nv_bfloat16><<<dim3((s.dk * s.dv + 255) / 256, s.B * s.H), 256, 0, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  gla_bwd_tc_chunk<<<grid, NT, L.bytes, st>>>(a);
+  return cudaGetLastError();
+}
+
 template <typename TI>
 cudaError_t run_bwd(const void* q, const void* k, const void* v, const float* la, const void* dout, void* dq,
                     void* dk, void* dv, float* dla, const GlaShape& s, void* workspace, cudaStream_t st) {
@@ -591,7 +996,8 @@ cudaError_t run_bwd(const void* q, const void* k, const void* v, const float* la
   a.H = s.H;
   a.dk = s.dk;
   a.dv = s.dv;
-  const int MC = chunk_rows(s);
+  const bool tc = use_tc(s, sizeof(TI) == 2);
+  const int MC = tc ? kTcRows : chunk_rows(s);
   a.NC = (s.T() + MC - 1) / MC;
   a.g = make_geom(s.Hg, s.Wg, s.dir);
   const size_t BH = (size_t)s.B * s.H;
@@ -601,6 +1007,9 @@ cudaError_t run_bwd(const void* q, const void* k, const void* v, const float* la
   a.dd = reinterpret_cast<float*>(ws + big);
   a.gamma = reinterpret_cast<float*>(ws + 2 * big);
   a.flags = reinterpret_cast<int*>(ws + 2 * big + rup(BH * a.NC * s.dk * 4, 256));
+  if constexpr (sizeof(TI) == 2) {
+    if (tc) return launch_bwd_tc(a, s, st);
+  }
   return MC == 64 ? launch_bwd<TI, 64>(a, s, st) : launch_bwd<TI, 32>(a, s, st);
 }
 

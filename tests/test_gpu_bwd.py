@@ -1,14 +1,14 @@
 """GPU parity of the GLA backward (gla_bwd, gla_bwd_f32) against the fp64 oracle's
 reverse sweep (oracle.gla_bwd), through the C ABI.
 
-The pages state no tolerance for the backward.  The kernels do every product and
-sum in fp32 from inputs that both sides read exactly, so:
-  * fp32 outputs (gla_bwd_f32's dq, dk, dv and both entry points' dlog_alpha): the
-    GLA path's fp32 bar, max-abs error <= 1e-4, and a relative RMS error <= 1e-4
-    per (batch, head) (fp32 rounding over a few hundred terms, with margin);
-  * bf16 dq, dk, dv: every element within 2^-8 |oracle| + 1e-3 RMS(head) (the
-    store's rounding to bf16, half an ulp of an 8-bit significand, plus the fp32
-    arithmetic), and a relative RMS error <= 2e-2 per (batch, head) (the bf16 bar).
+The pages state no tolerance for the backward; the gates follow its arithmetic:
+  * gla_bwd_f32 (fp32 inputs, every product and sum in fp32 on CUDA cores): the GLA
+    path's fp32 bar, max-abs error <= 1e-4, and a relative RMS error <= 1e-4 per
+    (batch, head) (fp32 rounding over a few hundred terms, with margin);
+  * gla_bwd (bf16 inputs; for dk, dv <= 80 the chunk products run on tensor cores
+    from bf16 operands Q~, K^, A, P, G, D with fp32 accumulation): the forward's bf16
+    gates on all four outputs -- relative RMS error <= 2e-2 per (batch, head), every
+    element within 2^-8 |oracle| + 0.1 RMS(head).
 Inputs: workloads.gla_inputs and workloads.gla_dout (seeded, synthetic).
 """
 import math
@@ -26,7 +26,7 @@ F32_MAX_ABS = 1e-4
 F32_REL_RMS = 1e-4
 BF16_REL_RMS = 2e-2
 BF16_ELT_REL = 2.0 ** -8
-BF16_ELT_RMS = 1e-3
+BF16_ELT_RMS = 0.1
 NAMES = ("dq", "dk", "dv", "dlog_alpha")
 
 
@@ -41,7 +41,7 @@ def per_head(a):
     return a.transpose(0, 2, 1, 3).reshape(B * H, T, d)
 
 
-def check(got, ref, name, bf16_store):
+def check(got, ref, name, bf16_store, elt_rms=BF16_ELT_RMS):
     assert np.all(np.isfinite(got)), name
     g, r = per_head(got), per_head(ref)
     for h in range(g.shape[0]):
@@ -50,7 +50,7 @@ def check(got, ref, name, bf16_store):
         rel = float(np.linalg.norm(err) / max(np.linalg.norm(r[h]), 1e-300))
         if bf16_store:
             assert rel <= BF16_REL_RMS, f"{name} head {h}: relative RMS {rel:.3e}"
-            bound = BF16_ELT_REL * np.abs(r[h]) + BF16_ELT_RMS * rms
+            bound = BF16_ELT_REL * np.abs(r[h]) + elt_rms * rms
             worst = float(np.max(np.abs(err) - bound)) if err.size else -1.0
             assert worst <= 0.0, f"{name} head {h}: element bound exceeded by {worst:.3e} (RMS {rms:.3e})"
         else:
@@ -72,13 +72,13 @@ def run_case(dig, w, direction, seed=0, la=None, heads=None):
     if heads is None:
         ref = oracle.gla_bwd(q, k, v, la, do, w.Hgrid, w.Wgrid, direction)
         for g, r, n in zip(got, ref, NAMES):
-            check(g, r, n, w.dtype == "bf16" and n != "dlog_alpha")
+            check(g, r, n, w.dtype == "bf16")
         return got, ref
     for lo, hi in heads:
         ref = oracle.gla_bwd(q, k, v, la, do, w.Hgrid, w.Wgrid, direction, nthreads=1, heads=(lo, hi))
         for g, r, n in zip(got, ref, NAMES):
             check(per_head(g)[lo:hi][None].transpose(0, 2, 1, 3), per_head(r)[lo:hi][None].transpose(0, 2, 1, 3),
-                  f"{n} heads {lo}:{hi}", w.dtype == "bf16" and n != "dlog_alpha")
+                  f"{n} heads {lo}:{hi}", w.dtype == "bf16")
     return got, None
 
 

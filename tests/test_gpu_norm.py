@@ -35,7 +35,7 @@ def run(dig, w, direction, seed=0, scale=None, eps=EPS, q_shift=0.0):
     assert dig.device_status() == 0
     got = got.float().cpu().numpy().astype(np.float64)
     ref = oracle.gla_norm_fwd(q, k, v, w.Hgrid, w.Wgrid, direction, eps=eps)
-    check(got, ref, f"norm dir {direction}", w.dtype == "bf16")
+    check(got, ref, f"norm dir {direction}", w.dtype == "bf16", elt_rms=1e-3)
     return got, ref
 
 
