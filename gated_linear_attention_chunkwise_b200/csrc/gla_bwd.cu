@@ -917,6 +917,136 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
   }
 }
 
+// Kernel 1 on tensor cores (bf16 inputs, dk and dv at most 80): per 128-row chunk,
+// K^T V and Qbar^T dO as M = 128 MMAs whose A operands are the k and q tiles read
+// MN-major (M = key channels; the tiles hold 128 channels, zero past dk).
+constexpr uint32_t kTcLocalBytes(int dk, int dv) {
+  return 2u * 8u * kTcRows * 32u + 2u * (uint32_t)((dv + 15) / 16) * kTcRows * 32u +
+         (uint32_t)kTcRows * (uint32_t)(dk + 1) * 4u + 512u + 64u + 1024u;
+}
+
+__global__ void __launch_bounds__(NT, 1) gla_bwd_tc_local(const BwdArgs<__nv_bfloat16> a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw_tl[];
+  uint8_t* sm = smem_raw_tl + ((1024u - (smem_u32(smem_raw_tl) & 1023u)) & 1023u);
+  constexpr int MC = kTcRows;
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const uint32_t Np = (uint32_t)(a.dv + 15) / 16 * 16;
+  const uint32_t oK = 0, oQ = 8u * MC * 32u, oV = 16u * MC * 32u, oO = oV + Np / 16 * MC * 32u;
+  const uint32_t oU = oO + Np / 16 * MC * 32u;
+  float* sU = reinterpret_cast<float*>(sm + oU);
+  float* sTot = sU + MC * (a.dk + 1);
+  uint64_t* sBar = reinterpret_cast<uint64_t*>(sTot + 128);
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(sBar + 1);
+  const int pu = a.dk + 1;
+  const uint32_t sb = smem_u32(sm);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool rev = a.g.reverse;
+  const int f0 = chunk_first_base_pos(a.g, c, MC);
+  if (warp == 0) {
+    tmem_alloc(smem_u32(sTmem), 256);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(sBar), 1);
+    fence_mbar_init();
+  }
+  stage<MC>(sU, a.la, a.dk, a.g, f0, b, h, a.H);
+  {
+    const int cv = (int)Np / 8;
+    for (int idx = threadIdx.x; idx < MC * (16 + 16 + 2 * cv); idx += NT) {
+      const int r = idx % MC, w = idx / MC;
+      int which, cc;
+      if (w < 16) which = 0, cc = w;
+      else if (w < 32) which = 1, cc = w - 16;
+      else if (w < 32 + cv) which = 2, cc = w - 32;
+      else which = 3, cc = w - 32 - cv;
+      const int d = which < 2 ? a.dk : a.dv;
+      const __nv_bfloat16* src = which == 0 ? a.k : which == 1 ? a.q : which == 2 ? a.v : a.dout;
+      const uint32_t tile = which == 0 ? oK : which == 1 ? oQ : which == 2 ? oV : oO;
+      const int f = f0 + r;
+      uint4 val = make_uint4(0u, 0u, 0u, 0u);
+      if (f >= 0 && f < a.g.T && cc * 8 < d)
+        val = *reinterpret_cast<const uint4*>(src + row_off(a, b, h, f, d) + cc * 8);
+      *reinterpret_cast<uint4*>(sm + tile + sw32_at(MC, (uint32_t)r, (uint32_t)(cc * 8))) = val;
+    }
+  }
+  __syncthreads();
+  // Qbar = q e^{b}: b the inclusive prefix of the log-gates in scan order, walked
+  // directly (a -inf gate gives 0, not inf - inf).
+  for (int i = threadIdx.x; i < a.dk; i += NT) {
+    float acc = 0.f;
+    for (int st = 0; st < MC; ++st) {
+      const int r = rev ? (MC - 1 - st) : st;
+      acc += sU[r * pu + i];
+      __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(sm + oQ + sw32_at(MC, (uint32_t)r, (uint32_t)i));
+      *p = __float2bfloat16_rn(__bfloat162float(*p) * expf(acc));
+    }
+  }
+  __syncthreads();
+  const int code = suffix_sums<MC>(sU, sTot, a.dk, rev);
+  if (code & 2) report_status(GLA_ERR_RANGE);
+  const int wide = __syncthreads_or(code != 0);
+  // K^ = k e^{u}: the exponent is a sum of log-gates, so decays only shrink it.
+  for (int idx = threadIdx.x; idx < MC * (a.dk / 8); idx += NT) {
+    const int r = idx % MC, cc = idx / MC;
+    uint4* pk = reinterpret_cast<uint4*>(sm + oK + sw32_at(MC, (uint32_t)r, (uint32_t)(cc * 8)));
+    uint4 wk = *pk;
+    uint32_t* uk = reinterpret_cast<uint32_t*>(&wk);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = unpack_bf16x2(uk[e]);
+      uk[e] = pack_bf16x2(x.x * expf(sU[r * pu + cc * 8 + 2 * e]), x.y * expf(sU[r * pu + cc * 8 + 2 * e + 1]));
+    }
+    *pk = wk;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *sTmem;
+  const uint32_t bar = smem_u32(sBar);
+  if (threadIdx.x == 0) {
+    const uint32_t id = idesc_bf16_f32(MC, (int)Np, true, true);
+    for (int kk = 0; kk < MC / 16; ++kk)
+      umma_ss(tbase, dmn(sb + oK, MC, kk), dmn(sb + oV, MC, kk), id, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < MC / 16; ++kk)
+      umma_ss(tbase + 128, dmn(sb + oQ, MC, kk), dmn(sb + oO, MC, kk), id, kk > 0 ? 1u : 0u);
+    umma_commit(bar);
+  }
+  const bool ok = __syncthreads_and(mbar_wait(bar, 0u));
+  if (!ok && threadIdx.x == 0) report_status(GLA_ERR_TIMEOUT);
+  tc_fence_after();
+  // TMEM lane = key channel i; warps 0-3 write K^T V, warps 4-7 Qbar^T dO.
+  const int64_t cid = (int64_t)bh * a.NC + c;
+  if (ok) {
+    const int i = 32 * (warp & 3) + lane;
+    const uint32_t col = (warp >> 2) ? 128u : 0u;
+    float* dst = ((warp >> 2) ? a.dd : a.sx) + cid * a.dk * a.dv + (size_t)i * a.dv;
+    for (int g = 0; g < (int)Np / 16; ++g) {
+      float x[16];
+      tmem_ld16(tbase + ((uint32_t)(32 * (warp & 3)) << 16) + col + (uint32_t)(16 * g), x);
+      if (i < a.dk)
+        for (int q4 = 0; q4 < 4; ++q4)
+          if (16 * g + 4 * q4 < a.dv)
+            *reinterpret_cast<float4*>(dst + 16 * g + 4 * q4) =
+                make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
+    }
+  }
+  if (threadIdx.x < a.dk) a.gamma[cid * a.dk + threadIdx.x] = expf(sTot[threadIdx.x]);
+  if (threadIdx.x == 0) a.flags[cid] = wide;
+  tc_fence_before();
+  __syncthreads();
+  if (!ok && threadIdx.x == 0) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, 0u) && clock64() - t0 < kWaitCycles) {
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tbase, 256);
+}
+
 bool use_tc(const GlaShape& s, int bf16) { return bf16 && s.dk <= 80 && s.dv <= 80; }
 
 size_t rup(size_t x, size_t m) { return (x + m - 1) / m * m; }
@@ -960,19 +1090,20 @@ cudaError_t launch_bwd(const BwdArgs<TI>& a, const GlaShape& s, cudaStream_t st)
   return cudaGetLastError();
 }
 
-// The tensor-core path: kernels 1 and 2 with 128-row chunks, then gla_bwd_tc_chunk.
+// The tensor-core path: gla_bwd_tc_local, the chunk scans over 128-row chunks, then
+// gla_bwd_tc_chunk.
 cudaError_t launch_bwd_tc(const BwdArgs<__nv_bfloat16>& a, const GlaShape& s, cudaStream_t st) {
-  const size_t s1 = smem_local<kTcRows>(s);
+  const size_t s1 = kTcLocalBytes(s.dk, s.dv);
   const TcLayout L = tc_layout(s.dk, s.dv);
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(gla_bwd_local<__nv_bfloat16, kTcRows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)s1)) != cudaSuccess)
+  if ((e = cudaFuncSetAttribute(gla_bwd_tc_local, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1)) !=
+      cudaSuccess)
     return e;
   if ((e = cudaFuncSetAttribute(gla_bwd_tc_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.bytes)) !=
       cudaSuccess)
     return e;
   const dim3 grid(a.NC, s.B * s.H);
-  gla_bwd_local<__nv_bfloat16, kTcRows><<<grid, NT, s1, st>>>(a);
+  gla_bwd_tc_local<<<grid, NT, s1, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   gla_bwd_scan<__nv_bfloat16><<<dim3((s.dk * s.dv + 255) / 256, s.B * s.H), 256, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
