@@ -148,11 +148,11 @@ __device__ __forceinline__ void chunk_carry(const float* D, const float* Sout, i
 // the total leave the fp32-safe range (evaluate token by token), bit 2 if growth
 // gates exceed it (not representable).
 template <int MC>
-__device__ __forceinline__ int suffix_sums(float* sU, float* sTot, int dk, int reverse) {
+__device__ __forceinline__ int suffix_sums(float* sU, float* sTot, int dk, int reverse, int pw_ = 0) {
   const int i = threadIdx.x;
   int code = 0;
   if (i < dk) {
-    const int pw = pitch_of(dk);
+    const int pw = pw_ ? pw_ : pitch_of(dk);
     float acc = 0.f, lo = 0.f, hi = 0.f;
     for (int s = 0; s < MC; ++s) {
       const int r = reverse ? s : (MC - 1 - s);
@@ -569,6 +569,35 @@ __device__ __forceinline__ uint64_t dmn(uint32_t tile, uint32_t rows, int kk) {
 
 __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) { tmem_ld16(taddr, v); }
 
+// Asynchronous staging of rows f0 .. f0+127 (zero outside the sequence and past d):
+// bf16 operand tiles in the 32-byte-swizzled layout (`nch` channels, a multiple of 8)
+// and the fp32 log-gate tile with a pitch of dk + 4 floats.  Every 16-byte copy of the
+// CTA is in flight at once; the caller waits with cp_async_wait_all and a barrier.
+template <typename TI>
+__device__ __forceinline__ void tc_stage_bf16(uint8_t* sm, uint32_t tile, const __nv_bfloat16* src, int d, int nch,
+                                              const BwdArgs<TI>& a, int f0, int b, int h) {
+  const int cc_n = nch / 8;
+  for (int idx = threadIdx.x; idx < kTcRows * cc_n; idx += NT) {
+    const int r = idx % kTcRows, cc = idx / kTcRows;
+    const int f = f0 + r;
+    const bool valid = f >= 0 && f < a.g.T && cc * 8 < d;
+    const __nv_bfloat16* p = valid ? src + row_off(a, b, h, f, d) + cc * 8 : src;
+    cp_async16(smem_u32(sm + tile + sw32_at(kTcRows, (uint32_t)r, (uint32_t)(cc * 8))), p, valid);
+  }
+}
+template <typename TI>
+__device__ __forceinline__ void tc_stage_gates(float* sU, const BwdArgs<TI>& a, int f0, int b, int h) {
+  const int cpr = a.dk / 4, pw = a.dk + 4;
+  for (int idx = threadIdx.x; idx < kTcRows * cpr; idx += NT) {
+    const int r = idx / cpr, cc = idx - r * cpr;
+    const int f = f0 + r;
+    const bool valid = f >= 0 && f < a.g.T;
+    const float* p = valid ? a.la + row_off(a, b, h, f, a.dk) + cc * 4 : a.la;
+    cp_async16(smem_u32(sU + r * pw + cc * 4), p, valid);
+  }
+}
+
+
 // Exact sweep of a flagged chunk from fp32 tiles (alpha, k, v) staged in shared
 // memory; q and dout rows are read from global memory one position at a time.
 __device__ void tc_chunk_serial(const BwdArgs<__nv_bfloat16>& a, float* smem, int c, int b, int h, int f0) {
@@ -660,7 +689,7 @@ __host__ __device__ inline TcLayout tc_layout(int dk, int dv) {
   L.oG = L.oP + 8u * kTcRows * 32u;
   L.oD = L.oG + (Np / 16) * Kp * 32u;
   L.oU = L.oD + (Np / 16) * Kp * 32u;
-  L.oMisc = (L.oU + (uint32_t)kTcRows * (uint32_t)(dk + 1) * 4u + 15u) / 16u * 16u;
+  L.oMisc = (L.oU + (uint32_t)kTcRows * (uint32_t)(dk + 4) * 4u + 15u) / 16u * 16u;
   L.bytes = L.oMisc + 1024u + 64u + 1024u;  // gate totals, carry, barrier, TMEM address; alignment slack
   return L;
 }
@@ -675,12 +704,12 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
   const TcLayout L = tc_layout(a.dk, a.dv);
   const uint32_t Kp = (uint32_t)(a.dk + 15) / 16 * 16, Np = (uint32_t)(a.dv + 15) / 16 * 16;
   const uint32_t sb = smem_u32(smem_tc);
-  float* sU = reinterpret_cast<float*>(smem_tc + L.oU);   // [MC][dk+1]: log-gates, u, then db
+  float* sU = reinterpret_cast<float*>(smem_tc + L.oU);   // [MC][dk+4]: log-gates, u, then db
   float* sTot = reinterpret_cast<float*>(smem_tc + L.oMisc);
   float* sCarry = sTot + 128;
   uint64_t* sBar = reinterpret_cast<uint64_t*>(sCarry + 128);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sBar + 1);
-  const int pu = a.dk + 1;
+  const int pu = a.dk + 4;
   const int f0 = chunk_first_base_pos(a.g, c, MC);
   const int64_t cid = (int64_t)bh * a.NC + c;
   const bool rev = a.g.reverse;
@@ -699,29 +728,16 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
     fence_mbar_init();
   }
   // ---- staging: log-gates (fp32), q, k, v, dout (bf16, swizzled, zero past the
-  // channels and rows), G = Diag(e^g) S_in and D (bf16, [Kp][Np] tiles)
-  stage<MC>(sU, a.la, a.dk, a.g, f0, b, h, a.H);
-  {
-    const int cq = (int)Kp / 8, cv = (int)Np / 8;
-    for (int idx = threadIdx.x; idx < MC * (2 * cq + 2 * cv); idx += NT) {
-      const int r = idx % MC, w = idx / MC;  // consecutive threads: consecutive rows
-      int which, cc;
-      if (w < cq) which = 0, cc = w;
-      else if (w < 2 * cq) which = 1, cc = w - cq;
-      else if (w < 2 * cq + cv) which = 2, cc = w - 2 * cq;
-      else which = 3, cc = w - 2 * cq - cv;
-      const int d = which < 2 ? a.dk : a.dv;
-      const __nv_bfloat16* src = which == 0 ? a.q : which == 1 ? a.k : which == 2 ? a.v : a.dout;
-      const uint32_t tile = which == 0 ? L.oQ : which == 1 ? L.oK : which == 2 ? L.oV : L.oO;
-      const int f = f0 + r;
-      uint4 val = make_uint4(0u, 0u, 0u, 0u);
-      if (f >= 0 && f < a.g.T && cc * 8 < d)
-        val = *reinterpret_cast<const uint4*>(src + row_off(a, b, h, f, d) + cc * 8);
-      *reinterpret_cast<uint4*>(smem_tc + tile + sw32_at(MC, (uint32_t)r, (uint32_t)(cc * 8))) = val;
-    }
-  }
+  // channels and rows) in flight together; then G = Diag(e^g) S_in and D
+  tc_stage_gates(sU, a, f0, b, h);
+  tc_stage_bf16(smem_tc, L.oQ, a.q, a.dk, (int)Kp, a, f0, b, h);
+  tc_stage_bf16(smem_tc, L.oK, a.k, a.dk, (int)Kp, a, f0, b, h);
+  tc_stage_bf16(smem_tc, L.oV, a.v, a.dv, (int)Np, a, f0, b, h);
+  tc_stage_bf16(smem_tc, L.oO, a.dout, a.dv, (int)Np, a, f0, b, h);
+  cp_async_commit();
+  cp_async_wait_all();
   __syncthreads();
-  suffix_sums<MC>(sU, sTot, a.dk, rev);
+  suffix_sums<MC>(sU, sTot, a.dk, rev, pu);
   __syncthreads();
   {
     const size_t st = (size_t)a.dk * a.dv;
@@ -922,7 +938,7 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
 // MN-major (M = key channels; the tiles hold 128 channels, zero past dk).
 constexpr uint32_t kTcLocalBytes(int dk, int dv) {
   return 2u * 8u * kTcRows * 32u + 2u * (uint32_t)((dv + 15) / 16) * kTcRows * 32u +
-         (uint32_t)kTcRows * (uint32_t)(dk + 1) * 4u + 512u + 64u + 1024u;
+         (uint32_t)kTcRows * (uint32_t)(dk + 4) * 4u + 512u + 64u + 1024u;
 }
 
 __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_local(const BwdArgs<__nv_bfloat16> a) {
@@ -935,10 +951,10 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_local(const BwdArgs<__nv_bfl
   const uint32_t oK = 0, oQ = 8u * MC * 32u, oV = 16u * MC * 32u, oO = oV + Np / 16 * MC * 32u;
   const uint32_t oU = oO + Np / 16 * MC * 32u;
   float* sU = reinterpret_cast<float*>(sm + oU);
-  float* sTot = sU + MC * (a.dk + 1);
+  float* sTot = sU + MC * (a.dk + 4);
   uint64_t* sBar = reinterpret_cast<uint64_t*>(sTot + 128);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sBar + 1);
-  const int pu = a.dk + 1;
+  const int pu = a.dk + 4;
   const uint32_t sb = smem_u32(sm);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool rev = a.g.reverse;
@@ -951,26 +967,13 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_local(const BwdArgs<__nv_bfl
     mbar_init(smem_u32(sBar), 1);
     fence_mbar_init();
   }
-  stage<MC>(sU, a.la, a.dk, a.g, f0, b, h, a.H);
-  {
-    const int cv = (int)Np / 8;
-    for (int idx = threadIdx.x; idx < MC * (16 + 16 + 2 * cv); idx += NT) {
-      const int r = idx % MC, w = idx / MC;
-      int which, cc;
-      if (w < 16) which = 0, cc = w;
-      else if (w < 32) which = 1, cc = w - 16;
-      else if (w < 32 + cv) which = 2, cc = w - 32;
-      else which = 3, cc = w - 32 - cv;
-      const int d = which < 2 ? a.dk : a.dv;
-      const __nv_bfloat16* src = which == 0 ? a.k : which == 1 ? a.q : which == 2 ? a.v : a.dout;
-      const uint32_t tile = which == 0 ? oK : which == 1 ? oQ : which == 2 ? oV : oO;
-      const int f = f0 + r;
-      uint4 val = make_uint4(0u, 0u, 0u, 0u);
-      if (f >= 0 && f < a.g.T && cc * 8 < d)
-        val = *reinterpret_cast<const uint4*>(src + row_off(a, b, h, f, d) + cc * 8);
-      *reinterpret_cast<uint4*>(sm + tile + sw32_at(MC, (uint32_t)r, (uint32_t)(cc * 8))) = val;
-    }
-  }
+  tc_stage_gates(sU, a, f0, b, h);
+  tc_stage_bf16(sm, oK, a.k, a.dk, 128, a, f0, b, h);
+  tc_stage_bf16(sm, oQ, a.q, a.dk, 128, a, f0, b, h);
+  tc_stage_bf16(sm, oV, a.v, a.dv, (int)Np, a, f0, b, h);
+  tc_stage_bf16(sm, oO, a.dout, a.dv, (int)Np, a, f0, b, h);
+  cp_async_commit();
+  cp_async_wait_all();
   __syncthreads();
   // Qbar = q e^{b}: b the inclusive prefix of the log-gates in scan order, walked
   // directly (a -inf gate gives 0, not inf - inf).
@@ -984,7 +987,7 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_local(const BwdArgs<__nv_bfl
     }
   }
   __syncthreads();
-  const int code = suffix_sums<MC>(sU, sTot, a.dk, rev);
+  const int code = suffix_sums<MC>(sU, sTot, a.dk, rev, pu);
   if (code & 2) report_status(GLA_ERR_RANGE);
   const int wide = __syncthreads_or(code != 0);
   // K^ = k e^{u}: the exponent is a sum of log-gates, so decays only shrink it.
