@@ -134,12 +134,27 @@ __device__ __forceinline__ void zero48(float (&acc)[R][8]) {
 // memory): one warp per row i, lanes over j (coalesced), a fixed shuffle-tree sum.
 __device__ __forceinline__ void chunk_carry(const float* D, const float* Sout, int dk, int dv, float* carry) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  for (int i = warp; i < dk; i += nw) {
-    float acc = 0.f;
-    for (int j = lane; j < dv; j += 32) acc = fmaf(D[(size_t)i * dv + j], Sout[(size_t)i * dv + j], acc);
+  // Rows i = warp, warp + nw, ... four at a time, all their loads issued first.
+  for (int i0 = warp; i0 < dk; i0 += 4 * nw) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = lane; j < dv; j += 32) {
+      float x[4], y[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) carry[i] = acc;
+      for (int m = 0; m < 4; ++m) {
+        const int i = i0 + m * nw;
+        x[m] = i < dk ? D[(size_t)i * dv + j] : 0.f;
+        y[m] = i < dk ? Sout[(size_t)i * dv + j] : 0.f;
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) acc[m] = fmaf(x[m], y[m], acc[m]);
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], o);
+      const int i = i0 + m * nw;
+      if (lane == 0 && i < dk) carry[i] = acc[m];
+    }
   }
 }
 
@@ -763,19 +778,31 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
       *pq = wq;
       *pk = wk;
     }
-    // G[i][j] = e^{g_i} S_in[i][j] and D[i][j], bf16, rows i < Kp, channels j < Np
-    for (int e = threadIdx.x; e < (int)(Kp * Np); e += NT) {
-      const int i = e / (int)Np, j = e - i * (int)Np;
-      float gv = 0.f, dv_ = 0.f;
-      if (i < a.dk && j < a.dv) {
+    // G[i][j] = e^{g_i} S_in[i][j] and D[i][j], bf16, rows i < Kp, channels j < Np;
+    // eight elements per thread are loaded before any is converted.
+    const int nG = (int)(Kp * Np);
+    for (int e0 = threadIdx.x; e0 < nG; e0 += 8 * NT) {
+      float gs[8], ds[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int e = e0 + m * NT;
+        const int i = e / (int)Np, j = e - i * (int)Np;
+        const bool in = e < nG && i < a.dk && j < a.dv;
         const size_t o = (size_t)i * a.dv + j;
-        gv = sin ? expf(sTot[i]) * sin[o] : 0.f;
-        dv_ = dd[o];
+        gs[m] = in && sin ? sin[o] : 0.f;
+        ds[m] = in ? dd[o] : 0.f;
       }
-      *reinterpret_cast<__nv_bfloat16*>(smem_tc + L.oG + sw32_at(Kp, (uint32_t)i, (uint32_t)j)) =
-          __float2bfloat16_rn(gv);
-      *reinterpret_cast<__nv_bfloat16*>(smem_tc + L.oD + sw32_at(Kp, (uint32_t)i, (uint32_t)j)) =
-          __float2bfloat16_rn(dv_);
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int e = e0 + m * NT;
+        if (e >= nG) break;
+        const int i = e / (int)Np, j = e - i * (int)Np;
+        const float gv = i < a.dk ? expf(sTot[i]) * gs[m] : 0.f;
+        *reinterpret_cast<__nv_bfloat16*>(smem_tc + L.oG + sw32_at(Kp, (uint32_t)i, (uint32_t)j)) =
+            __float2bfloat16_rn(gv);
+        *reinterpret_cast<__nv_bfloat16*>(smem_tc + L.oD + sw32_at(Kp, (uint32_t)i, (uint32_t)j)) =
+            __float2bfloat16_rn(ds[m]);
+      }
     }
   }
   fence_proxy_async_smem();
