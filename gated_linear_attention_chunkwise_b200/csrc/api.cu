@@ -344,8 +344,8 @@ cudaError_t run_bwd(void* ws, void* ctx) {
   return arrange(dl2, c->dla, s, rl, 1, c->st);
 }
 size_t bwd_ws_bytes(const GlaShape& s, int bf16) {
-  return s.dir < 4 ? dig::gla_bwd_workspace_bytes(s)
-                   : arranged_bytes(s, bf16 ? 2 : 4, 4, 3, 2) + dig::gla_bwd_workspace_bytes(line_shape(s));
+  return s.dir < 4 ? dig::gla_bwd_workspace_bytes(s, bf16)
+                   : arranged_bytes(s, bf16 ? 2 : 4, 4, 3, 2) + dig::gla_bwd_workspace_bytes(line_shape(s), bf16);
 }
 int gla_bwd_common(const void* q, const void* k, const void* v, const float* la, const void* dout, int B, int H,
                    int Hgrid, int Wgrid, int dk, int dv, int dir, void* dq, void* dk_out, void* dv_out, float* dla,

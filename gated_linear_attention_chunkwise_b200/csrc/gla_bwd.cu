@@ -1176,8 +1176,8 @@ cudaError_t run_bwd(const void* q, const void* k, const void* v, const float* la
 
 }  // namespace
 
-size_t gla_bwd_workspace_bytes(const GlaShape& s) {
-  const int MC = chunk_rows(s);
+size_t gla_bwd_workspace_bytes(const GlaShape& s, int bf16) {
+  const int MC = use_tc(s, bf16) ? kTcRows : chunk_rows(s);
   const size_t NC = (size_t)(s.T() + MC - 1) / MC;
   const size_t BH = (size_t)s.B * s.H;
   return rup(BH * NC * s.dk * s.dv * 4, 256) * 2 + rup(BH * NC * s.dk * 4, 256) + rup(BH * NC * 4, 256);

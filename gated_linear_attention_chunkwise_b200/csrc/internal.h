@@ -34,8 +34,9 @@ size_t gla_f32_workspace_bytes(const GlaShape& s);
 cudaError_t gla_f32_forward(const float* q, const float* k, const float* v, const float* la, float* out,
                             const GlaShape& s, void* workspace, cudaStream_t st);
 
-// ---- GLA backward on CUDA cores (chunks of 32 scan positions) ----
-size_t gla_bwd_workspace_bytes(const GlaShape& s);
+// ---- GLA backward: tensor cores for bf16 with dk, dv <= 80 (chunks of 128 scan
+// positions), else CUDA cores (chunks of 32) ----
+size_t gla_bwd_workspace_bytes(const GlaShape& s, int bf16);
 cudaError_t gla_bwd_launch(const void* q, const void* k, const void* v, const float* la, const void* dout, void* dq,
                            void* dk, void* dv, float* dla, const GlaShape& s, int bf16, void* workspace,
                            cudaStream_t st);

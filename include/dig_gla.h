@@ -166,22 +166,26 @@ int gla_fwd_f32_noalloc(const float* q, const float* k, const float* v, const fl
  *   dlog_alpha    [B][T][H][dk] fp32        (d L / d log_alpha, not d alpha)
  * from q, k [B][T][H][dk] bf16, v and dout [B][T][H][dv] bf16 and log_alpha
  * [B][T][H][dk] fp32, all at canonical token positions.
- * Arithmetic: every product and sum in fp32 on CUDA cores, from the bf16 inputs
- * widened exactly; dq, dk, dv rounded to nearest even on the store.  Chunks of 32
- * scan positions; a chunk whose gates decay by more than e^80 inside it (a full
- * reset, -inf) is differentiated token by token (exact, slower).  Growth gates whose product exceeds e^80 inside a chunk record
- * GLA_ERR_RANGE.  Shapes, dims, directions and errors as gla_fwd; no output may
- * overlap an input or another output.  Workspace: 2 * B*H*ceil(T/32) * dk*dv fp32
- * values plus per-chunk gates (520 MB for B=2, H=16, T=12544, d=72), stream-ordered
- * from the library's pool as gla_fwd's.
+ * Arithmetic: for dk, dv <= 80, chunks of M = 128 scan positions whose products run
+ * on tensor cores from bf16 operands (the gated q and k, the masked dout v^T and
+ * q k^T scores, the carried state and its gradient, each rounded to bf16) with fp32
+ * accumulation; gate sums, scans over chunks and d log_alpha in fp32.  Wider heads:
+ * chunks of M = 32 with every product in fp32 on CUDA cores.  dq, dk, dv rounded to
+ * nearest even on the store.  A chunk whose gates decay by more than e^80 inside it
+ * (a full reset, -inf) is differentiated token by token in fp32 (exact, slower).
+ * Growth gates whose product exceeds e^80 inside a chunk record GLA_ERR_RANGE.
+ * Shapes, dims, directions and errors as gla_fwd; no output may overlap an input or
+ * another output.  Workspace: 2 * B*H*ceil(T/M) * dk*dv fp32 values plus per-chunk
+ * gates (130 MB for B=2, H=16, T=12544, d=72), stream-ordered from the library's
+ * pool as gla_fwd's; zigzag orders add copies of the nine tensors in scan order.
  */
 int gla_bwd(const void* q, const void* k, const void* v, const float* log_alpha, const void* dout, int B, int H,
             int Hgrid, int Wgrid, int dk, int dv, int dir, void* dq, void* dk_out, void* dv_out, float* dlog_alpha,
             cudaStream_t stream);
 
 /*
- * gla_bwd_f32 -- gla_bwd with fp32 q, k, v, dout, dq, dk, dv (same arithmetic, no
- * rounding on the store).
+ * gla_bwd_f32 -- gla_bwd with fp32 q, k, v, dout, dq, dk, dv: every product and sum
+ * in fp32 on CUDA cores (chunks of M = 32), no rounding on the store.
  */
 int gla_bwd_f32(const float* q, const float* k, const float* v, const float* log_alpha, const float* dout, int B,
                 int H, int Hgrid, int Wgrid, int dk, int dv, int dir, float* dq, float* dk_out, float* dv_out,
