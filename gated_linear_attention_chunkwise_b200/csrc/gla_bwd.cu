@@ -584,33 +584,79 @@ __device__ __forceinline__ uint64_t dmn(uint32_t tile, uint32_t rows, int kk) {
 
 __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) { tmem_ld16(taddr, v); }
 
-// Asynchronous staging of rows f0 .. f0+127 (zero outside the sequence and past d):
+// Token index of each of the chunk's rows (base positions f0 .. f0+127), -1 for rows
+// outside the sequence; the staging and the d log alpha stores index through it.
+__device__ __forceinline__ void tc_row_tokens(int* sRow, const ScanGeom& g, int f0) {
+  for (int r = threadIdx.x; r < kTcRows; r += NT) {
+    const int f = f0 + r;
+    sRow[r] = (f >= 0 && f < g.T) ? base_pos_to_token(g, f) : -1;
+  }
+}
+template <typename TI>
+__device__ __forceinline__ int64_t tok_off(const BwdArgs<TI>& a, int b, int h, int tok, int d) {
+  return (((int64_t)b * a.g.T + tok) * a.H + h) * d;
+}
+
+// Asynchronous staging of the chunk's rows (zero outside the sequence and past d):
 // bf16 operand tiles in the 32-byte-swizzled layout (`nch` channels, a multiple of 8)
 // and the fp32 log-gate tile with a pitch of dk + 4 floats.  Every 16-byte copy of the
 // CTA is in flight at once; the caller waits with cp_async_wait_all and a barrier.
 template <typename TI>
 __device__ __forceinline__ void tc_stage_bf16(uint8_t* sm, uint32_t tile, const __nv_bfloat16* src, int d, int nch,
-                                              const BwdArgs<TI>& a, int f0, int b, int h) {
+                                              const BwdArgs<TI>& a, const int* sRow, int b, int h) {
   const int cc_n = nch / 8;
   for (int idx = threadIdx.x; idx < kTcRows * cc_n; idx += NT) {
     const int r = idx % kTcRows, cc = idx / kTcRows;
-    const int f = f0 + r;
-    const bool valid = f >= 0 && f < a.g.T && cc * 8 < d;
-    const __nv_bfloat16* p = valid ? src + row_off(a, b, h, f, d) + cc * 8 : src;
+    const int tok = sRow[r];
+    const bool valid = tok >= 0 && cc * 8 < d;
+    const __nv_bfloat16* p = valid ? src + tok_off(a, b, h, tok, d) + cc * 8 : src;
     cp_async16(smem_u32(sm + tile + sw32_at(kTcRows, (uint32_t)r, (uint32_t)(cc * 8))), p, valid);
   }
 }
 template <typename TI>
-__device__ __forceinline__ void tc_stage_gates(float* sU, const BwdArgs<TI>& a, int f0, int b, int h) {
+__device__ __forceinline__ void tc_stage_gates(float* sU, const BwdArgs<TI>& a, const int* sRow, int b, int h) {
   const int cpr = a.dk / 4, pw = a.dk + 4;
   for (int idx = threadIdx.x; idx < kTcRows * cpr; idx += NT) {
     const int r = idx / cpr, cc = idx - r * cpr;
-    const int f = f0 + r;
-    const bool valid = f >= 0 && f < a.g.T;
-    const float* p = valid ? a.la + row_off(a, b, h, f, a.dk) + cc * 4 : a.la;
-    cp_async16(smem_u32(sU + r * pw + cc * 4), p, valid);
+    const int tok = sRow[r];
+    const float* p = tok >= 0 ? a.la + tok_off(a, b, h, tok, a.dk) + cc * 4 : a.la;
+    cp_async16(smem_u32(sU + r * pw + cc * 4), p, tok >= 0);
   }
 }
+// n fp32 values (a multiple of 4) from src, or zeros when src is null.
+__device__ __forceinline__ void tc_stage_f32(float* dst, const float* src, int n, const float* any) {
+  for (int e = 4 * (int)threadIdx.x; e < n; e += 4 * NT) cp_async16(smem_u32(dst + e), src ? src + e : any, src != nullptr);
+}
+
+// Segmented walks along a chunk's scan order: thread t takes channel i = t % dk and
+// segment s = t / dk, the scan steps [st0, st1) of nseg nearly equal segments (three
+// for dk > 64, else four; dk <= 80 on this path).  A walk first needs the totals of
+// the other segments (phase 1, one barrier), then runs over its own steps only.
+constexpr int kSegMax = 43;  // ceil(128 / 3)
+struct SegWalk {
+  int i, s, nseg, st0, st1;
+  bool active;
+};
+__device__ __forceinline__ SegWalk seg_walk(int dk) {
+  SegWalk w;
+  w.nseg = dk > 64 ? 3 : 4;
+  const int len = (kTcRows + w.nseg - 1) / w.nseg;
+  w.i = (int)threadIdx.x % dk;
+  w.s = (int)threadIdx.x / dk;
+  w.active = w.s < w.nseg;
+  w.st0 = w.s * len;
+  w.st1 = min(w.st0 + len, kTcRows);
+  return w;
+}
+// Sums of the other segments' totals (sPart[s][i], 128 floats per segment): those
+// before s in scan order and those after it, each added in a fixed order.
+__device__ __forceinline__ void seg_offsets(const SegWalk& w, const float* sPart, float& before, float& after) {
+  before = 0.f;
+  after = 0.f;
+  for (int s2 = 0; s2 < w.s; ++s2) before += sPart[s2 * kTcRows + w.i];
+  for (int s2 = w.nseg - 1; s2 > w.s; --s2) after += sPart[s2 * kTcRows + w.i];
+}
+__device__ __forceinline__ int seg_row(int st, bool rev) { return rev ? (kTcRows - 1 - st) : st; }
 
 
 // Exact sweep of a flagged chunk from fp32 tiles (alpha, k, v) staged in shared
@@ -691,6 +737,7 @@ __device__ void tc_chunk_serial(const BwdArgs<__nv_bfloat16>& a, float* smem, in
 
 struct TcLayout {
   uint32_t oQ, oK, oV, oO, oA, oP, oG, oD, oU, oMisc, bytes;
+  int nst;  // fp32 chunk states staged in the A/P area: S_in, D, and S_out when it fits
 };
 __host__ __device__ inline TcLayout tc_layout(int dk, int dv) {
   const uint32_t Kp = (uint32_t)(dk + 15) / 16 * 16, Np = (uint32_t)(dv + 15) / 16 * 16;
@@ -705,7 +752,10 @@ __host__ __device__ inline TcLayout tc_layout(int dk, int dv) {
   L.oD = L.oG + (Np / 16) * Kp * 32u;
   L.oU = L.oD + (Np / 16) * Kp * 32u;
   L.oMisc = (L.oU + (uint32_t)kTcRows * (uint32_t)(dk + 4) * 4u + 15u) / 16u * 16u;
-  L.bytes = L.oMisc + 1024u + 64u + 1024u;  // gate totals, carry, barrier, TMEM address; alignment slack
+  // gate totals, e^{totals}, carry (128 floats each), segment totals (4 x 128), row
+  // tokens (128), barrier and TMEM address; alignment slack
+  L.bytes = L.oMisc + 3u * 512u + 2048u + 512u + 64u + 1024u;
+  L.nst = 3u * (uint32_t)dk * (uint32_t)dv * 4u <= 2u * 8u * kTcRows * 32u ? 3 : 2;
   return L;
 }
 
@@ -721,13 +771,22 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
   const uint32_t sb = smem_u32(smem_tc);
   float* sU = reinterpret_cast<float*>(smem_tc + L.oU);   // [MC][dk+4]: log-gates, u, then db
   float* sTot = reinterpret_cast<float*>(smem_tc + L.oMisc);
-  float* sCarry = sTot + 128;
-  uint64_t* sBar = reinterpret_cast<uint64_t*>(sCarry + 128);
+  float* sGam = sTot + 128;
+  float* sCarry = sGam + 128;
+  float* sPart = sCarry + 128;                            // [4][128] segment totals
+  int* sRow = reinterpret_cast<int*>(sPart + 4 * 128);    // [128] row tokens
+  uint64_t* sBar = reinterpret_cast<uint64_t*>(sRow + 128);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sBar + 1);
+  // fp32 chunk states, staged over the A and P tiles (written only after the first MMAs)
+  float* sSin = reinterpret_cast<float*>(smem_tc + L.oA);
+  const int dkv = a.dk * a.dv;
+  float* sDs = sSin + dkv;
+  float* sSo = sDs + dkv;
   const int pu = a.dk + 4;
   const int f0 = chunk_first_base_pos(a.g, c, MC);
   const int64_t cid = (int64_t)bh * a.NC + c;
   const bool rev = a.g.reverse;
+  const size_t st = (size_t)dkv;
 
   if (a.flags[cid]) {
     tc_chunk_serial(a, reinterpret_cast<float*>(smem_tc), c, b, h, f0);
@@ -742,22 +801,46 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
     mbar_init(smem_u32(sBar), 1);
     fence_mbar_init();
   }
-  // ---- staging: log-gates (fp32), q, k, v, dout (bf16, swizzled, zero past the
-  // channels and rows) in flight together; then G = Diag(e^g) S_in and D
-  tc_stage_gates(sU, a, f0, b, h);
-  tc_stage_bf16(smem_tc, L.oQ, a.q, a.dk, (int)Kp, a, f0, b, h);
-  tc_stage_bf16(smem_tc, L.oK, a.k, a.dk, (int)Kp, a, f0, b, h);
-  tc_stage_bf16(smem_tc, L.oV, a.v, a.dv, (int)Np, a, f0, b, h);
-  tc_stage_bf16(smem_tc, L.oO, a.dout, a.dv, (int)Np, a, f0, b, h);
+  tc_row_tokens(sRow, a.g, f0);
+  __syncthreads();
+  // ---- staging, all in flight together: log-gates (fp32), q, k, v, dout (bf16,
+  // swizzled, zero past the channels and rows), S_in, D and (when it fits) S_out
+  tc_stage_gates(sU, a, sRow, b, h);
+  tc_stage_bf16(smem_tc, L.oQ, a.q, a.dk, (int)Kp, a, sRow, b, h);
+  tc_stage_bf16(smem_tc, L.oK, a.k, a.dk, (int)Kp, a, sRow, b, h);
+  tc_stage_bf16(smem_tc, L.oV, a.v, a.dv, (int)Np, a, sRow, b, h);
+  tc_stage_bf16(smem_tc, L.oO, a.dout, a.dv, (int)Np, a, sRow, b, h);
+  tc_stage_f32(sSin, c > 0 ? a.sx + (cid - 1) * st : nullptr, dkv, a.la);
+  tc_stage_f32(sDs, a.dd + cid * st, dkv, a.la);
+  if (L.nst == 3) tc_stage_f32(sSo, a.sx + cid * st, dkv, a.la);
   cp_async_commit();
   cp_async_wait_all();
   __syncthreads();
-  suffix_sums<MC>(sU, sTot, a.dk, rev, pu);
+  // ---- u: exclusive suffix sums of the log-gates in scan order, in place (segmented)
+  const SegWalk w = seg_walk(a.dk);
+  if (w.active) {
+    float t = 0.f;
+    for (int st2 = w.st0; st2 < w.st1; ++st2) t += sU[seg_row(st2, rev) * pu + w.i];
+    sPart[w.s * MC + w.i] = t;
+  }
+  __syncthreads();
+  if (w.active) {
+    float before, acc;
+    seg_offsets(w, sPart, before, acc);
+#pragma unroll 4
+    for (int st2 = w.st1 - 1; st2 >= w.st0; --st2) {
+      float* p = sU + seg_row(st2, rev) * pu + w.i;
+      const float l = *p;
+      *p = acc;
+      acc += l;
+    }
+    if (w.s == 0) {
+      sTot[w.i] = acc;
+      sGam[w.i] = expf(acc);
+    }
+  }
   __syncthreads();
   {
-    const size_t st = (size_t)a.dk * a.dv;
-    const float* sin = c > 0 ? a.sx + (cid - 1) * st : nullptr;
-    const float* dd = a.dd + cid * st;
     // Q~ = q e^{-u}, K^ = k e^{u} in place (8 channels per thread), padding stays 0
     const int cq = (int)Kp / 8;
     for (int idx = threadIdx.x; idx < MC * cq; idx += NT) {
@@ -772,36 +855,32 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
       for (int e = 0; e < 4; ++e) {
         const float u0 = sU[r * pu + cc * 8 + 2 * e], u1 = sU[r * pu + cc * 8 + 2 * e + 1];
         const float2 xq = unpack_bf16x2(uq[e]), xk = unpack_bf16x2(uk[e]);
-        uq[e] = pack_bf16x2(xq.x * expf(-u0), xq.y * expf(-u1));
-        uk[e] = pack_bf16x2(xk.x * expf(u0), xk.y * expf(u1));
+        uq[e] = pack_bf16x2(xq.x * __expf(-u0), xq.y * __expf(-u1));
+        uk[e] = pack_bf16x2(xk.x * __expf(u0), xk.y * __expf(u1));
       }
       *pq = wq;
       *pk = wk;
     }
-    // G[i][j] = e^{g_i} S_in[i][j] and D[i][j], bf16, rows i < Kp, channels j < Np;
-    // eight elements per thread are loaded before any is converted.
+    // G[i][j] = e^{g_i} S_in[i][j] and D[i][j] as bf16 tiles, rows i < Kp, channels j < Np
     const int nG = (int)(Kp * Np);
-    for (int e0 = threadIdx.x; e0 < nG; e0 += 8 * NT) {
-      float gs[8], ds[8];
+    for (int e = threadIdx.x; e < nG; e += NT) {
+      const int i = e / (int)Np, j = e - i * (int)Np;
+      const bool in = i < a.dk && j < a.dv;
+      const float gv = in ? sGam[i] * sSin[i * a.dv + j] : 0.f;
+      const float dv_ = in ? sDs[i * a.dv + j] : 0.f;
+      *reinterpret_cast<__nv_bfloat16*>(smem_tc + L.oG + sw32_at(Kp, (uint32_t)i, (uint32_t)j)) =
+          __float2bfloat16_rn(gv);
+      *reinterpret_cast<__nv_bfloat16*>(smem_tc + L.oD + sw32_at(Kp, (uint32_t)i, (uint32_t)j)) =
+          __float2bfloat16_rn(dv_);
+    }
+    // carry[i] = sum_j D[i][j] S_out[i][j]: one warp per row, a fixed shuffle tree
+    if (L.nst == 3) {
+      for (int i = warp; i < a.dk; i += NT / 32) {
+        float acc = 0.f;
+        for (int j = lane; j < a.dv; j += 32) acc = fmaf(sDs[i * a.dv + j], sSo[i * a.dv + j], acc);
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int e = e0 + m * NT;
-        const int i = e / (int)Np, j = e - i * (int)Np;
-        const bool in = e < nG && i < a.dk && j < a.dv;
-        const size_t o = (size_t)i * a.dv + j;
-        gs[m] = in && sin ? sin[o] : 0.f;
-        ds[m] = in ? dd[o] : 0.f;
-      }
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int e = e0 + m * NT;
-        if (e >= nG) break;
-        const int i = e / (int)Np, j = e - i * (int)Np;
-        const float gv = i < a.dk ? expf(sTot[i]) * gs[m] : 0.f;
-        *reinterpret_cast<__nv_bfloat16*>(smem_tc + L.oG + sw32_at(Kp, (uint32_t)i, (uint32_t)j)) =
-            __float2bfloat16_rn(gv);
-        *reinterpret_cast<__nv_bfloat16*>(smem_tc + L.oD + sw32_at(Kp, (uint32_t)i, (uint32_t)j)) =
-            __float2bfloat16_rn(ds[m]);
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) sCarry[i] = acc;
       }
     }
   }
@@ -837,18 +916,18 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
         const int s0 = 64 * hf + 16 * g;
         float x[16];
         tc_ld16(tbase + lane_base + col + (uint32_t)s0, x);
-        uint32_t w[8];
+        uint32_t wv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int sa = s0 + 2 * e, sbb = sa + 1;
           const float x0 = (rev ? sa >= r : sa <= r) ? x[2 * e] : 0.f;
           const float x1 = (rev ? sbb >= r : sbb <= r) ? x[2 * e + 1] : 0.f;
-          w[e] = pack_bf16x2(x0, x1);
+          wv[e] = pack_bf16x2(x0, x1);
         }
         *reinterpret_cast<uint4*>(smem_tc + tile + sw32_at(MC, (uint32_t)r, (uint32_t)s0)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+            make_uint4(wv[0], wv[1], wv[2], wv[3]);
         *reinterpret_cast<uint4*>(smem_tc + tile + sw32_at(MC, (uint32_t)r, (uint32_t)(s0 + 8))) =
-            make_uint4(w[4], w[5], w[6], w[7]);
+            make_uint4(wv[4], wv[5], wv[6], wv[7]);
       }
     }
   }
@@ -883,11 +962,11 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
   }
   tc_fence_after();
   // ---- epilogue: row r, 16-channel groups g with g % 2 == hf
-  const int f = f0 + r;
-  const bool real = f >= 0 && f < a.g.T;
+  const int tok = sRow[r];
+  const bool real = tok >= 0;
   if (ok) {
     // q dq - k dk = Q~ dQ~ - K^ dK^, with Q~ and K^ the bf16 tiles of the MMAs.
-    const int64_t ok_ = real ? row_off(a, b, h, f, a.dk) : 0;
+    const int64_t ok_ = real ? tok_off(a, b, h, tok, a.dk) : 0;
     for (int g = hf; g < (int)Kp / 16; g += 2) {
       float xq[16], xk[16];
       tc_ld16(tbase + lane_base + cDQ + (uint32_t)(16 * g), xq);
@@ -907,8 +986,8 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
           const float a0 = xq[8 * half + 2 * e], a1 = xq[8 * half + 2 * e + 1];
           const float b0 = xk[8 * half + 2 * e], b1 = xk[8 * half + 2 * e + 1];
           const float u0 = sU[r * pu + i], u1 = sU[r * pu + i + 1];
-          pq[e] = pack_bf16x2(expf(-u0) * a0, expf(-u1) * a1);
-          pk[e] = pack_bf16x2(expf(u0) * b0, expf(u1) * b1);
+          pq[e] = pack_bf16x2(__expf(-u0) * a0, __expf(-u1) * a1);
+          pk[e] = pack_bf16x2(__expf(u0) * b0, __expf(u1) * b1);
           sU[r * pu + i] = real ? tq.x * a0 - tk.x * b0 : 0.f;
           sU[r * pu + i + 1] = real ? tq.y * a1 - tk.y * b1 : 0.f;
         }
@@ -918,7 +997,7 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
         }
       }
     }
-    const int64_t ov_ = real ? row_off(a, b, h, f, a.dv) : 0;
+    const int64_t ov_ = real ? tok_off(a, b, h, tok, a.dv) : 0;
     for (int g = hf; g < (int)Np / 16; g += 2) {
       float xv[16];
       tc_ld16(tbase + lane_base + cDV + (uint32_t)(16 * g), xv);
@@ -944,48 +1023,74 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tbase, 512);
   if (!ok) return;
-  {
-    const size_t st = (size_t)a.dk * a.dv;
+  if (L.nst != 3) {
     chunk_carry(a.dd + cid * st, a.sx + cid * st, a.dk, a.dv, sCarry);
+    __syncthreads();
+  }
+  // ---- d log alpha_r = carry + sum over the chunk's rows at or after r of db
+  // (segmented: segment totals, then each segment's walk from its end)
+  if (w.active) {
+    float t = 0.f;
+    for (int st2 = w.st0; st2 < w.st1; ++st2) t += sU[seg_row(st2, rev) * pu + w.i];
+    sPart[w.s * MC + w.i] = t;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < a.dk; i += NT) {
-    float acc = sCarry[i];
-    for (int step = MC - 1; step >= 0; --step) {
-      const int rr = rev ? (MC - 1 - step) : step;
-      acc += sU[rr * pu + i];
-      const int ff = f0 + rr;
-      if (ff >= 0 && ff < a.g.T) a.dla[row_off(a, b, h, ff, a.dk) + i] = acc;
+  if (w.active) {
+    float before, after;
+    seg_offsets(w, sPart, before, after);
+    float acc = sCarry[w.i] + after;
+#pragma unroll 4
+    for (int st2 = w.st1 - 1; st2 >= w.st0; --st2) {
+      const int rr = seg_row(st2, rev);
+      acc += sU[rr * pu + w.i];
+      const int tk = sRow[rr];
+      if (tk >= 0) a.dla[tok_off(a, b, h, tk, a.dk) + w.i] = acc;
     }
   }
 }
 
 // Kernel 1 on tensor cores (bf16 inputs, dk and dv at most 80): per 128-row chunk,
 // K^T V and Qbar^T dO as M = 128 MMAs whose A operands are the k and q tiles read
-// MN-major (M = key channels; the tiles hold 128 channels, zero past dk).
-constexpr uint32_t kTcLocalBytes(int dk, int dv) {
-  return 2u * 8u * kTcRows * 32u + 2u * (uint32_t)((dv + 15) / 16) * kTcRows * 32u +
-         (uint32_t)kTcRows * (uint32_t)(dk + 4) * 4u + 512u + 64u + 1024u;
+// MN-major (M = key channels).  The tiles hold Kp channels; the MMA's A rows past Kp
+// read whatever follows a tile (the next tile) and only reach accumulator rows past
+// dk, which are never stored, so the tiles sit back to back and two CTAs fit per SM.
+// Each thread (channel, segment) holds its log-gates in registers and gates Qbar and
+// K^ during its two walks: no fp32 gate tile is staged.
+struct TlLayout {
+  uint32_t oK, oQ, oV, oO, oMisc, bytes;
+};
+__host__ __device__ inline TlLayout tl_layout(int dk, int dv) {
+  const uint32_t Kp = (uint32_t)(dk + 15) / 16 * 16, Np = (uint32_t)(dv + 15) / 16 * 16;
+  TlLayout L;
+  L.oK = 0;
+  L.oQ = Kp / 16 * kTcRows * 32u;
+  L.oV = L.oQ + Kp / 16 * kTcRows * 32u;
+  L.oO = L.oV + Np / 16 * kTcRows * 32u;
+  const uint32_t end = L.oO + Np / 16 * kTcRows * 32u;
+  const uint32_t reach = L.oQ + 8u * kTcRows * 32u;  // the q operand's last MMA read
+  L.oMisc = end > reach ? end : reach;
+  // segment totals (4 x 128 floats), row tokens (128), barrier, TMEM address; slack
+  L.bytes = L.oMisc + 2048u + 512u + 64u + 1024u;
+  return L;
 }
 
-__global__ void __launch_bounds__(NT, 1) gla_bwd_tc_local(const BwdArgs<__nv_bfloat16> a) {
+__global__ void __launch_bounds__(NT, 2) gla_bwd_tc_local(const BwdArgs<__nv_bfloat16> a) {
   extern __shared__ __align__(1024) uint8_t smem_raw_tl[];
   uint8_t* sm = smem_raw_tl + ((1024u - (smem_u32(smem_raw_tl) & 1023u)) & 1023u);
   constexpr int MC = kTcRows;
   const int c = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
-  const uint32_t Np = (uint32_t)(a.dv + 15) / 16 * 16;
-  const uint32_t oK = 0, oQ = 8u * MC * 32u, oV = 16u * MC * 32u, oO = oV + Np / 16 * MC * 32u;
-  const uint32_t oU = oO + Np / 16 * MC * 32u;
-  float* sU = reinterpret_cast<float*>(sm + oU);
-  float* sTot = sU + MC * (a.dk + 4);
-  uint64_t* sBar = reinterpret_cast<uint64_t*>(sTot + 128);
+  const uint32_t Kp = (uint32_t)(a.dk + 15) / 16 * 16, Np = (uint32_t)(a.dv + 15) / 16 * 16;
+  const TlLayout L = tl_layout(a.dk, a.dv);
+  float* sPart = reinterpret_cast<float*>(sm + L.oMisc);  // [4][128] segment totals
+  int* sRow = reinterpret_cast<int*>(sPart + 4 * 128);
+  uint64_t* sBar = reinterpret_cast<uint64_t*>(sRow + 128);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sBar + 1);
-  const int pu = a.dk + 4;
   const uint32_t sb = smem_u32(sm);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool rev = a.g.reverse;
   const int f0 = chunk_first_base_pos(a.g, c, MC);
+  const int64_t cid = (int64_t)bh * a.NC + c;
   if (warp == 0) {
     tmem_alloc(smem_u32(sTmem), 256);
     tmem_relinquish();
@@ -994,42 +1099,74 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_local(const BwdArgs<__nv_bfl
     mbar_init(smem_u32(sBar), 1);
     fence_mbar_init();
   }
-  tc_stage_gates(sU, a, f0, b, h);
-  tc_stage_bf16(sm, oK, a.k, a.dk, 128, a, f0, b, h);
-  tc_stage_bf16(sm, oQ, a.q, a.dk, 128, a, f0, b, h);
-  tc_stage_bf16(sm, oV, a.v, a.dv, (int)Np, a, f0, b, h);
-  tc_stage_bf16(sm, oO, a.dout, a.dv, (int)Np, a, f0, b, h);
+  tc_row_tokens(sRow, a.g, f0);
+  __syncthreads();
+  tc_stage_bf16(sm, L.oK, a.k, a.dk, (int)Kp, a, sRow, b, h);
+  tc_stage_bf16(sm, L.oQ, a.q, a.dk, (int)Kp, a, sRow, b, h);
+  tc_stage_bf16(sm, L.oV, a.v, a.dv, (int)Np, a, sRow, b, h);
+  tc_stage_bf16(sm, L.oO, a.dout, a.dv, (int)Np, a, sRow, b, h);
   cp_async_commit();
+  // This thread's log-gates (its channel, its segment's rows) into registers while
+  // the tiles arrive; then the segment's total.
+  const SegWalk w = seg_walk(a.dk);
+  float lg[kSegMax];
+#pragma unroll
+  for (int t = 0; t < kSegMax; ++t) {
+    const int st2 = w.st0 + t;
+    float x = 0.f;
+    if (w.active && st2 < w.st1) {
+      const int tk = sRow[seg_row(st2, rev)];
+      if (tk >= 0) x = a.la[tok_off(a, b, h, tk, a.dk) + w.i];
+    }
+    lg[t] = x;
+  }
+  if (w.active) {
+    float t = 0.f;
+#pragma unroll
+    for (int t2 = 0; t2 < kSegMax; ++t2) t += lg[t2];
+    sPart[w.s * MC + w.i] = t;
+  }
   cp_async_wait_all();
   __syncthreads();
-  // Qbar = q e^{b}: b the inclusive prefix of the log-gates in scan order, walked
-  // directly (a -inf gate gives 0, not inf - inf).
-  for (int i = threadIdx.x; i < a.dk; i += NT) {
-    float acc = 0.f;
-    for (int st = 0; st < MC; ++st) {
-      const int r = rev ? (MC - 1 - st) : st;
-      acc += sU[r * pu + i];
-      __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(sm + oQ + sw32_at(MC, (uint32_t)r, (uint32_t)i));
-      *p = __float2bfloat16_rn(__bfloat162float(*p) * expf(acc));
+  int code = 0;
+  if (w.active) {
+    float before, after;
+    seg_offsets(w, sPart, before, after);
+    // Qbar = q e^{b}, b the inclusive prefix of the log-gates in scan order, built by
+    // additions only (a -inf gate gives 0, not inf - inf)
+    float acc = before;
+#pragma unroll
+    for (int t = 0; t < kSegMax; ++t) {
+      const int st2 = w.st0 + t;
+      if (st2 < w.st1) {
+        acc += lg[t];
+        __nv_bfloat16* p =
+            reinterpret_cast<__nv_bfloat16*>(sm + L.oQ + sw32_at(MC, (uint32_t)seg_row(st2, rev), (uint32_t)w.i));
+        *p = __float2bfloat16_rn(__bfloat162float(*p) * __expf(acc));
+      }
     }
+    // K^ = k e^{u}, u the exclusive suffix (decays only shrink it); the range check
+    // covers every u and the chunk total
+    acc = after;
+    float lo = acc, hi = acc;
+#pragma unroll
+    for (int t = kSegMax - 1; t >= 0; --t) {
+      const int st2 = w.st0 + t;
+      if (st2 < w.st1) {
+        __nv_bfloat16* p =
+            reinterpret_cast<__nv_bfloat16*>(sm + L.oK + sw32_at(MC, (uint32_t)seg_row(st2, rev), (uint32_t)w.i));
+        *p = __float2bfloat16_rn(__bfloat162float(*p) * __expf(acc));
+        acc += lg[t];
+        lo = fminf(lo, acc);
+        hi = fmaxf(hi, acc);
+      }
+    }
+    if (w.s == 0) a.gamma[cid * a.dk + w.i] = expf(acc);
+    if (!(lo >= -kRange) || !(hi <= kRange)) code |= 1;
+    if (!(hi <= kRange)) code |= 2;
   }
-  __syncthreads();
-  const int code = suffix_sums<MC>(sU, sTot, a.dk, rev, pu);
   if (code & 2) report_status(GLA_ERR_RANGE);
   const int wide = __syncthreads_or(code != 0);
-  // K^ = k e^{u}: the exponent is a sum of log-gates, so decays only shrink it.
-  for (int idx = threadIdx.x; idx < MC * (a.dk / 8); idx += NT) {
-    const int r = idx % MC, cc = idx / MC;
-    uint4* pk = reinterpret_cast<uint4*>(sm + oK + sw32_at(MC, (uint32_t)r, (uint32_t)(cc * 8)));
-    uint4 wk = *pk;
-    uint32_t* uk = reinterpret_cast<uint32_t*>(&wk);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 x = unpack_bf16x2(uk[e]);
-      uk[e] = pack_bf16x2(x.x * expf(sU[r * pu + cc * 8 + 2 * e]), x.y * expf(sU[r * pu + cc * 8 + 2 * e + 1]));
-    }
-    *pk = wk;
-  }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -1039,16 +1176,15 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_local(const BwdArgs<__nv_bfl
   if (threadIdx.x == 0) {
     const uint32_t id = idesc_bf16_f32(MC, (int)Np, true, true);
     for (int kk = 0; kk < MC / 16; ++kk)
-      umma_ss(tbase, dmn(sb + oK, MC, kk), dmn(sb + oV, MC, kk), id, kk > 0 ? 1u : 0u);
+      umma_ss(tbase, dmn(sb + L.oK, MC, kk), dmn(sb + L.oV, MC, kk), id, kk > 0 ? 1u : 0u);
     for (int kk = 0; kk < MC / 16; ++kk)
-      umma_ss(tbase + 128, dmn(sb + oQ, MC, kk), dmn(sb + oO, MC, kk), id, kk > 0 ? 1u : 0u);
+      umma_ss(tbase + 128, dmn(sb + L.oQ, MC, kk), dmn(sb + L.oO, MC, kk), id, kk > 0 ? 1u : 0u);
     umma_commit(bar);
   }
   const bool ok = __syncthreads_and(mbar_wait(bar, 0u));
   if (!ok && threadIdx.x == 0) report_status(GLA_ERR_TIMEOUT);
   tc_fence_after();
   // TMEM lane = key channel i; warps 0-3 write K^T V, warps 4-7 Qbar^T dO.
-  const int64_t cid = (int64_t)bh * a.NC + c;
   if (ok) {
     const int i = 32 * (warp & 3) + lane;
     const uint32_t col = (warp >> 2) ? 128u : 0u;
@@ -1063,7 +1199,6 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_local(const BwdArgs<__nv_bfl
                 make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
     }
   }
-  if (threadIdx.x < a.dk) a.gamma[cid * a.dk + threadIdx.x] = expf(sTot[threadIdx.x]);
   if (threadIdx.x == 0) a.flags[cid] = wide;
   tc_fence_before();
   __syncthreads();
@@ -1123,7 +1258,7 @@ cudaError_t launch_bwd(const BwdArgs<TI>& a, const GlaShape& s, cudaStream_t st)
 // The tensor-core path: gla_bwd_tc_local, the chunk scans over 128-row chunks, then
 // gla_bwd_tc_chunk.
 cudaError_t launch_bwd_tc(const BwdArgs<__nv_bfloat16>& a, const GlaShape& s, cudaStream_t st) {
-  const size_t s1 = kTcLocalBytes(s.dk, s.dv);
+  const size_t s1 = tl_layout(s.dk, s.dv).bytes;
   const TcLayout L = tc_layout(s.dk, s.dv);
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(gla_bwd_tc_local, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1)) !=
