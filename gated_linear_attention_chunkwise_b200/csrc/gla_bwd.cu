@@ -85,7 +85,7 @@ __device__ __forceinline__ void stage(float* dst, const TE* src, int d, const Sc
                                       int H) {
   const int cpr = d / 8;
   const int pitch = pitch_of(d);
-  for (int idx = threadIdx.x; idx < MC * cpr; idx += NT) {
+  for (int idx = threadIdx.x; idx < MC * cpr; idx += blockDim.x) {
     const int r = idx / cpr;
     const int cc = idx - r * cpr;
     const int f = f0 + r;
@@ -567,6 +567,7 @@ __global__ void __launch_bounds__(NT) gla_bwd_chunk(const BwdArgs<TI> a) {
 // ways.  Chunks flagged by kernel 1 take an exact token-by-token sweep instead.
 // ---------------------------------------------------------------------------
 constexpr int kTcRows = 128;
+constexpr int kTcChunkNT = 512;  // threads of the gradient kernel (16 warps, one CTA per SM)
 constexpr uint32_t kLayoutSW32b = 6;  // UMMA layout type of the 32-byte swizzle
 
 __device__ __forceinline__ uint32_t sw32_at(uint32_t rows, uint32_t r, uint32_t ch) {
@@ -587,7 +588,7 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) { tmem_l
 // Token index of each of the chunk's rows (base positions f0 .. f0+127), -1 for rows
 // outside the sequence; the staging and the d log alpha stores index through it.
 __device__ __forceinline__ void tc_row_tokens(int* sRow, const ScanGeom& g, int f0) {
-  for (int r = threadIdx.x; r < kTcRows; r += NT) {
+  for (int r = threadIdx.x; r < kTcRows; r += blockDim.x) {
     const int f = f0 + r;
     sRow[r] = (f >= 0 && f < g.T) ? base_pos_to_token(g, f) : -1;
   }
@@ -605,7 +606,7 @@ template <typename TI>
 __device__ __forceinline__ void tc_stage_bf16(uint8_t* sm, uint32_t tile, const __nv_bfloat16* src, int d, int nch,
                                               const BwdArgs<TI>& a, const int* sRow, int b, int h) {
   const int cc_n = nch / 8;
-  for (int idx = threadIdx.x; idx < kTcRows * cc_n; idx += NT) {
+  for (int idx = threadIdx.x; idx < kTcRows * cc_n; idx += blockDim.x) {
     const int r = idx % kTcRows, cc = idx / kTcRows;
     const int tok = sRow[r];
     const bool valid = tok >= 0 && cc * 8 < d;
@@ -616,7 +617,7 @@ __device__ __forceinline__ void tc_stage_bf16(uint8_t* sm, uint32_t tile, const 
 template <typename TI>
 __device__ __forceinline__ void tc_stage_gates(float* sU, const BwdArgs<TI>& a, const int* sRow, int b, int h) {
   const int cpr = a.dk / 4, pw = a.dk + 4;
-  for (int idx = threadIdx.x; idx < kTcRows * cpr; idx += NT) {
+  for (int idx = threadIdx.x; idx < kTcRows * cpr; idx += blockDim.x) {
     const int r = idx / cpr, cc = idx - r * cpr;
     const int tok = sRow[r];
     const float* p = tok >= 0 ? a.la + tok_off(a, b, h, tok, a.dk) + cc * 4 : a.la;
@@ -625,21 +626,23 @@ __device__ __forceinline__ void tc_stage_gates(float* sU, const BwdArgs<TI>& a, 
 }
 // n fp32 values (a multiple of 4) from src, or zeros when src is null.
 __device__ __forceinline__ void tc_stage_f32(float* dst, const float* src, int n, const float* any) {
-  for (int e = 4 * (int)threadIdx.x; e < n; e += 4 * NT) cp_async16(smem_u32(dst + e), src ? src + e : any, src != nullptr);
+  for (int e = 4 * (int)threadIdx.x; e < n; e += 4 * (int)blockDim.x) cp_async16(smem_u32(dst + e), src ? src + e : any, src != nullptr);
 }
 
 // Segmented walks along a chunk's scan order: thread t takes channel i = t % dk and
-// segment s = t / dk, the scan steps [st0, st1) of nseg nearly equal segments (three
-// for dk > 64, else four; dk <= 80 on this path).  A walk first needs the totals of
-// the other segments (phase 1, one barrier), then runs over its own steps only.
-constexpr int kSegMax = 43;  // ceil(128 / 3)
+// segment s = t / dk, the scan steps [st0, st1) of nseg nearly equal segments, as
+// many as the block has threads for (at most 8; at least 3 for 256 threads and
+// dk <= 80, the widest heads on this path).  A walk first needs the totals of the
+// other segments (phase 1, one barrier), then runs over its own steps only.
+constexpr int kMaxSegs = 8;
+constexpr int kSegMax = 43;  // ceil(128 / 3): the longest segment with 256 threads
 struct SegWalk {
   int i, s, nseg, st0, st1;
   bool active;
 };
 __device__ __forceinline__ SegWalk seg_walk(int dk) {
   SegWalk w;
-  w.nseg = dk > 64 ? 3 : 4;
+  w.nseg = min(kMaxSegs, (int)blockDim.x / dk);
   const int len = (kTcRows + w.nseg - 1) / w.nseg;
   w.i = (int)threadIdx.x % dk;
   w.s = (int)threadIdx.x / dk;
@@ -676,12 +679,12 @@ __device__ void tc_chunk_serial(const BwdArgs<__nv_bfloat16>& a, float* smem, in
   const size_t st = (size_t)a.dk * a.dv;
   const float* sin = c > 0 ? a.sx + (cid - 1) * st : nullptr;
   const float* dd = a.dd + cid * st;
-  for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+  for (int e = threadIdx.x; e < a.dk * a.dv; e += blockDim.x) {
     const int i = e / a.dv, j = e - i * a.dv;
     sGg[i * pv + j] = dd[e];
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < MC * a.dk; e += NT) {
+  for (int e = threadIdx.x; e < MC * a.dk; e += blockDim.x) {
     const int r = e / a.dk, i = e - r * a.dk;
     sAl[r * pk + i] = expf(sAl[r * pk + i]);
   }
@@ -692,7 +695,7 @@ __device__ void tc_chunk_serial(const BwdArgs<__nv_bfloat16>& a, float* smem, in
     const bool real = f >= 0 && f < a.g.T;
     const int64_t ok = real ? row_off(a, b, h, f, a.dk) : 0;
     const int64_t ov = real ? row_off(a, b, h, f, a.dv) : 0;
-    for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+    for (int e = threadIdx.x; e < a.dk * a.dv; e += blockDim.x) {
       const int i = e / a.dv, j = e - i * a.dv;
       float w = sin ? sin[e] : 0.f;
       for (int s2 = 0; s2 < step; ++s2) {
@@ -706,7 +709,7 @@ __device__ void tc_chunk_serial(const BwdArgs<__nv_bfloat16>& a, float* smem, in
       }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < a.dk; i += NT) {
+    for (int i = threadIdx.x; i < a.dk; i += blockDim.x) {
       const float al = sAl[r * pk + i], ki = sK[r * pk + i];
       float gq = 0.f, gk = 0.f, gl = 0.f;
       for (int j = 0; j < a.dv; ++j) {
@@ -721,13 +724,13 @@ __device__ void tc_chunk_serial(const BwdArgs<__nv_bfloat16>& a, float* smem, in
         a.dla[ok + i] = al * gl;
       }
     }
-    for (int j = threadIdx.x; j < a.dv; j += NT) {
+    for (int j = threadIdx.x; j < a.dv; j += blockDim.x) {
       float gv = 0.f;
       for (int i = 0; i < a.dk; ++i) gv = fmaf(sK[r * pk + i], sGg[i * pv + j], gv);
       if (real) store1(a.dv_out + ov + j, gv);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < a.dk * a.dv; e += NT) {
+    for (int e = threadIdx.x; e < a.dk * a.dv; e += blockDim.x) {
       const int i = e / a.dv, j = e - i * a.dv;
       sGg[i * pv + j] *= sAl[r * pk + i];
     }
@@ -752,14 +755,14 @@ __host__ __device__ inline TcLayout tc_layout(int dk, int dv) {
   L.oD = L.oG + (Np / 16) * Kp * 32u;
   L.oU = L.oD + (Np / 16) * Kp * 32u;
   L.oMisc = (L.oU + (uint32_t)kTcRows * (uint32_t)(dk + 4) * 4u + 15u) / 16u * 16u;
-  // gate totals, e^{totals}, carry (128 floats each), segment totals (4 x 128), row
+  // gate totals, e^{totals}, carry (128 floats each), segment totals (8 x 128), row
   // tokens (128), barrier and TMEM address; alignment slack
-  L.bytes = L.oMisc + 3u * 512u + 2048u + 512u + 64u + 1024u;
+  L.bytes = L.oMisc + 3u * 512u + 4096u + 512u + 64u + 1024u;
   L.nst = 3u * (uint32_t)dk * (uint32_t)dv * 4u <= 2u * 8u * kTcRows * 32u ? 3 : 2;
   return L;
 }
 
-__global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfloat16> a) {
+__global__ void __launch_bounds__(kTcChunkNT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfloat16> a) {
   extern __shared__ __align__(1024) uint8_t smem_raw_tc[];
   // Swizzled operand tiles start on a 1024-byte boundary.
   uint8_t* smem_tc = smem_raw_tc + ((1024u - (smem_u32(smem_raw_tc) & 1023u)) & 1023u);
@@ -773,8 +776,8 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
   float* sTot = reinterpret_cast<float*>(smem_tc + L.oMisc);
   float* sGam = sTot + 128;
   float* sCarry = sGam + 128;
-  float* sPart = sCarry + 128;                            // [4][128] segment totals
-  int* sRow = reinterpret_cast<int*>(sPart + 4 * 128);    // [128] row tokens
+  float* sPart = sCarry + 128;                            // [8][128] segment totals
+  int* sRow = reinterpret_cast<int*>(sPart + kMaxSegs * 128);  // [128] row tokens
   uint64_t* sBar = reinterpret_cast<uint64_t*>(sRow + 128);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sBar + 1);
   // fp32 chunk states, staged over the A and P tiles (written only after the first MMAs)
@@ -843,7 +846,7 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
   {
     // Q~ = q e^{-u}, K^ = k e^{u} in place (8 channels per thread), padding stays 0
     const int cq = (int)Kp / 8;
-    for (int idx = threadIdx.x; idx < MC * cq; idx += NT) {
+    for (int idx = threadIdx.x; idx < MC * cq; idx += blockDim.x) {
       const int r = idx % MC, cc = idx / MC;
       if (cc * 8 >= a.dk) continue;
       uint4* pq = reinterpret_cast<uint4*>(smem_tc + L.oQ + sw32_at(MC, (uint32_t)r, (uint32_t)(cc * 8)));
@@ -861,21 +864,28 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
       *pq = wq;
       *pk = wk;
     }
-    // G[i][j] = e^{g_i} S_in[i][j] and D[i][j] as bf16 tiles, rows i < Kp, channels j < Np
-    const int nG = (int)(Kp * Np);
-    for (int e = threadIdx.x; e < nG; e += NT) {
-      const int i = e / (int)Np, j = e - i * (int)Np;
-      const bool in = i < a.dk && j < a.dv;
-      const float gv = in ? sGam[i] * sSin[i * a.dv + j] : 0.f;
-      const float dv_ = in ? sDs[i * a.dv + j] : 0.f;
-      *reinterpret_cast<__nv_bfloat16*>(smem_tc + L.oG + sw32_at(Kp, (uint32_t)i, (uint32_t)j)) =
-          __float2bfloat16_rn(gv);
-      *reinterpret_cast<__nv_bfloat16*>(smem_tc + L.oD + sw32_at(Kp, (uint32_t)i, (uint32_t)j)) =
-          __float2bfloat16_rn(dv_);
+    // G[i][j] = e^{g_i} S_in[i][j] and D[i][j] as bf16 tiles, rows i < Kp, channels
+    // j < Np, eight channels (one 16-byte tile row piece) per item; dv is a multiple of 8
+    const int n8 = (int)Np / 8;
+    for (int idx = threadIdx.x; idx < (int)Kp * n8; idx += blockDim.x) {
+      const int i = idx / n8, j0 = 8 * (idx - i * n8);
+      uint4 wg = make_uint4(0u, 0u, 0u, 0u), wd = wg;
+      if (i < a.dk && j0 < a.dv) {
+        const float4* ps = reinterpret_cast<const float4*>(sSin + i * a.dv + j0);
+        const float4* pd = reinterpret_cast<const float4*>(sDs + i * a.dv + j0);
+        const float4 s0 = ps[0], s1 = ps[1], d0 = pd[0], d1 = pd[1];
+        const float gm = sGam[i];
+        wg = make_uint4(pack_bf16x2(gm * s0.x, gm * s0.y), pack_bf16x2(gm * s0.z, gm * s0.w),
+                        pack_bf16x2(gm * s1.x, gm * s1.y), pack_bf16x2(gm * s1.z, gm * s1.w));
+        wd = make_uint4(pack_bf16x2(d0.x, d0.y), pack_bf16x2(d0.z, d0.w), pack_bf16x2(d1.x, d1.y),
+                        pack_bf16x2(d1.z, d1.w));
+      }
+      *reinterpret_cast<uint4*>(smem_tc + L.oG + sw32_at(Kp, (uint32_t)i, (uint32_t)j0)) = wg;
+      *reinterpret_cast<uint4*>(smem_tc + L.oD + sw32_at(Kp, (uint32_t)i, (uint32_t)j0)) = wd;
     }
     // carry[i] = sum_j D[i][j] S_out[i][j]: one warp per row, a fixed shuffle tree
     if (L.nst == 3) {
-      for (int i = warp; i < a.dk; i += NT / 32) {
+      for (int i = warp; i < a.dk; i += (int)(blockDim.x >> 5)) {
         float acc = 0.f;
         for (int j = lane; j < a.dv; j += 32) acc = fmaf(sDs[i * a.dv + j], sSo[i * a.dv + j], acc);
 #pragma unroll
@@ -904,16 +914,17 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
   ok = __syncthreads_and(mbar_wait(bar, 0u));
   if (!ok && threadIdx.x == 0) report_status(GLA_ERR_TIMEOUT);
   tc_fence_after();
-  // ---- mask and round: lane = row r (TMEM lane), warp pair splits the 128 columns
-  const int qd = warp & 3, hf = warp >> 2;
+  // ---- mask and round: lane = row r (TMEM lane); the four warps of a lane quarter
+  // split the 128 columns into quarters
+  const int qd = warp & 3, hf = warp >> 2;  // hf: column quarter
   const int r = 32 * qd + lane;
   const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
   if (ok) {
     for (int which = 0; which < 2; ++which) {
       const uint32_t col = which ? cP : cA;
       const uint32_t tile = which ? L.oP : L.oA;
-      for (int g = 0; g < 4; ++g) {
-        const int s0 = 64 * hf + 16 * g;
+      for (int g = 0; g < 2; ++g) {
+        const int s0 = 32 * hf + 16 * g;
         float x[16];
         tc_ld16(tbase + lane_base + col + (uint32_t)s0, x);
         uint32_t wv[8];
@@ -961,13 +972,13 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
     if (!ok && threadIdx.x == 0) report_status(GLA_ERR_TIMEOUT);
   }
   tc_fence_after();
-  // ---- epilogue: row r, 16-channel groups g with g % 2 == hf
+  // ---- epilogue: row r, 16-channel groups g with g % 4 == hf
   const int tok = sRow[r];
   const bool real = tok >= 0;
   if (ok) {
     // q dq - k dk = Q~ dQ~ - K^ dK^, with Q~ and K^ the bf16 tiles of the MMAs.
     const int64_t ok_ = real ? tok_off(a, b, h, tok, a.dk) : 0;
-    for (int g = hf; g < (int)Kp / 16; g += 2) {
+    for (int g = hf; g < (int)Kp / 16; g += 4) {
       float xq[16], xk[16];
       tc_ld16(tbase + lane_base + cDQ + (uint32_t)(16 * g), xq);
       tc_ld16(tbase + lane_base + cDK + (uint32_t)(16 * g), xk);
@@ -998,7 +1009,7 @@ __global__ void __launch_bounds__(NT, 1) gla_bwd_tc_chunk(const BwdArgs<__nv_bfl
       }
     }
     const int64_t ov_ = real ? tok_off(a, b, h, tok, a.dv) : 0;
-    for (int g = hf; g < (int)Np / 16; g += 2) {
+    for (int g = hf; g < (int)Np / 16; g += 4) {
       float xv[16];
       tc_ld16(tbase + lane_base + cDV + (uint32_t)(16 * g), xv);
       for (int half = 0; half < 2; ++half) {
@@ -1069,8 +1080,8 @@ __host__ __device__ inline TlLayout tl_layout(int dk, int dv) {
   const uint32_t end = L.oO + Np / 16 * kTcRows * 32u;
   const uint32_t reach = L.oQ + 8u * kTcRows * 32u;  // the q operand's last MMA read
   L.oMisc = end > reach ? end : reach;
-  // segment totals (4 x 128 floats), row tokens (128), barrier, TMEM address; slack
-  L.bytes = L.oMisc + 2048u + 512u + 64u + 1024u;
+  // segment totals (8 x 128 floats), row tokens (128), barrier, TMEM address; slack
+  L.bytes = L.oMisc + 4096u + 512u + 64u + 1024u;
   return L;
 }
 
@@ -1082,8 +1093,8 @@ __global__ void __launch_bounds__(NT, 2) gla_bwd_tc_local(const BwdArgs<__nv_bfl
   const int b = bh / a.H, h = bh % a.H;
   const uint32_t Kp = (uint32_t)(a.dk + 15) / 16 * 16, Np = (uint32_t)(a.dv + 15) / 16 * 16;
   const TlLayout L = tl_layout(a.dk, a.dv);
-  float* sPart = reinterpret_cast<float*>(sm + L.oMisc);  // [4][128] segment totals
-  int* sRow = reinterpret_cast<int*>(sPart + 4 * 128);
+  float* sPart = reinterpret_cast<float*>(sm + L.oMisc);  // [8][128] segment totals
+  int* sRow = reinterpret_cast<int*>(sPart + kMaxSegs * 128);
   uint64_t* sBar = reinterpret_cast<uint64_t*>(sRow + 128);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sBar + 1);
   const uint32_t sb = smem_u32(sm);
@@ -1272,7 +1283,7 @@ cudaError_t launch_bwd_tc(const BwdArgs<__nv_bfloat16>& a, const GlaShape& s, cu
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   gla_bwd_scan<__nv_bfloat16><<<dim3((s.dk * s.dv + 255) / 256, s.B * s.H), 256, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  gla_bwd_tc_chunk<<<grid, NT, L.bytes, st>>>(a);
+  gla_bwd_tc_chunk<<<grid, kTcChunkNT, L.bytes, st>>>(a);
   return cudaGetLastError();
 }
 
