@@ -584,6 +584,26 @@ __device__ __forceinline__ uint64_t dmn(uint32_t tile, uint32_t rows, int kk) {
 }
 
 __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) { tmem_ld16(taddr, v); }
+// 16-column TMEM load without its wait (several loads share one tcgen05.wait::ld),
+// and the tie that orders every later use of the registers after that wait.
+__device__ __forceinline__ void tc_ld16_issue(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tc_tie16(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]));
+}
+// Waits until at most N of this thread's cp.async groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Token index of each of the chunk's rows (base positions f0 .. f0+127), -1 for rows
 // outside the sequence; the staging and the d log alpha stores index through it.
@@ -631,11 +651,9 @@ __device__ __forceinline__ void tc_stage_f32(float* dst, const float* src, int n
 
 // Segmented walks along a chunk's scan order: thread t takes channel i = t % dk and
 // segment s = t / dk, the scan steps [st0, st1) of nseg nearly equal segments, as
-// many as the block has threads for (at most 8; at least 3 for 256 threads and
-// dk <= 80, the widest heads on this path).  A walk first needs the totals of the
+// many as the block has threads for (at most 8).  A walk first needs the totals of the
 // other segments (phase 1, one barrier), then runs over its own steps only.
 constexpr int kMaxSegs = 8;
-constexpr int kSegMax = 43;  // ceil(128 / 3): the longest segment with 256 threads
 struct SegWalk {
   int i, s, nseg, st0, st1;
   bool active;
@@ -660,6 +678,25 @@ __device__ __forceinline__ void seg_offsets(const SegWalk& w, const float* sPart
   for (int s2 = w.nseg - 1; s2 > w.s; --s2) after += sPart[s2 * kTcRows + w.i];
 }
 __device__ __forceinline__ int seg_row(int st, bool rev) { return rev ? (kTcRows - 1 - st) : st; }
+// The same segmentation over channel pairs (p = t % (dk/2)): 6 to 8 segments of at
+// most kPairSegMax steps for dk <= 80 and 256 threads.
+constexpr int kPairSegMax = 22;  // ceil(128 / 6)
+struct PairWalk {
+  int p, s, nseg, st0, st1;
+  bool active;
+};
+__device__ __forceinline__ PairWalk pair_walk(int dk) {
+  const int np = dk / 2;
+  PairWalk w;
+  w.nseg = min(kMaxSegs, (int)blockDim.x / np);
+  const int len = (kTcRows + w.nseg - 1) / w.nseg;
+  w.p = (int)threadIdx.x % np;
+  w.s = (int)threadIdx.x / np;
+  w.active = w.s < w.nseg;
+  w.st0 = w.s * len;
+  w.st1 = min(w.st0 + len, kTcRows);
+  return w;
+}
 
 
 // Exact sweep of a flagged chunk from fp32 tiles (alpha, k, v) staged in shared
@@ -806,18 +843,21 @@ __global__ void __launch_bounds__(kTcChunkNT, 1) gla_bwd_tc_chunk(const BwdArgs<
   }
   tc_row_tokens(sRow, a.g, f0);
   __syncthreads();
-  // ---- staging, all in flight together: log-gates (fp32), q, k, v, dout (bf16,
-  // swizzled, zero past the channels and rows), S_in, D and (when it fits) S_out
+  // ---- staging, all in flight together, in three groups waited for in the order of
+  // use: log-gates (fp32); q, k (bf16, swizzled, zero past the channels and rows);
+  // v, dout, S_in, D and (when it fits) S_out
   tc_stage_gates(sU, a, sRow, b, h);
+  cp_async_commit();
   tc_stage_bf16(smem_tc, L.oQ, a.q, a.dk, (int)Kp, a, sRow, b, h);
   tc_stage_bf16(smem_tc, L.oK, a.k, a.dk, (int)Kp, a, sRow, b, h);
+  cp_async_commit();
   tc_stage_bf16(smem_tc, L.oV, a.v, a.dv, (int)Np, a, sRow, b, h);
   tc_stage_bf16(smem_tc, L.oO, a.dout, a.dv, (int)Np, a, sRow, b, h);
   tc_stage_f32(sSin, c > 0 ? a.sx + (cid - 1) * st : nullptr, dkv, a.la);
   tc_stage_f32(sDs, a.dd + cid * st, dkv, a.la);
   if (L.nst == 3) tc_stage_f32(sSo, a.sx + cid * st, dkv, a.la);
   cp_async_commit();
-  cp_async_wait_all();
+  cp_async_wait_group<2>();
   __syncthreads();
   // ---- u: exclusive suffix sums of the log-gates in scan order, in place (segmented)
   const SegWalk w = seg_walk(a.dk);
@@ -842,6 +882,7 @@ __global__ void __launch_bounds__(kTcChunkNT, 1) gla_bwd_tc_chunk(const BwdArgs<
       sGam[w.i] = expf(acc);
     }
   }
+  cp_async_wait_group<1>();
   __syncthreads();
   {
     // Q~ = q e^{-u}, K^ = k e^{u} in place (8 channels per thread), padding stays 0
@@ -864,6 +905,8 @@ __global__ void __launch_bounds__(kTcChunkNT, 1) gla_bwd_tc_chunk(const BwdArgs<
       *pq = wq;
       *pk = wk;
     }
+    cp_async_wait_group<0>();
+    __syncthreads();
     // G[i][j] = e^{g_i} S_in[i][j] and D[i][j] as bf16 tiles, rows i < Kp, channels
     // j < Np, eight channels (one 16-byte tile row piece) per item; dv is a multiple of 8
     const int n8 = (int)Np / 8;
@@ -923,10 +966,18 @@ __global__ void __launch_bounds__(kTcChunkNT, 1) gla_bwd_tc_chunk(const BwdArgs<
     for (int which = 0; which < 2; ++which) {
       const uint32_t col = which ? cP : cA;
       const uint32_t tile = which ? L.oP : L.oA;
+      uint32_t xr[2][16];
+      tc_ld16_issue(tbase + lane_base + col + (uint32_t)(32 * hf), xr[0]);
+      tc_ld16_issue(tbase + lane_base + col + (uint32_t)(32 * hf + 16), xr[1]);
+      tmem_ld_wait();
+      tc_tie16(xr[0]);
+      tc_tie16(xr[1]);
+#pragma unroll
       for (int g = 0; g < 2; ++g) {
         const int s0 = 32 * hf + 16 * g;
         float x[16];
-        tc_ld16(tbase + lane_base + col + (uint32_t)s0, x);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(xr[g][e]);
         uint32_t wv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -1065,8 +1116,8 @@ __global__ void __launch_bounds__(kTcChunkNT, 1) gla_bwd_tc_chunk(const BwdArgs<
 // MN-major (M = key channels).  The tiles hold Kp channels; the MMA's A rows past Kp
 // read whatever follows a tile (the next tile) and only reach accumulator rows past
 // dk, which are never stored, so the tiles sit back to back and two CTAs fit per SM.
-// Each thread (channel, segment) holds its log-gates in registers and gates Qbar and
-// K^ during its two walks: no fp32 gate tile is staged.
+// Each thread (channel pair, segment) holds its log-gates in registers and gates Qbar
+// and K^ during its two walks: no fp32 gate tile is staged.
 struct TlLayout {
   uint32_t oK, oQ, oV, oO, oMisc, bytes;
 };
@@ -1117,62 +1168,96 @@ __global__ void __launch_bounds__(NT, 2) gla_bwd_tc_local(const BwdArgs<__nv_bfl
   tc_stage_bf16(sm, L.oV, a.v, a.dv, (int)Np, a, sRow, b, h);
   tc_stage_bf16(sm, L.oO, a.dout, a.dv, (int)Np, a, sRow, b, h);
   cp_async_commit();
-  // This thread's log-gates (its channel, its segment's rows) into registers while
-  // the tiles arrive; then the segment's total.
-  const SegWalk w = seg_walk(a.dk);
-  float lg[kSegMax];
+  // This thread's log-gates (its channel pair, its segment's rows) into registers
+  // while the tiles arrive; then the segment's totals.
+  const PairWalk w = pair_walk(a.dk);
+  float2 lg[kPairSegMax];
 #pragma unroll
-  for (int t = 0; t < kSegMax; ++t) {
+  for (int t = 0; t < kPairSegMax; ++t) {
     const int st2 = w.st0 + t;
-    float x = 0.f;
+    float2 x = make_float2(0.f, 0.f);
     if (w.active && st2 < w.st1) {
       const int tk = sRow[seg_row(st2, rev)];
-      if (tk >= 0) x = a.la[tok_off(a, b, h, tk, a.dk) + w.i];
+      if (tk >= 0) x = *reinterpret_cast<const float2*>(a.la + tok_off(a, b, h, tk, a.dk) + 2 * w.p);
     }
     lg[t] = x;
   }
   if (w.active) {
-    float t = 0.f;
+    float2 t = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int t2 = 0; t2 < kSegMax; ++t2) t += lg[t2];
-    sPart[w.s * MC + w.i] = t;
+    for (int t2 = 0; t2 < kPairSegMax; ++t2) {
+      t.x += lg[t2].x;
+      t.y += lg[t2].y;
+    }
+    sPart[w.s * MC + 2 * w.p] = t.x;
+    sPart[w.s * MC + 2 * w.p + 1] = t.y;
   }
   cp_async_wait_all();
   __syncthreads();
   int code = 0;
   if (w.active) {
-    float before, after;
-    seg_offsets(w, sPart, before, after);
+    float2 before = make_float2(0.f, 0.f), after = make_float2(0.f, 0.f);
+    for (int s2 = 0; s2 < w.s; ++s2) {
+      before.x += sPart[s2 * MC + 2 * w.p];
+      before.y += sPart[s2 * MC + 2 * w.p + 1];
+    }
+    for (int s2 = w.nseg - 1; s2 > w.s; --s2) {
+      after.x += sPart[s2 * MC + 2 * w.p];
+      after.y += sPart[s2 * MC + 2 * w.p + 1];
+    }
+    // Each walk loads its segment's pairs, gates them, then stores them all.
+    uint32_t x[kPairSegMax];
+    // tile offset of this thread's pair in scan step st2
+    auto pair_at = [&](uint32_t tile, int st2) {
+      return tile + sw32_at(MC, (uint32_t)seg_row(st2, rev), (uint32_t)(2 * w.p));
+    };
     // Qbar = q e^{b}, b the inclusive prefix of the log-gates in scan order, built by
     // additions only (a -inf gate gives 0, not inf - inf)
-    float acc = before;
 #pragma unroll
-    for (int t = 0; t < kSegMax; ++t) {
+    for (int t = 0; t < kPairSegMax; ++t) {
       const int st2 = w.st0 + t;
-      if (st2 < w.st1) {
-        acc += lg[t];
-        __nv_bfloat16* p =
-            reinterpret_cast<__nv_bfloat16*>(sm + L.oQ + sw32_at(MC, (uint32_t)seg_row(st2, rev), (uint32_t)w.i));
-        *p = __float2bfloat16_rn(__bfloat162float(*p) * __expf(acc));
+      if (st2 < w.st1) x[t] = *reinterpret_cast<const uint32_t*>(sm + pair_at(L.oQ, st2));
+    }
+    float2 acc = before;
+#pragma unroll
+    for (int t = 0; t < kPairSegMax; ++t) {
+      if (w.st0 + t < w.st1) {
+        acc.x += lg[t].x;
+        acc.y += lg[t].y;
+        const float2 xq = unpack_bf16x2(x[t]);
+        x[t] = pack_bf16x2(xq.x * __expf(acc.x), xq.y * __expf(acc.y));
       }
     }
+#pragma unroll
+    for (int t = 0; t < kPairSegMax; ++t)
+      if (w.st0 + t < w.st1) *reinterpret_cast<uint32_t*>(sm + pair_at(L.oQ, w.st0 + t)) = x[t];
     // K^ = k e^{u}, u the exclusive suffix (decays only shrink it); the range check
     // covers every u and the chunk total
-    acc = after;
-    float lo = acc, hi = acc;
 #pragma unroll
-    for (int t = kSegMax - 1; t >= 0; --t) {
+    for (int t = 0; t < kPairSegMax; ++t) {
       const int st2 = w.st0 + t;
-      if (st2 < w.st1) {
-        __nv_bfloat16* p =
-            reinterpret_cast<__nv_bfloat16*>(sm + L.oK + sw32_at(MC, (uint32_t)seg_row(st2, rev), (uint32_t)w.i));
-        *p = __float2bfloat16_rn(__bfloat162float(*p) * __expf(acc));
-        acc += lg[t];
-        lo = fminf(lo, acc);
-        hi = fmaxf(hi, acc);
+      if (st2 < w.st1) x[t] = *reinterpret_cast<const uint32_t*>(sm + pair_at(L.oK, st2));
+    }
+    acc = after;
+    float lo = fminf(acc.x, acc.y), hi = fmaxf(acc.x, acc.y);
+#pragma unroll
+    for (int t = kPairSegMax - 1; t >= 0; --t) {
+      if (w.st0 + t < w.st1) {
+        const float2 xk = unpack_bf16x2(x[t]);
+        x[t] = pack_bf16x2(xk.x * __expf(acc.x), xk.y * __expf(acc.y));
+        acc.x += lg[t].x;
+        acc.y += lg[t].y;
+        lo = fminf(lo, fminf(acc.x, acc.y));
+        hi = fmaxf(hi, fmaxf(acc.x, acc.y));
       }
     }
-    if (w.s == 0) a.gamma[cid * a.dk + w.i] = expf(acc);
+#pragma unroll
+    for (int t = 0; t < kPairSegMax; ++t)
+      if (w.st0 + t < w.st1) *reinterpret_cast<uint32_t*>(sm + pair_at(L.oK, w.st0 + t)) = x[t];
+    if (w.s == 0) {
+      a.gamma[cid * a.dk + 2 * w.p] = expf(acc.x);
+      a.gamma[cid * a.dk + 2 * w.p + 1] = expf(acc.y);
+    }
     if (!(lo >= -kRange) || !(hi <= kRange)) code |= 1;
     if (!(hi <= kRange)) code |= 2;
   }
