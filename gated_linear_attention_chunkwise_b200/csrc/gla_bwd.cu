@@ -256,54 +256,77 @@ __global__ void __launch_bounds__(NT) gla_bwd_local(const BwdArgs<TI> a) {
 // S_in(c+1) = gamma_c S_in(c) + (K^T V)_c and the reverse scan
 // D(c-1) = gamma_c D(c) + (Qbar^T dO)_c, each written over its local term.
 // ---------------------------------------------------------------------------
+// Each thread takes four consecutive state elements of one row i (dv is a multiple of
+// 8, so a group never crosses a row) as float4.  Chunks go in batches of kScanBatch
+// held in two register sets: the next batch's loads are in flight while the current
+// one is folded, so the scan is not one memory latency per chunk.
+constexpr int kScanBatch = 8;
 template <typename TI>
 __global__ void __launch_bounds__(256) gla_bwd_scan(const BwdArgs<TI> a) {
   const int bh = blockIdx.y;
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= a.dk * a.dv) return;
-  const int i = e / a.dv;
-  const size_t st = (size_t)a.dk * a.dv;
-  float* sx = a.sx + (size_t)bh * a.NC * st + e;
-  float* dd = a.dd + (size_t)bh * a.NC * st + e;
+  const int e4 = blockIdx.x * blockDim.x + threadIdx.x;
+  if (4 * e4 >= a.dk * a.dv) return;
+  const int i = 4 * e4 / a.dv;
+  const size_t st4 = (size_t)a.dk * a.dv / 4;
+  float4* sx = reinterpret_cast<float4*>(a.sx) + (size_t)bh * a.NC * st4 + e4;
+  float4* dd = reinterpret_cast<float4*>(a.dd) + (size_t)bh * a.NC * st4 + e4;
   const float* gam = a.gamma + (size_t)bh * a.NC * a.dk + i;
-  // Batches of kBatch chunks: the loads of a batch are issued before its dependent
-  // chain of fmas, so the scan is not one memory latency per chunk.
-  constexpr int kBatch = 32;
-  float S = 0.f;
-  for (int c0 = 0; c0 < a.NC; c0 += kBatch) {
-    float x[kBatch], gm[kBatch];
+  const int NC = a.NC;
+  float4 xa[kScanBatch], xb[kScanBatch];
+  float ga[kScanBatch], gb[kScanBatch];
+  // chunks c0, c0 + dir, ... (kScanBatch of them, those inside [0, NC))
+  auto load = [&](const float4* src, int c0, int dir, float4 (&x)[kScanBatch], float (&g)[kScanBatch]) {
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int c = c0 + u;
-      x[u] = c < a.NC ? sx[c * st] : 0.f;
-      gm[u] = c < a.NC ? gam[(size_t)c * a.dk] : 0.f;
+    for (int u = 0; u < kScanBatch; ++u) {
+      const int c = c0 + dir * u;
+      const bool in = c >= 0 && c < NC;
+      x[u] = in ? src[(size_t)c * st4] : make_float4(0.f, 0.f, 0.f, 0.f);
+      g[u] = in ? gam[(size_t)c * a.dk] : 0.f;
     }
+  };
+  // forward: S_in(c+1) = gamma_c S_in(c) + (K^T V)_c, written over the local term
+  auto fwd = [&](int c0, const float4 (&x)[kScanBatch], const float (&g)[kScanBatch], float4& S) {
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
+    for (int u = 0; u < kScanBatch; ++u) {
       const int c = c0 + u;
-      if (c < a.NC) {
-        S = fmaf(gm[u], S, x[u]);
-        sx[c * st] = S;
+      if (c < NC) {
+        S.x = fmaf(g[u], S.x, x[u].x);
+        S.y = fmaf(g[u], S.y, x[u].y);
+        S.z = fmaf(g[u], S.z, x[u].z);
+        S.w = fmaf(g[u], S.w, x[u].w);
+        sx[(size_t)c * st4] = S;
       }
     }
-  }
-  float D = 0.f;
-  for (int c0 = a.NC - 1; c0 >= 0; c0 -= kBatch) {
-    float x[kBatch], gm[kBatch];
+  };
+  // reverse: D(c) is written over the local term, then D(c-1) = gamma_c D(c) + (Qbar^T dO)_c
+  auto rev = [&](int c0, const float4 (&x)[kScanBatch], const float (&g)[kScanBatch], float4& D) {
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int c = c0 - u;
-      x[u] = c >= 0 ? dd[c * st] : 0.f;
-      gm[u] = c >= 0 ? gam[(size_t)c * a.dk] : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
+    for (int u = 0; u < kScanBatch; ++u) {
       const int c = c0 - u;
       if (c >= 0) {
-        dd[c * st] = D;
-        D = fmaf(gm[u], D, x[u]);
+        dd[(size_t)c * st4] = D;
+        D.x = fmaf(g[u], D.x, x[u].x);
+        D.y = fmaf(g[u], D.y, x[u].y);
+        D.z = fmaf(g[u], D.z, x[u].z);
+        D.w = fmaf(g[u], D.w, x[u].w);
       }
     }
+  };
+  float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
+  load(sx, 0, 1, xa, ga);
+  for (int c0 = 0; c0 < NC; c0 += 2 * kScanBatch) {
+    load(sx, c0 + kScanBatch, 1, xb, gb);
+    fwd(c0, xa, ga, S);
+    load(sx, c0 + 2 * kScanBatch, 1, xa, ga);
+    fwd(c0 + kScanBatch, xb, gb, S);
+  }
+  float4 D = make_float4(0.f, 0.f, 0.f, 0.f);
+  load(dd, NC - 1, -1, xa, ga);
+  for (int c0 = NC - 1; c0 >= 0; c0 -= 2 * kScanBatch) {
+    load(dd, c0 - kScanBatch, -1, xb, gb);
+    rev(c0, xa, ga, D);
+    load(dd, c0 - 2 * kScanBatch, -1, xa, ga);
+    rev(c0 - kScanBatch, xb, gb, D);
   }
 }
 
@@ -1345,7 +1368,7 @@ cudaError_t launch_bwd(const BwdArgs<TI>& a, const GlaShape& s, cudaStream_t st)
   const dim3 grid(a.NC, s.B * s.H);
   gla_bwd_local<TI, MC><<<grid, NT, s1, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  gla_bwd_scan<TI><<<dim3((s.dk * s.dv + 255) / 256, s.B * s.H), 256, 0, st>>>(a);
+  gla_bwd_scan<TI><<<dim3((s.dk * s.dv / 4 + 255) / 256, s.B * s.H), 256, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   chunk_kernel<<<grid, NT, s3, st>>>(a);
   return cudaGetLastError();
@@ -1366,7 +1389,7 @@ cudaError_t launch_bwd_tc(const BwdArgs<__nv_bfloat16>& a, const GlaShape& s, cu
   const dim3 grid(a.NC, s.B * s.H);
   gla_bwd_tc_local<<<grid, NT, s1, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  gla_bwd_scan<__nv_bfloat16><<<dim3((s.dk * s.dv + 255) / 256, s.B * s.H), 256, 0, st>>>(a);
+  gla_bwd_scan<__nv_bfloat16><<<dim3((s.dk * s.dv / 4 + 255) / 256, s.B * s.H), 256, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   gla_bwd_tc_chunk<<<grid, kTcChunkNT, L.bytes, st>>>(a);
   return cudaGetLastError();
