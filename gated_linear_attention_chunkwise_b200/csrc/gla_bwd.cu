@@ -1,5 +1,6 @@
-// gla_bwd.cu -- chunk-wise GLA backward on CUDA cores (fp32 arithmetic; bf16 or
-// fp32 q/k/v/dout/dq/dk/dv, fp32 log-gates and their gradient).
+// gla_bwd.cu -- chunk-wise GLA backward: bf16 q/k/v/dout/dq/dk/dv with dk, dv <= 80
+// on tensor cores (tcgen05, bf16 operands, fp32 accumulation), everything else on
+// CUDA cores in fp32; fp32 log-gates and their gradient.
 //
 // The gradient of the recurrence S_t = Diag(alpha_t) S_{t-1} + k_t^T v_t,
 // o_t = q_t S_t (DiG trains like DiT, so the GLA layers are differentiated) is
@@ -21,9 +22,10 @@
 // chunk is the gradient of a scalar gate placed at the chunk's end,
 // carry_c[i] = sum_j D(c)[i][j] S_in(c+1)[i][j], so every chunk finishes on its own.
 //
-// Chunks of 32 scan positions.  Three kernels: per-chunk local terms (K^T V and Qbar^T dO), the two scans over
-// chunks (one thread per state element), and the per-chunk gradients.  Chunks
-// whose gates leave the fp32-safe range (|u| > 80, e.g. a full reset) take an exact
+// Three kernels: per-chunk local terms (K^T V and Qbar^T dO), the two scans over
+// chunks (four state elements per thread), and the per-chunk gradients.  Chunks of
+// 128 scan positions on the tensor-core path, 32 on the CUDA-core one.  Chunks whose
+// gates leave the fp32-safe range (|u| > 80, e.g. a full reset) take an exact
 // token-by-token reverse sweep from S_in and D instead of the factorised form.
 #include <math.h>
 
@@ -596,14 +598,22 @@ constexpr uint32_t kLayoutSW32b = 6;  // UMMA layout type of the 32-byte swizzle
 __device__ __forceinline__ uint32_t sw32_at(uint32_t rows, uint32_t r, uint32_t ch) {
   return (ch >> 4) * (rows * 32u) + r * 32u + (((((ch >> 3) & 1u) ^ (r >> 2)) & 1u) << 4) + (ch & 7u) * 2u;
 }
-// K-major operand of a tile with `rows` rows: K step kk = channels 16kk..16kk+15.
-__device__ __forceinline__ uint64_t dkm(uint32_t tile, uint32_t rows, int kk) {
-  return umma_desc(tile + (uint32_t)kk * rows * 32u, 16u, 256u, kLayoutSW32b);
+// Operand descriptors of a tile with `rows` rows: K-major (rows = M or N, K step kk =
+// channels 16kk..16kk+15, one 32-byte-swizzled block of rows * 32 bytes each) or
+// MN-major (MN = channels, K step kk = rows 16kk..16kk+15, 512 bytes further).
+// The K steps of one operand: step kk's descriptor is the first one with its start
+// address field (the byte address / 16) advanced by kk * inc.  Tiles lie below 256 KB
+// of shared memory, so the field never carries into the next one; an MMA then costs
+// its issuing thread one add per operand instead of a descriptor build.
+struct OpSteps {
+  uint64_t d0, inc;
+  __device__ __forceinline__ uint64_t at(int kk) const { return d0 + (uint64_t)kk * inc; }
+};
+__device__ __forceinline__ OpSteps km_steps(uint32_t tile, uint32_t rows) {
+  return OpSteps{umma_desc(tile, 16u, 256u, kLayoutSW32b), (uint64_t)(rows * 32u >> 4)};
 }
-// MN-major operand (MN = channels, K = rows) of a tile with `rows` rows: K step kk =
-// rows 16kk..16kk+15.
-__device__ __forceinline__ uint64_t dmn(uint32_t tile, uint32_t rows, int kk) {
-  return umma_desc(tile + (uint32_t)kk * 512u, rows * 32u, 256u, kLayoutSW32b);
+__device__ __forceinline__ OpSteps mn_steps(uint32_t tile, uint32_t rows) {
+  return OpSteps{umma_desc(tile, rows * 32u, 256u, kLayoutSW32b), (uint64_t)(512u >> 4)};
 }
 
 __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) { tmem_ld16(taddr, v); }
@@ -971,10 +981,10 @@ __global__ void __launch_bounds__(kTcChunkNT, 1) gla_bwd_tc_chunk(const BwdArgs<
   // ---- A = dO V^T, P = Q~ K^^T
   if (threadIdx.x == 0) {
     const uint32_t idS = idesc_bf16_f32(MC, MC, false, false);
-    for (int kk = 0; kk < (int)Np / 16; ++kk)
-      umma_ss(tbase + cA, dkm(sb + L.oO, MC, kk), dkm(sb + L.oV, MC, kk), idS, kk > 0 ? 1u : 0u);
-    for (int kk = 0; kk < (int)Kp / 16; ++kk)
-      umma_ss(tbase + cP, dkm(sb + L.oQ, MC, kk), dkm(sb + L.oK, MC, kk), idS, kk > 0 ? 1u : 0u);
+    const OpSteps kO = km_steps(sb + L.oO, MC), kV = km_steps(sb + L.oV, MC);
+    const OpSteps kQ = km_steps(sb + L.oQ, MC), kK = km_steps(sb + L.oK, MC);
+    for (int kk = 0; kk < (int)Np / 16; ++kk) umma_ss(tbase + cA, kO.at(kk), kV.at(kk), idS, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < (int)Kp / 16; ++kk) umma_ss(tbase + cP, kQ.at(kk), kK.at(kk), idS, kk > 0 ? 1u : 0u);
     umma_commit(bar);
   }
   ok = __syncthreads_and(mbar_wait(bar, 0u));
@@ -1027,18 +1037,16 @@ __global__ void __launch_bounds__(kTcChunkNT, 1) gla_bwd_tc_chunk(const BwdArgs<
     const uint32_t idMM = idesc_bf16_f32(MC, (int)Kp, true, true);    // both MN-major
     const uint32_t idVM = idesc_bf16_f32(MC, (int)Np, true, true);
     const uint32_t idVK = idesc_bf16_f32(MC, (int)Np, false, true);   // A K-major, B MN-major
-    for (int kk = 0; kk < (int)Np / 16; ++kk)
-      umma_ss(tbase + cDQ, dkm(sb + L.oO, MC, kk), dkm(sb + L.oG, Kp, kk), idKK, kk > 0 ? 1u : 0u);
-    for (int kk = 0; kk < MC / 16; ++kk)
-      umma_ss(tbase + cDQ, dkm(sb + L.oA, MC, kk), dmn(sb + L.oK, MC, kk), idKM, 1u);
-    for (int kk = 0; kk < MC / 16; ++kk)
-      umma_ss(tbase + cDK, dmn(sb + L.oA, MC, kk), dmn(sb + L.oQ, MC, kk), idMM, kk > 0 ? 1u : 0u);
-    for (int kk = 0; kk < (int)Np / 16; ++kk)
-      umma_ss(tbase + cDK, dkm(sb + L.oV, MC, kk), dkm(sb + L.oD, Kp, kk), idKK, 1u);
-    for (int kk = 0; kk < MC / 16; ++kk)
-      umma_ss(tbase + cDV, dmn(sb + L.oP, MC, kk), dmn(sb + L.oO, MC, kk), idVM, kk > 0 ? 1u : 0u);
-    for (int kk = 0; kk < (int)Kp / 16; ++kk)
-      umma_ss(tbase + cDV, dkm(sb + L.oK, MC, kk), dmn(sb + L.oD, Kp, kk), idVK, 1u);
+    const OpSteps kO = km_steps(sb + L.oO, MC), kG = km_steps(sb + L.oG, Kp), kA = km_steps(sb + L.oA, MC);
+    const OpSteps mK = mn_steps(sb + L.oK, MC), mA = mn_steps(sb + L.oA, MC), mQ = mn_steps(sb + L.oQ, MC);
+    const OpSteps kV = km_steps(sb + L.oV, MC), kD = km_steps(sb + L.oD, Kp), mP = mn_steps(sb + L.oP, MC);
+    const OpSteps mO = mn_steps(sb + L.oO, MC), kK = km_steps(sb + L.oK, MC), mD = mn_steps(sb + L.oD, Kp);
+    for (int kk = 0; kk < (int)Np / 16; ++kk) umma_ss(tbase + cDQ, kO.at(kk), kG.at(kk), idKK, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < MC / 16; ++kk) umma_ss(tbase + cDQ, kA.at(kk), mK.at(kk), idKM, 1u);
+    for (int kk = 0; kk < MC / 16; ++kk) umma_ss(tbase + cDK, mA.at(kk), mQ.at(kk), idMM, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < (int)Np / 16; ++kk) umma_ss(tbase + cDK, kV.at(kk), kD.at(kk), idKK, 1u);
+    for (int kk = 0; kk < MC / 16; ++kk) umma_ss(tbase + cDV, mP.at(kk), mO.at(kk), idVM, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < (int)Kp / 16; ++kk) umma_ss(tbase + cDV, kK.at(kk), mD.at(kk), idVK, 1u);
     umma_commit(bar);
   }
   if (ok) {
@@ -1294,10 +1302,10 @@ __global__ void __launch_bounds__(NT, 2) gla_bwd_tc_local(const BwdArgs<__nv_bfl
   const uint32_t bar = smem_u32(sBar);
   if (threadIdx.x == 0) {
     const uint32_t id = idesc_bf16_f32(MC, (int)Np, true, true);
-    for (int kk = 0; kk < MC / 16; ++kk)
-      umma_ss(tbase, dmn(sb + L.oK, MC, kk), dmn(sb + L.oV, MC, kk), id, kk > 0 ? 1u : 0u);
-    for (int kk = 0; kk < MC / 16; ++kk)
-      umma_ss(tbase + 128, dmn(sb + L.oQ, MC, kk), dmn(sb + L.oO, MC, kk), id, kk > 0 ? 1u : 0u);
+    const OpSteps mK = mn_steps(sb + L.oK, MC), mV = mn_steps(sb + L.oV, MC);
+    const OpSteps mQ = mn_steps(sb + L.oQ, MC), mO = mn_steps(sb + L.oO, MC);
+    for (int kk = 0; kk < MC / 16; ++kk) umma_ss(tbase, mK.at(kk), mV.at(kk), id, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < MC / 16; ++kk) umma_ss(tbase + 128, mQ.at(kk), mO.at(kk), id, kk > 0 ? 1u : 0u);
     umma_commit(bar);
   }
   const bool ok = __syncthreads_and(mbar_wait(bar, 0u));
