@@ -450,6 +450,22 @@ def run_gpu(args):
     return 0
 
 
+def device_us(fn, stream, reps):
+    """Median device time in microseconds of one of `reps` back-to-back calls of fn.
+    The stream first spins on the GPU (about 1 ms) while the host enqueues every call,
+    so the calls run back to back and the host's own work per call (argument checks,
+    the binding, the launches) falls between no pair of events."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    torch.cuda.synchronize()
+    torch.cuda._sleep(2_000_000)
+    evs[0].record(stream)
+    for i in range(reps):
+        fn()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(reps))
+
+
 def other_configs(dig, dev, stream, hbm, reps=10):
     """GLA forward alone on the other bf16 configurations (median of `reps` calls per
     scan direction, event-timed, inputs resident in HBM; c2 and c3 fit in L2, so their
@@ -465,15 +481,7 @@ def other_configs(dig, dev, stream, hbm, reps=10):
         for d in range(4):
             for _ in range(3):
                 dig.gla_fwd(q, k, v, la, cw.Hgrid, cw.Wgrid, d, out=out)
-            ts = []
-            for _ in range(reps):
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                dig.gla_fwd(q, k, v, la, cw.Hgrid, cw.Wgrid, d, out=out)
-                e1.record(stream)
-                torch.cuda.synchronize(dev)
-                ts.append(e0.elapsed_time(e1) * 1e3)
-            per_dir.append(statistics.median(ts))
+            per_dir.append(device_us(lambda: dig.gla_fwd(q, k, v, la, cw.Hgrid, cw.Wgrid, d, out=out), stream, reps))
         us = statistics.mean(per_dir)
         res[name] = {"workload": cw.name, "us_per_dir": per_dir, "bytes": nbytes,
                      "tokens_heads_per_s": cw.token_heads / (us / 1e6),
@@ -609,15 +617,7 @@ def bwd_configs(dig, dev, stream, hbm, reps=5):
         per_dir = []
         for d in range(4):
             dig.gla_bwd(q, k, v, la, do, cw.Hgrid, cw.Wgrid, d)
-            ts = []
-            for _ in range(reps):
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                dig.gla_bwd(q, k, v, la, do, cw.Hgrid, cw.Wgrid, d)
-                e1.record(stream)
-                torch.cuda.synchronize(dev)
-                ts.append(e0.elapsed_time(e1) * 1e3)
-            per_dir.append(statistics.median(ts))
+            per_dir.append(device_us(lambda: dig.gla_bwd(q, k, v, la, do, cw.Hgrid, cw.Wgrid, d), stream, reps))
         us = statistics.mean(per_dir)
         if name == "c2":
             import oracle
@@ -647,15 +647,7 @@ def zigzag_c4(dig, dev, stream, dev_in, outs, hbm, reps=5):
     per = []
     for j in range(8):
         dig.gla_fwd(q, k, v, la, w.Hgrid, w.Wgrid, 4 + j, out=outs[0])
-        ts = []
-        for _ in range(reps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            dig.gla_fwd(q, k, v, la, w.Hgrid, w.Wgrid, 4 + j, out=outs[0])
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            ts.append(e0.elapsed_time(e1) * 1e3)
-        per.append(statistics.median(ts))
+        per.append(device_us(lambda: dig.gla_fwd(q, k, v, la, w.Hgrid, w.Wgrid, 4 + j, out=outs[0]), stream, reps))
     status = dig.device_status()
     if status != 0:
         raise RuntimeError(f"device status after the zigzag orders: {dig.status_string(status)}")
@@ -683,15 +675,7 @@ def norm_configs(dig, dev, stream, hbm, reps=5):
         per_dir = []
         for d in range(4):
             dig.gla_norm_fwd(q, k, v, cw.Hgrid, cw.Wgrid, d)
-            ts = []
-            for _ in range(reps):
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                dig.gla_norm_fwd(q, k, v, cw.Hgrid, cw.Wgrid, d)
-                e1.record(stream)
-                torch.cuda.synchronize(dev)
-                ts.append(e0.elapsed_time(e1) * 1e3)
-            per_dir.append(statistics.median(ts))
+            per_dir.append(device_us(lambda: dig.gla_norm_fwd(q, k, v, cw.Hgrid, cw.Wgrid, d), stream, reps))
         us = statistics.mean(per_dir)
         if name == "c2":
             import oracle
@@ -722,15 +706,7 @@ def glogit_c4(dig, dev, stream, hbm, reps=10):
     for d in range(4):
         for _ in range(2):
             dig.gla_fwd_glogit(q, k, v, g, w.Hgrid, w.Wgrid, d, out=out)
-        ts = []
-        for _ in range(reps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            dig.gla_fwd_glogit(q, k, v, g, w.Hgrid, w.Wgrid, d, out=out)
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            ts.append(e0.elapsed_time(e1) * 1e3)
-        per_dir.append(statistics.median(ts))
+        per_dir.append(device_us(lambda: dig.gla_fwd_glogit(q, k, v, g, w.Hgrid, w.Wgrid, d, out=out), stream, reps))
     status = dig.device_status()
     if status != 0:
         raise RuntimeError(f"device status after the gate-logit forward: {dig.status_string(status)}")
