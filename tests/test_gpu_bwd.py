@@ -110,6 +110,17 @@ def test_bwd_wide_heads(dig, dims):
         run_case(dig, workloads.custom(1, 2, 7, 11, dk, dv, "bf16"), direction, seed=5)
 
 
+@pytest.mark.parametrize("dims", [(8, 8), (16, 80), (80, 16), (48, 72), (80, 80)])
+def test_bwd_tensor_core_head_shapes(dig, dims):
+    """bf16 heads of at most 80 channels take the tensor-core kernels: the smallest
+    head, dk != dv both ways, and the widest (80 x 80, where only S_in and D are staged
+    with the tiles and the end-of-chunk carry reads S_out from global memory); a 9x23
+    grid gives one full 128-row chunk and a ragged one."""
+    dk, dv = dims
+    for direction in (0, 3):
+        run_case(dig, workloads.custom(1, 2, 9, 23, dk, dv, "bf16"), direction, seed=21)
+
+
 def test_bwd_tiny_and_single_token(dig):
     for Hg, Wg in [(1, 1), (1, 5), (3, 2)]:
         for direction in range(4):
