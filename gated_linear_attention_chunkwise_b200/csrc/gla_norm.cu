@@ -21,11 +21,6 @@ namespace dig {
 
 namespace {
 
-__device__ __forceinline__ float ld(const float* p) { return *p; }
-__device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }
-__device__ __forceinline__ void st(float* p, float x) { *p = x; }
-__device__ __forceinline__ void st(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
-
 // elu(x) + 1: x + 1 above zero, e^x at or below.
 __device__ __forceinline__ float feature(float x) { return x > 0.f ? x + 1.f : expf(x); }
 
@@ -34,33 +29,80 @@ __device__ __forceinline__ float log_sigmoid(float x) {
   return x >= 0.f ? -log1pf(expf(-x)) : x - log1pf(expf(x));
 }
 
+// Four consecutive elements (dk, dv and the extended width are multiples of 8, so a
+// group of four never crosses a row and is 16-byte aligned in fp32).
+__device__ __forceinline__ void ld4(const float* p, float (&x)[4]) {
+  const float4 t = *reinterpret_cast<const float4*>(p);
+  x[0] = t.x;
+  x[1] = t.y;
+  x[2] = t.z;
+  x[3] = t.w;
+}
+__device__ __forceinline__ void ld4(const __nv_bfloat16* p, float (&x)[4]) {
+  const uint2 t = *reinterpret_cast<const uint2*>(p);
+  const float2 a = unpack_bf16x2(t.x), b = unpack_bf16x2(t.y);
+  x[0] = a.x;
+  x[1] = a.y;
+  x[2] = b.x;
+  x[3] = b.y;
+}
+__device__ __forceinline__ void st4(float* p, const float (&x)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+}
+__device__ __forceinline__ void st4(__nv_bfloat16* p, const float (&x)[4]) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
+}
+
+// One warp per (token, head) row, four columns per lane.
 template <typename TI>
 __global__ void __launch_bounds__(256) gla_norm_prep(const TI* __restrict__ q, const TI* __restrict__ k,
                                                      const TI* __restrict__ v, float* __restrict__ fq,
                                                      float* __restrict__ fk, float* __restrict__ la,
                                                      float* __restrict__ va, int64_t rows, int dk, int dv, int dva) {
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < rows * dk; e += stride) {
-    const float x = ld(q + e), y = ld(k + e);
-    fq[e] = feature(x);
-    fk[e] = feature(y);
-    la[e] = log_sigmoid(x * y);
-  }
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < rows * dva; e += stride) {
-    const int64_t r = e / dva;
-    const int j = (int)(e - r * dva);
-    va[e] = j < dv ? ld(v + r * dv + j) : (j == dv ? 1.f : 0.f);
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows; r += warps) {
+    for (int c = 4 * lane; c < dk; c += 128) {
+      const int64_t e = r * dk + c;
+      float x[4], y[4], a[4], b[4], l[4];
+      ld4(q + e, x);
+      ld4(k + e, y);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        a[m] = feature(x[m]);
+        b[m] = feature(y[m]);
+        l[m] = log_sigmoid(x[m] * y[m]);
+      }
+      st4(fq + e, a);
+      st4(fk + e, b);
+      st4(la + e, l);
+    }
+    for (int c = 4 * lane; c < dva; c += 128) {
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
+      if (c < dv)
+        ld4(v + r * dv + c, x);
+      else if (c == dv)
+        x[0] = 1.f;
+      st4(va + r * dva + c, x);
+    }
   }
 }
 
+// One warp per row: out = numerator / max(denominator, eps), four columns per lane.
 template <typename TI>
 __global__ void __launch_bounds__(256) gla_norm_post(const float* __restrict__ oa, TI* __restrict__ out,
                                                      int64_t rows, int dv, int dva, float eps) {
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < rows * dv; e += stride) {
-    const int64_t r = e / dv;
-    const int j = (int)(e - r * dv);
-    st(out + e, oa[r * dva + j] / fmaxf(oa[r * dva + dv], eps));
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows; r += warps) {
+    const float den = fmaxf(oa[r * dva + dv], eps);
+    for (int c = 4 * lane; c < dv; c += 128) {
+      float x[4];
+      ld4(oa + r * dva + c, x);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) x[m] = x[m] / den;
+      st4(out + r * dv + c, x);
+    }
   }
 }
 
@@ -76,7 +118,7 @@ int grid_for(int64_t n) {
 
 cudaError_t gla_norm_prep_launch(const void* q, const void* k, const void* v, float* fq, float* fk, float* la,
                                  float* va, int64_t rows, int dk, int dv, int dva, int bf16, cudaStream_t s) {
-  const int grid = grid_for(rows * (dk > dva ? dk : dva));
+  const int grid = grid_for(rows * 32);
   if (bf16)
     gla_norm_prep<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q),
                                                        static_cast<const __nv_bfloat16*>(k),
@@ -90,7 +132,7 @@ cudaError_t gla_norm_prep_launch(const void* q, const void* k, const void* v, fl
 
 cudaError_t gla_norm_post_launch(const float* oa, void* out, int64_t rows, int dv, int dva, float eps, int bf16,
                                  cudaStream_t s) {
-  const int grid = grid_for(rows * dv);
+  const int grid = grid_for(rows * 32);
   if (bf16)
     gla_norm_post<__nv_bfloat16><<<grid, 256, 0, s>>>(oa, static_cast<__nv_bfloat16*>(out), rows, dv, dva, eps);
   else
