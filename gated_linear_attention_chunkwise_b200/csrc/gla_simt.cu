@@ -188,8 +188,11 @@ __global__ void __launch_bounds__(NT) gla_f32_output(const F32Args a) {
   float* sLA = sK + MC * pk;
   float* sV = sLA + MC * pk;
   float* sG = sV + MC * pv;          // [dv][pitch_of(dk)]: G^T
-  float* sA = sG + a.dv * pk;        // [MC][MC+1]
-  float* sBL = sA + MC * pa;
+  // The score tile [MC][MC+1] reuses the log-gate tile when it fits (dk >= MC): the
+  // gates are dead once Q~ and K^ are formed, which frees a second block per SM.
+  const bool a_in_la = pk >= pa;
+  float* sA = a_in_la ? sLA : sG + a.dv * pk;
+  float* sBL = a_in_la ? sG + a.dv * pk : sA + MC * pa;
 
   const int f0 = chunk_first_base_pos(a.g, c, MC);
   stage_rows(sQ, a.q, a.dk, a.g, f0, b, h, a.H);
@@ -319,7 +322,8 @@ cudaError_t gla_f32_forward(const float* q, const float* k, const float* v, cons
 
   const size_t pk = pitch_of(s.dk), pv = pitch_of(s.dv);
   const size_t smem_state = (MC * pk * 2 + MC * pv + s.dk) * sizeof(float);
-  const size_t smem_out = (MC * pk * 3 + MC * pv + s.dv * pk + MC * (MC + 1) + s.dk) * sizeof(float);
+  const size_t score = pk >= (size_t)MC + 1 ? 0 : (size_t)MC * (MC + 1);  // else in the log-gate tile
+  const size_t smem_out = (MC * pk * 3 + MC * pv + s.dv * pk + score + s.dk) * sizeof(float);
   cudaError_t e;
   e = cudaFuncSetAttribute(gla_f32_chunk_state, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_state);
   if (e != cudaSuccess) return e;
