@@ -161,19 +161,54 @@ __global__ void __launch_bounds__(NT) gla_f32_chunk_state(const F32Args a) {
   if (threadIdx.x == 0) a.flags[cid] = wide;
 }
 
+// Each thread takes four consecutive state elements (i, ..., i+3) of one value column
+// j (dk is a multiple of 8) as float4.  Chunks go in batches of kPrefixBatch held in
+// two register sets: the next batch's loads are in flight while the current one is
+// folded, so the walk is not one memory latency per chunk.
+constexpr int kPrefixBatch = 4;
 __global__ void __launch_bounds__(256) gla_f32_prefix(const F32Args a) {
   const int bh = blockIdx.y;
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= a.dk * a.dv) return;
-  const int j = e / a.dk, i = e - j * a.dk;
-  float S = 0.f;
-  for (int c = 0; c < a.NC; ++c) {
-    const int64_t cid = (int64_t)bh * a.NC + c;
-    const float G = a.gamma[cid * a.dk + i] * S;
-    const float sl = a.s_locT[(cid * a.dv + j) * a.dk + i];
-    a.GT[(cid * a.dv + j) * a.dk + i] = G;
-    if (a.flags[cid]) a.s_locT[(cid * a.dv + j) * a.dk + i] = S;  // exact S_in for pass 3
-    S = G + sl;
+  const int e4 = blockIdx.x * blockDim.x + threadIdx.x;
+  if (4 * e4 >= a.dk * a.dv) return;
+  const int j = 4 * e4 / a.dk, i = 4 * e4 - j * a.dk;
+  const int NC = a.NC;
+  const int64_t c0id = (int64_t)bh * NC;
+  // element (j, i) of chunk c in the [dv][dk] slots, and the chunk's gates at i
+  auto slot = [&](int c) { return ((c0id + c) * a.dv + j) * a.dk + i; };
+  float4 xa[kPrefixBatch], xb[kPrefixBatch], ga[kPrefixBatch], gb[kPrefixBatch];
+  int fa[kPrefixBatch], fb[kPrefixBatch];
+  auto load = [&](int c0, float4 (&x)[kPrefixBatch], float4 (&g)[kPrefixBatch], int (&fl)[kPrefixBatch]) {
+#pragma unroll
+    for (int u = 0; u < kPrefixBatch; ++u) {
+      const int c = c0 + u;
+      const bool in = c < NC;
+      x[u] = in ? *reinterpret_cast<const float4*>(a.s_locT + slot(c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      g[u] = in ? *reinterpret_cast<const float4*>(a.gamma + (c0id + c) * a.dk + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      fl[u] = in ? a.flags[c0id + c] : 0;
+    }
+  };
+  // G = Diag(gamma) S_in is written for every chunk, S_in itself for chunks that pass
+  // 3 evaluates token by token; then S = G + S_loc.
+  auto fold = [&](int c0, const float4 (&x)[kPrefixBatch], const float4 (&g)[kPrefixBatch],
+                  const int (&fl)[kPrefixBatch], float4& S) {
+#pragma unroll
+    for (int u = 0; u < kPrefixBatch; ++u) {
+      const int c = c0 + u;
+      if (c < NC) {
+        const float4 G = make_float4(g[u].x * S.x, g[u].y * S.y, g[u].z * S.z, g[u].w * S.w);
+        *reinterpret_cast<float4*>(a.GT + slot(c)) = G;
+        if (fl[u]) *reinterpret_cast<float4*>(a.s_locT + slot(c)) = S;
+        S = make_float4(G.x + x[u].x, G.y + x[u].y, G.z + x[u].z, G.w + x[u].w);
+      }
+    }
+  };
+  float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
+  load(0, xa, ga, fa);
+  for (int c0 = 0; c0 < NC; c0 += 2 * kPrefixBatch) {
+    load(c0 + kPrefixBatch, xb, gb, fb);
+    fold(c0, xa, ga, fa, S);
+    load(c0 + 2 * kPrefixBatch, xa, ga, fa);
+    fold(c0 + kPrefixBatch, xb, gb, fb, S);
   }
 }
 
@@ -332,7 +367,7 @@ cudaError_t gla_f32_forward(const float* q, const float* k, const float* v, cons
   const dim3 grid(a.NC, s.B * s.H);
   gla_f32_chunk_state<<<grid, NT, smem_state, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  gla_f32_prefix<<<dim3((s.dk * s.dv + 255) / 256, s.B * s.H), 256, 0, st>>>(a);
+  gla_f32_prefix<<<dim3((s.dk * s.dv / 4 + 255) / 256, s.B * s.H), 256, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   gla_f32_output<<<grid, NT, smem_out, st>>>(a);
   return cudaGetLastError();
