@@ -165,11 +165,11 @@ __device__ __forceinline__ void chunk_carry(const float* D, const float* Sout, i
 // the total leave the fp32-safe range (evaluate token by token), bit 2 if growth
 // gates exceed it (not representable).
 template <int MC>
-__device__ __forceinline__ int suffix_sums(float* sU, float* sTot, int dk, int reverse, int pw_ = 0) {
+__device__ __forceinline__ int suffix_sums(float* sU, float* sTot, int dk, int reverse) {
   const int i = threadIdx.x;
   int code = 0;
   if (i < dk) {
-    const int pw = pw_ ? pw_ : pitch_of(dk);
+    const int pw = pitch_of(dk);
     float acc = 0.f, lo = 0.f, hi = 0.f;
     for (int s = 0; s < MC; ++s) {
       const int r = reverse ? s : (MC - 1 - s);
